@@ -1,0 +1,323 @@
+/*
+ * bitlinear_oracle.c -- plain, slow CPU oracle for the BitLinear W1.58A8 forward
+ * of BitNet b1.58.
+ *
+ * TEST INFRASTRUCTURE. Only the test suite, the smoke check and the benchmark's
+ * CPU-baseline leg load this file's library. The product path (the CUDA
+ * library) neither includes, links nor calls anything here, and this file
+ * includes nothing from the product. Each function is the step of the method
+ * written out as naive loops, in the order the method defines it, with no
+ * blocking, fusion or reordering.
+ *
+ * Sources (pages on BitNet b1.58 2B4T; each function cites the passage it follows):
+ *   [card]  "BitNet b1.58 2B4T Technical Report" paper card (ai-papers.xuzou.cn),
+ *           sections "Method Adaptation", "Compute Setup", "Bottleneck".
+ *   [news]  fishai news digest of the 2B4T report (news.fishai.com.cn/news/3455510),
+ *           the list of what a BitLinear layer contains.
+ *   [dig]   dignews article on the 2B4T release (dignews.cc), section 2
+ *           "core innovations of the architecture".
+ *   [wiki]  wikiprompt "1.58-bit large language model", introduction.
+ *
+ * Readings where the pages are silent (every one is listed with its reason in the
+ * design notes of the repository):
+ *   - gamma is one scalar per weight tensor: gamma = mean |W|, summed in fp64 in
+ *     row-major order, divided in fp64 by N*K and rounded once to fp32.
+ *   - Wq = clip(rint(W / (gamma + 1e-5f)), -1, 1); the division is one IEEE fp32
+ *     division and rint rounds half to even.
+ *   - s = 127 / max(max_k |x|, 1e-5f) per token (IEEE fp32 division);
+ *     xq = clip(rint(x * s), -128, 127) with x * s one fp32 multiply.
+ *   - packed byte j of row n holds weights k = 4j..4j+3; weight 4j+i sits in bits
+ *     2i..2i+1 as the code q + 1 (0, 1, 2); code 3 is invalid.
+ *   - y = bf16_rn(float(acc) * (gamma / s)), optionally
+ *     y = bf16_rn(float(residual) + float(acc) * (gamma / s)).
+ *   - FFN: g, u dequantised in fp32 (not rounded to bf16); h = (max(g,0)^2) * u;
+ *     subln RMSNorm with unit weight: r = 1 / sqrtf(float(sum_j h_j^2 / f) + 1e-5f)
+ *     with the sum in fp64; hn = h * r; hn re-quantised per token like x; down
+ *     projection dequantised and added to the bf16 residual.
+ *
+ * Build: gcc -O2 -std=c11 -ffp-contract=off -fno-fast-math -fopenmp -shared -fPIC.
+ * -ffp-contract=off keeps every multiply and add a separately rounded IEEE
+ * operation, which is what the readings above specify.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORC_W_EPS 1e-5f   /* eps in W / (gamma + eps) */
+#define ORC_X_EPS 1e-5f   /* floor on the per-token absmax */
+#define ORC_QB 127.0f     /* int8 activation range: codes in [-128, 127], scale to 127 */
+#define ORC_RMS_EPS 1e-5f /* subln RMSNorm eps */
+
+/* ------------------------------------------------------------------------- */
+/* bf16 <-> fp32. bf16 is the upper half of an fp32 word; widening is exact and
+ * narrowing rounds to nearest, ties to even, keeping NaN a NaN.              */
+float orc_bf16_to_f32(uint16_t h) {
+    uint32_t u = (uint32_t)h << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return f;
+}
+
+uint16_t orc_f32_to_bf16(float f) {
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    if ((u & 0x7fffffffu) > 0x7f800000u) return (uint16_t)((u >> 16) | 0x0040u);
+    uint32_t keep = u >> 16;
+    uint32_t rest = u & 0xffffu;
+    if (rest > 0x8000u || (rest == 0x8000u && (keep & 1u))) keep += 1u;
+    return (uint16_t)keep;
+}
+
+void orc_bf16_to_f32_array(const uint16_t* h, int64_t n, float* out) {
+    for (int64_t i = 0; i < n; ++i) out[i] = orc_bf16_to_f32(h[i]);
+}
+
+void orc_f32_to_bf16_array(const float* f, int64_t n, uint16_t* out) {
+    for (int64_t i = 0; i < n; ++i) out[i] = orc_f32_to_bf16(f[i]);
+}
+
+/* ------------------------------------------------------------------------- */
+/* absmean weight quantisation, [card] "Method Adaptation" (weights quantised to
+ * the ternary values {-1, 0, +1} with absmean quantisation in the forward pass),
+ * [news] BitLinear list (weight quantisation), [dig] section 2.
+ * gamma = mean |W| over the whole tensor.                                      */
+float orc_absmean(const float* W, int64_t n) {
+    double s = 0.0;
+    for (int64_t i = 0; i < n; ++i) s += fabs((double)W[i]);
+    return (float)(s / (double)n);
+}
+
+/* Wq = clip(rint(W / (gamma + eps)), -1, 1). */
+void orc_ternarize(const float* W, int64_t n, float gamma, int8_t* q) {
+    float d = gamma + ORC_W_EPS;
+    for (int64_t i = 0; i < n; ++i) {
+        float r = rintf(W[i] / d);
+        if (r > 1.0f) r = 1.0f;
+        if (r < -1.0f) r = -1.0f;
+        q[i] = (int8_t)r;
+    }
+}
+
+/* ------------------------------------------------------------------------- */
+/* Packing: four ternary weights in one 8-bit value stored in HBM, [card]
+ * "Method Adaptation" (pack-store-load-unpack-compute), [dig] section 2.
+ * q is [N, K] row-major, Wp is [N, K/4] row-major, K % 4 == 0.                 */
+void orc_pack(const int8_t* q, int64_t N, int64_t K, uint8_t* Wp) {
+    int64_t KB = K / 4;
+    for (int64_t n = 0; n < N; ++n) {
+        for (int64_t j = 0; j < KB; ++j) {
+            unsigned b = 0;
+            for (int i = 0; i < 4; ++i) {
+                unsigned code = (unsigned)(q[n * K + 4 * j + i] + 1);
+                b |= code << (2 * i);
+            }
+            Wp[n * KB + j] = (uint8_t)b;
+        }
+    }
+}
+
+/* Inverse of orc_pack. Returns the number of invalid (== 3) codes; an invalid
+ * code decodes to 0 so that the output is defined.                            */
+int64_t orc_unpack(const uint8_t* Wp, int64_t N, int64_t K, int8_t* q) {
+    int64_t KB = K / 4, bad = 0;
+    for (int64_t n = 0; n < N; ++n) {
+        for (int64_t k = 0; k < K; ++k) {
+            unsigned code = ((unsigned)Wp[n * KB + k / 4] >> (2 * (k % 4))) & 3u;
+            if (code == 3u) {
+                ++bad;
+                q[n * K + k] = 0;
+            } else {
+                q[n * K + k] = (int8_t)((int)code - 1);
+            }
+        }
+    }
+    return bad;
+}
+
+/* Whole weight path: gamma, ternarise, pack. Wq scratch is allocated here. */
+int orc_pack_weights(const float* W, int64_t N, int64_t K, uint8_t* Wp, float* gamma_out) {
+    int8_t* q = (int8_t*)malloc((size_t)(N * K));
+    if (!q) return -1;
+    float gamma = orc_absmean(W, N * K);
+    orc_ternarize(W, N * K, gamma, q);
+    orc_pack(q, N, K, Wp);
+    free(q);
+    *gamma_out = gamma;
+    return 0;
+}
+
+/* ------------------------------------------------------------------------- */
+/* absmax per-token activation quantisation to int8, [card] "Method Adaptation"
+ * (activations quantised per token with absmax to 8-bit integers), [news]
+ * BitLinear list (activation quantisation). x is [M, K] fp32 (bf16 widened).  */
+void orc_quant_act(const float* x, int64_t M, int64_t K, int8_t* xq, float* s, int32_t* xsum) {
+    for (int64_t m = 0; m < M; ++m) {
+        const float* xr = x + m * K;
+        float amax = 0.0f;
+        for (int64_t k = 0; k < K; ++k) {
+            float a = fabsf(xr[k]);
+            if (a > amax) amax = a;
+        }
+        float sm = ORC_QB / fmaxf(amax, ORC_X_EPS);
+        int32_t sum = 0;
+        for (int64_t k = 0; k < K; ++k) {
+            float r = rintf(xr[k] * sm);
+            if (r > 127.0f) r = 127.0f;
+            if (r < -128.0f) r = -128.0f;
+            xq[m * K + k] = (int8_t)r;
+            sum += (int32_t)r;
+        }
+        s[m] = sm;
+        if (xsum) xsum[m] = sum;
+    }
+}
+
+/* ------------------------------------------------------------------------- */
+/* The integer contraction acc[m, n] = sum_k Wq[n, k] * xq[m, k], [card]
+ * "Method Adaptation" (the unpacked weights multiplied with the int8
+ * activations). Exact in int64, stored as int32 (|acc| <= 127 * K < 2^31).   */
+void orc_int_gemm(const int8_t* q, const int8_t* xq, int64_t M, int64_t N, int64_t K, int32_t* acc) {
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int64_t m = 0; m < M; ++m) {
+        for (int64_t n = 0; n < N; ++n) {
+            int64_t a = 0;
+            for (int64_t k = 0; k < K; ++k) a += (int64_t)q[n * K + k] * (int64_t)xq[m * K + k];
+            acc[m * N + n] = (int32_t)a;
+        }
+    }
+}
+
+/* Same contraction reading the packed bytes directly (decode per element). */
+void orc_int_gemm_packed(const uint8_t* Wp, const int8_t* xq, int64_t M, int64_t N, int64_t K, int32_t* acc) {
+    int64_t KB = K / 4;
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int64_t m = 0; m < M; ++m) {
+        for (int64_t n = 0; n < N; ++n) {
+            int64_t a = 0;
+            for (int64_t k = 0; k < K; ++k) {
+                int code = (int)(((unsigned)Wp[n * KB + k / 4] >> (2 * (k % 4))) & 3u);
+                a += (int64_t)(code - 1) * (int64_t)xq[m * K + k];
+            }
+            acc[m * N + n] = (int32_t)a;
+        }
+    }
+}
+
+/* ------------------------------------------------------------------------- */
+/* Dequantisation y = acc * gamma / s (reading: gamma / s as one fp32 division,
+ * then one fp32 multiply), optional bf16 residual added in fp32, bf16 output. */
+void orc_dequant(const int32_t* acc, float gamma, const float* s, int64_t M, int64_t N,
+                 const uint16_t* residual, uint16_t* y, float* y32) {
+    for (int64_t m = 0; m < M; ++m) {
+        float deq = gamma / s[m];
+        for (int64_t n = 0; n < N; ++n) {
+            float v = (float)acc[m * N + n] * deq;
+            if (residual) v = orc_bf16_to_f32(residual[m * N + n]) + v;
+            if (y32) y32[m * N + n] = v;
+            y[m * N + n] = orc_f32_to_bf16(v);
+        }
+    }
+}
+
+/* ------------------------------------------------------------------------- */
+/* One BitLinear forward, [dig] section 2 (nn.Linear replaced by BitLinear),
+ * [card] "Method Adaptation": quantise x per token, contract with the packed
+ * ternary weights, dequantise to bf16. No bias ([news], [card]: no bias terms).
+ * x, residual and y are bf16 bit patterns. Optional outputs may be NULL.      */
+int orc_forward(const uint8_t* Wp, float gamma, int64_t N, int64_t K,
+                const uint16_t* x, int64_t M, const uint16_t* residual,
+                uint16_t* y, int32_t* acc_out, int8_t* xq_out, float* s_out, int32_t* xsum_out) {
+    float* xf = (float*)malloc(sizeof(float) * (size_t)(M * K));
+    int8_t* xq = (int8_t*)malloc((size_t)(M * K));
+    float* s = (float*)malloc(sizeof(float) * (size_t)M);
+    int32_t* xsum = (int32_t*)malloc(sizeof(int32_t) * (size_t)M);
+    int32_t* acc = (int32_t*)malloc(sizeof(int32_t) * (size_t)(M * N));
+    if (!xf || !xq || !s || !xsum || !acc) {
+        free(xf); free(xq); free(s); free(xsum); free(acc);
+        return -1;
+    }
+    orc_bf16_to_f32_array(x, M * K, xf);
+    orc_quant_act(xf, M, K, xq, s, xsum);
+    orc_int_gemm_packed(Wp, xq, M, N, K, acc);
+    orc_dequant(acc, gamma, s, M, N, residual, y, NULL);
+    if (acc_out) memcpy(acc_out, acc, sizeof(int32_t) * (size_t)(M * N));
+    if (xq_out) memcpy(xq_out, xq, (size_t)(M * K));
+    if (s_out) memcpy(s_out, s, sizeof(float) * (size_t)M);
+    if (xsum_out) memcpy(xsum_out, xsum, sizeof(int32_t) * (size_t)M);
+    free(xf); free(xq); free(s); free(xsum); free(acc);
+    return 0;
+}
+
+/* ------------------------------------------------------------------------- */
+/* subln RMSNorm with unit weight over one token's f features ([news] BitLinear
+ * list: sub-layer normalisation; [card] "Method Adaptation": subln).
+ * Returns r = 1 / sqrtf(float(sum h^2 / f) + eps); hn = h * r.              */
+float orc_subln_rms(const float* h, int64_t f, float* hn) {
+    double ss = 0.0;
+    for (int64_t j = 0; j < f; ++j) ss += (double)h[j] * (double)h[j];
+    float ms = (float)(ss / (double)f);
+    float r = 1.0f / sqrtf(ms + ORC_RMS_EPS);
+    for (int64_t j = 0; j < f; ++j) hn[j] = h[j] * r;
+    return r;
+}
+
+/* ReLU^2 gating of one element ([news]: ReLU^2 in the FFN sub-layer; [card]
+ * "Method Adaptation": ReLU^2 feed-forward): (max(g, 0))^2 * u, each product
+ * rounded to fp32.                                                          */
+float orc_relu2_gate(float g, float u) {
+    float t = g > 0.0f ? g : 0.0f;
+    return (t * t) * u;
+}
+
+/* One FFN sub-layer on M tokens: d -> f (gate, up) -> f -> d (down).
+ *   xq, s = quant(x); g = deq(Wg . xq); u = deq(Wu . xq); h = relu(g)^2 * u;
+ *   hn = subln(h); q2, s2 = quant(hn); y = bf16(residual + deq(Wd . q2)).
+ * Packed weights: Wg, Wu [f, d/4]; Wd [d, f/4]. x, residual, y: [M, d] bf16.
+ * Optional outputs (NULL to skip): h_out [M, f] fp32, q2_out [M, f] int8,
+ * s2_out [M], r_out [M], accd_out [M, d].                                    */
+int orc_ffn_layer(const uint8_t* Wg, float gg, const uint8_t* Wu, float gu,
+                  const uint8_t* Wd, float gd, int64_t d, int64_t f,
+                  const uint16_t* x, int64_t M, const uint16_t* residual, uint16_t* y,
+                  float* h_out, int8_t* q2_out, float* s2_out, float* r_out, int32_t* accd_out) {
+    float* xf = (float*)malloc(sizeof(float) * (size_t)(M * d));
+    int8_t* xq = (int8_t*)malloc((size_t)(M * d));
+    float* s = (float*)malloc(sizeof(float) * (size_t)M);
+    int32_t* accg = (int32_t*)malloc(sizeof(int32_t) * (size_t)(M * f));
+    int32_t* accu = (int32_t*)malloc(sizeof(int32_t) * (size_t)(M * f));
+    float* h = (float*)malloc(sizeof(float) * (size_t)(M * f));
+    float* hn = (float*)malloc(sizeof(float) * (size_t)(M * f));
+    int8_t* q2 = (int8_t*)malloc((size_t)(M * f));
+    float* s2 = (float*)malloc(sizeof(float) * (size_t)M);
+    int32_t* accd = (int32_t*)malloc(sizeof(int32_t) * (size_t)(M * d));
+    int rc = 0;
+    if (!xf || !xq || !s || !accg || !accu || !h || !hn || !q2 || !s2 || !accd) {
+        rc = -1;
+        goto done;
+    }
+    orc_bf16_to_f32_array(x, M * d, xf);
+    orc_quant_act(xf, M, d, xq, s, NULL);
+    orc_int_gemm_packed(Wg, xq, M, f, d, accg);
+    orc_int_gemm_packed(Wu, xq, M, f, d, accu);
+    for (int64_t m = 0; m < M; ++m) {
+        float deqg = gg / s[m];
+        float dequ = gu / s[m];
+        for (int64_t j = 0; j < f; ++j) {
+            float g = (float)accg[m * f + j] * deqg;
+            float u = (float)accu[m * f + j] * dequ;
+            h[m * f + j] = orc_relu2_gate(g, u);
+        }
+        float r = orc_subln_rms(h + m * f, f, hn + m * f);
+        if (r_out) r_out[m] = r;
+    }
+    orc_quant_act(hn, M, f, q2, s2, NULL);
+    orc_int_gemm_packed(Wd, q2, M, d, f, accd);
+    orc_dequant(accd, gd, s2, M, d, residual, y, NULL);
+    if (h_out) memcpy(h_out, h, sizeof(float) * (size_t)(M * f));
+    if (q2_out) memcpy(q2_out, q2, (size_t)(M * f));
+    if (s2_out) memcpy(s2_out, s2, sizeof(float) * (size_t)M);
+    if (accd_out) memcpy(accd_out, accd, sizeof(int32_t) * (size_t)(M * d));
+done:
+    free(xf); free(xq); free(s); free(accg); free(accu); free(h); free(hn); free(q2); free(s2); free(accd);
+    return rc;
+}

@@ -1,0 +1,307 @@
+"""Pins of the CPU oracle to facts outside itself (CPU only).
+
+Each test checks the oracle against a hand-worked example, a closed form, an
+invariant, a brute force over every case, or a library routine, chosen so that a
+plausible slip (a dropped eps, a wrong bit order, a transposed operand, a wrong
+rounding mode, a dropped ReLU or square) fails at least one of them.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from bitlinear_w1_a8_02_b200 import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def bf16_bits(t: torch.Tensor) -> np.ndarray:
+    return t.contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+# ----------------------------------------------------------------------------- bf16
+
+def test_bf16_rounding_matches_torch():
+    rng = np.random.default_rng(0)
+    vals = np.concatenate([
+        rng.standard_normal(20000).astype(np.float32) * np.float32(3.0),
+        rng.standard_normal(2000).astype(np.float32) * np.float32(1e-30),
+        np.array([0.0, -0.0, np.inf, -np.inf, 3.3895314e38, -3.3895314e38, 1e-45], np.float32),
+    ])
+    # exact ties: low 16 bits == 0x8000, both parities of the kept part
+    ties = (np.arange(1, 2000, dtype=np.uint32) << 16 | 0x8000).view(np.float32)
+    vals = np.concatenate([vals, ties, -ties]).astype(np.float32)
+    ours = oracle.f32_to_bf16(vals)
+    ref = bf16_bits(torch.from_numpy(vals).to(torch.bfloat16))
+    assert np.array_equal(ours, ref)
+    back = oracle.bf16_to_f32(ours)
+    assert np.array_equal(back, torch.from_numpy(ours.view(np.int16)).view(torch.bfloat16).float().numpy())
+
+
+# ----------------------------------------------------------------------------- packing
+
+def test_pack_unpack_all_ternary_quads():
+    quads = np.array(np.meshgrid(*([[-1, 0, 1]] * 4), indexing="ij")).reshape(4, -1).T.astype(np.int8)
+    assert quads.shape == (81, 4)
+    Wp = oracle.pack(quads)
+    q, bad = oracle.unpack(Wp, 4)
+    assert bad == 0
+    assert np.array_equal(q, quads)
+    assert len(set(Wp[:, 0].tolist())) == 81
+
+
+def test_pack_bit_order_and_code_offset():
+    # weight i of a byte sits in bits 2i..2i+1 as code q+1
+    cases = {
+        (0, 0, 0, 0): 0x55, (-1, -1, -1, -1): 0x00, (1, 1, 1, 1): 0xAA,
+        (1, 0, 0, 0): 0x56, (0, 0, 0, 1): 0x95, (-1, 0, 0, 0): 0x54, (0, -1, 0, 0): 0x51,
+    }
+    for quad, byte in cases.items():
+        assert oracle.pack(np.array([quad], np.int8))[0, 0] == byte, quad
+    # second byte of a row holds weights 4..7
+    q = np.zeros((1, 8), np.int8)
+    q[0, 5] = 1
+    assert oracle.pack(q).tolist() == [[0x55, 0x59]]
+
+
+def test_unpack_all_bytes():
+    Wp = np.arange(256, dtype=np.uint8).reshape(256, 1)
+    q, bad = oracle.unpack(Wp, 4)
+    fields = [(b >> (2 * i)) & 3 for b in range(256) for i in range(4)]
+    assert bad == sum(f == 3 for f in fields)
+    valid = [b for b in range(256) if all(((b >> (2 * i)) & 3) != 3 for i in range(4))]
+    assert len(valid) == 81
+    assert set(np.unique(q[valid]).tolist()) == {-1, 0, 1}
+
+
+# ----------------------------------------------------------------------------- worked example
+
+def test_worked_4x4_example():
+    g = json.load(open(os.path.join(GOLDEN, "worked_4x4.json")))
+    W = np.array(g["W"], np.float32)
+    gamma = oracle.absmean(W)
+    assert gamma == np.float32(g["gamma"])
+    q = oracle.ternarize(W, gamma)
+    assert q.tolist() == g["q"]
+    Wp, gamma2 = oracle.pack_weights(W)
+    assert gamma2 == gamma
+    assert Wp[:, 0].tolist() == g["packed"]
+    x = np.array(g["x"], np.float32)
+    xq, s, xs = oracle.quant_act(x)
+    assert xq.tolist() == g["xq"]
+    assert s.tolist() == np.array(g["s"], np.float32).tolist()
+    assert xs.tolist() == g["xsum"]
+    acc = oracle.int_gemm_packed(Wp, xq)
+    assert acc.tolist() == g["acc"]
+    y, y32 = oracle.dequant(acc, gamma, s, want_f32=True)
+    assert y32.tolist() == np.array(g["y32"], np.float32).tolist()
+    assert np.array_equal(y, bf16_bits(torch.tensor(g["y32"], dtype=torch.float32).to(torch.bfloat16)))
+    # the whole forward reaches the same values from bf16 inputs
+    out = oracle.forward(Wp, gamma, bf16_bits(torch.tensor(g["x"]).to(torch.bfloat16)))
+    assert out["acc"].tolist() == g["acc"]
+    assert np.array_equal(out["y"], y)
+
+
+# ----------------------------------------------------------------------------- weights
+
+def test_ternarize_eps_and_half_even():
+    # mean |W| = 1/4 exactly; w0 / gamma = 0.5 + 2^-18 would round to 1 without
+    # the eps, but w0 / (gamma + 1e-5) < 0.5 rounds to 0.
+    W = np.array([[0.125 + 2.0 ** -20, 0.375 - 2.0 ** -20, 0.25, 0.25]], np.float32)
+    gamma = oracle.absmean(W)
+    assert gamma == np.float32(0.25)
+    assert oracle.ternarize(W, gamma).tolist() == [[0, 1, 1, 1]]
+    # exact halves of d round to even: 0.5 d -> 0, -0.5 d -> 0, 1.5 d -> 2 -> clip 1
+    d = np.float32(np.float32(0.25) + np.float32(1e-5))
+    W2 = np.array([0.5 * d, -0.5 * d, 1.5 * d, -1.5 * d, 2.5 * d, 0.0], np.float32)
+    assert np.array_equal(W2 / d, np.array([0.5, -0.5, 1.5, -1.5, 2.5, 0.0], np.float32))
+    assert oracle.ternarize(W2, np.float32(0.25)).tolist() == [0, 0, 1, -1, 1, 0]
+
+
+def test_absmean_closed_forms():
+    assert oracle.absmean(np.full(1000, -0.375, np.float32)) == np.float32(0.375)
+    W = (np.arange(1, 4097, dtype=np.float32) * np.float32(2.0 ** -12)) * np.where(np.arange(4096) % 2, 1, -1)
+    exact = math.fsum(abs(float(v)) for v in W) / W.size
+    assert oracle.absmean(W.astype(np.float32)) == np.float32(exact)
+    # all-zero W: gamma = 0, every code 0
+    Z = np.zeros((3, 8), np.float32)
+    Wp, g = oracle.pack_weights(Z)
+    assert g == 0.0 and np.all(Wp == 0x55)
+
+
+def test_gaussian_ternary_statistics():
+    # For W ~ N(0, sigma^2): gamma -> sigma*sqrt(2/pi), P(q = 0) = P(|Z| < sqrt(2/pi)/2)
+    sigma = synth.SIGMA_2B
+    W = synth.weights(1024, 4096, sigma, seed=7, dtype="fp32").numpy()
+    n = W.size
+    gamma = oracle.absmean(W)
+    g_exp = sigma * math.sqrt(2 / math.pi)
+    assert abs(gamma / g_exp - 1) < 5 * 0.756 / math.sqrt(n)
+    q = oracle.ternarize(W, gamma)
+    p0 = math.erf(math.sqrt(2 / math.pi) / 2 / math.sqrt(2))
+    assert abs(p0 - 0.31006) < 1e-4
+    frac0 = float(np.mean(q == 0))
+    assert abs(frac0 - p0) < 5 * math.sqrt(p0 * (1 - p0) / n) + 1e-4
+    pp = (1 - p0) / 2
+    assert abs(float(np.mean(q == 1)) - pp) < 5 * math.sqrt(pp * (1 - pp) / n) + 1e-4
+
+
+# ----------------------------------------------------------------------------- activations
+
+def test_quant_act_half_even_and_range():
+    # amax = 127 -> s = 1 exactly, so xq = rint(x) with ties to even
+    x = np.array([[127.0, 62.5, 63.5, 2.5, -0.5, 1.5, -2.5, -127.0]], np.float32)
+    xq, s, xs = oracle.quant_act(x)
+    assert s[0] == 1.0
+    assert xq.tolist() == [[127, 62, 64, 2, 0, 2, -2, -127]]
+    assert xs[0] == sum(xq[0].tolist())
+
+
+def test_quant_act_invariants():
+    x = synth.activations(64, 2560, seed=1, outliers=True).float().numpy()
+    x[5] = 0.0
+    xq, s, xs = oracle.quant_act(x)
+    nz = np.abs(x).max(axis=1) > 0
+    assert np.all(np.abs(xq[nz]).max(axis=1) == 127)
+    assert xq.min() >= -127 and xq.max() <= 127
+    assert np.all(xq[5] == 0) and s[5] == np.float32(127.0) / np.float32(1e-5)
+    assert np.array_equal(xs, xq.astype(np.int64).sum(axis=1))
+    # scaling a token by a power of two leaves the codes unchanged
+    for p in (-3, 4):
+        xq2, s2, _ = oracle.quant_act(x * np.float32(2.0 ** p))
+        assert np.array_equal(xq2, xq)
+        assert np.array_equal(s2[nz], s[nz] * np.float32(2.0 ** -p))
+
+
+def test_quant_act_tiny_token_uses_floor():
+    # amax = 1e-6 < 1e-5: s = 127 / 1e-5, so the largest code is 13, not 127
+    x = np.array([[1e-6, -5e-7, 0.0, 2.5e-7]], np.float32)
+    xq, s, _ = oracle.quant_act(x)
+    assert s[0] == np.float32(127.0) / np.float32(1e-5)
+    assert xq.tolist() == [[13, -6, 0, 3]]
+
+
+# ----------------------------------------------------------------------------- contraction
+
+@pytest.mark.parametrize("M,N,K", [(1, 1, 4), (3, 5, 8), (7, 3, 32), (8, 8, 12), (2, 17, 64)])
+def test_int_gemm_matches_numpy(M, N, K):
+    rng = np.random.default_rng(M * 100 + N * 10 + K)
+    q = rng.integers(-1, 2, (N, K)).astype(np.int8)
+    xq = rng.integers(-127, 128, (M, K)).astype(np.int8)
+    ref = xq.astype(np.int64) @ q.astype(np.int64).T
+    acc = oracle.int_gemm(q, xq)
+    assert acc.shape == (M, N)
+    assert np.array_equal(acc, ref)
+    assert np.array_equal(oracle.int_gemm_packed(oracle.pack(q), xq), ref)
+
+
+def test_int_gemm_special_cases():
+    rng = np.random.default_rng(3)
+    xq = rng.integers(-127, 128, (4, 40)).astype(np.int8)
+    rows = xq.astype(np.int64).sum(axis=1)
+    for c, expect in ((1, rows), (-1, -rows), (0, 0 * rows)):
+        q = np.full((6, 40), c, np.int8)
+        acc = oracle.int_gemm_packed(oracle.pack(q), xq)
+        assert np.array_equal(acc, np.repeat(expect[:, None], 6, axis=1))
+    # extreme magnitude: K = 28672 with every code and activation at its limit
+    K = 28672
+    q = np.ones((1, K), np.int8)
+    xq = np.full((1, K), -127, np.int8)
+    assert oracle.int_gemm_packed(oracle.pack(q), xq)[0, 0] == -127 * K
+
+
+# ----------------------------------------------------------------------------- dequant
+
+def test_dequant_exact_and_residual():
+    acc = np.array([[4, -8, 0, 3]], np.int32)
+    s = np.array([2.0], np.float32)
+    y, y32 = oracle.dequant(acc, np.float32(0.5), s, want_f32=True)
+    assert y32.tolist() == [[1.0, -2.0, 0.0, 0.75]]
+    res = bf16_bits(torch.tensor([[1.0, 1.0, -3.0, 256.0]]).to(torch.bfloat16))
+    y, y32 = oracle.dequant(acc, np.float32(0.5), s, residual=res, want_f32=True)
+    assert y32.tolist() == [[2.0, -1.0, -3.0, 256.75]]
+    # bf16 keeps 8 significant bits: 256.75 rounds to 256 (tie-free, nearest)
+    assert oracle.bf16_to_f32(y).tolist() == [[2.0, -1.0, -3.0, 256.0]]
+
+
+# ----------------------------------------------------------------------------- FFN
+
+def test_relu2_gate_values():
+    assert oracle.relu2_gate(2.0, 3.0) == 12.0
+    assert oracle.relu2_gate(-2.0, 3.0) == 0.0
+    assert oracle.relu2_gate(0.5, -4.0) == -1.0
+
+
+def test_subln_rms_closed_form():
+    h = np.array([3.0, -4.0, 0.0, 0.0], np.float32)  # mean h^2 = 6.25
+    r, hn = oracle.subln_rms(h)
+    assert abs(float(r) - 1 / math.sqrt(6.25 + 1e-5)) < 1e-7
+    hb = synth.activations(1, 6912, seed=4, outliers=False).float().numpy()[0] * np.float32(1e-3)
+    r, hn = oracle.subln_rms(hb)
+    ms = float(np.mean(hb.astype(np.float64) ** 2))
+    assert abs(float(r) / (1 / math.sqrt(ms + 1e-5)) - 1) < 1e-6
+    assert abs(float(np.mean(hn.astype(np.float64) ** 2)) - ms / (ms + 1e-5)) < 1e-5
+
+
+def _packed_rows(codes):
+    return oracle.pack(np.array(codes, np.int8))
+
+
+def test_ffn_structured_closed_form():
+    """Gate rows with j+1 leading +1 codes, up and down all +1, constant x.
+
+    g_j = (j+1) * gg * c, u_j = d * gu * c, h_j = ((j+1) gg c)^2 d gu c.
+    hn_j = h_j / sqrt(mean h^2 + eps); q2_j = rint(127 h_j / h_max);
+    y_n = res + gd * sum_j q2_j * hn_max / 127 for every output n.
+    A dropped ReLU, square, mean or eps moves y far outside bf16 rounding.
+    """
+    d, f = 16, 8
+    gg, gu, gd = np.float32(0.5), np.float32(0.25), np.float32(0.125)
+    Wg = _packed_rows([[1] * (j + 1) + [0] * (d - j - 1) for j in range(f)])
+    Wu = _packed_rows([[1] * d for _ in range(f)])
+    Wd = _packed_rows([[1] * f for _ in range(d)])
+    for c, res_val in ((0.0625, 1.0), (0.001, 0.0)):
+        x = bf16_bits(torch.full((1, d), c).to(torch.bfloat16))
+        res = bf16_bits(torch.full((1, d), res_val).to(torch.bfloat16))
+        out = oracle.ffn_layer(Wg, gg, Wu, gu, Wd, gd, x, residual=res)
+        cb = float(torch.tensor(c).to(torch.bfloat16))
+        g = np.array([(j + 1) * gg * cb for j in range(f)], np.float64)
+        u = d * gu * cb
+        h = g ** 2 * u
+        hn = h / math.sqrt(np.mean(h ** 2) + 1e-5)
+        q2 = np.rint(127 * h / h.max())
+        y = res_val + gd * q2.sum() * hn.max() / 127
+        assert np.array_equal(out["q2"][0], q2.astype(np.int8))
+        got = oracle.bf16_to_f32(out["y"])[0]
+        assert np.all(np.abs(got - y) <= 2.0 ** -8 * abs(y) + 1e-30), (got, y)
+
+
+def test_ffn_negative_gate_is_cut():
+    d, f = 8, 8
+    Wg = _packed_rows([[1] * d] * f)
+    Wd = _packed_rows([[1] * f] * d)
+    x = bf16_bits(torch.full((1, d), -0.5).to(torch.bfloat16))
+    res = bf16_bits(torch.full((1, d), 0.75).to(torch.bfloat16))
+    out = oracle.ffn_layer(Wg, 1.0, Wg, 1.0, Wd, 1.0, x, residual=res)
+    assert np.all(out["h"] == 0) and np.all(out["q2"] == 0)
+    assert np.all(oracle.bf16_to_f32(out["y"]) == 0.75)
+
+
+def test_ffn_requant_tracks_unnormalised_codes():
+    # RMSNorm is a positive per-token rescale, so requantising hn gives the codes
+    # of h itself except at rare rounding ties.
+    rng_seed = 11
+    d, f, M = 256, 512, 8
+    W = [synth.weights(f, d, 0.02, rng_seed + i) for i in range(2)] + [synth.weights(d, f, 0.02, rng_seed + 2)]
+    packed = [oracle.pack_weights(bf16_bits(w)) for w in W]
+    x = bf16_bits(synth.activations(M, d, seed=rng_seed, outliers=True))
+    out = oracle.ffn_layer(packed[0][0], packed[0][1], packed[1][0], packed[1][1],
+                           packed[2][0], packed[2][1], x, residual=x)
+    q_direct, _, _ = oracle.quant_act(out["h"])
+    mismatch = np.mean(q_direct != out["q2"])
+    assert mismatch < 1e-3
+    assert np.all(np.abs(q_direct.astype(int) - out["q2"].astype(int)) <= 1)
