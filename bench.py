@@ -1,0 +1,519 @@
+#!/usr/bin/env python
+"""Benchmark of the BitLinear W1.58A8 forward on B200.
+
+Headline (one JSON line on rank 0): decode GEMV throughput in GB/s of packed
+weight bytes. One step is a decode pass over a 2B-shaped model's BitLinear
+projections: 30 layers x the four decode shapes (K=2560 -> N in {2560, 640,
+6912}, K=6912 -> N=2560), one token (M=1), each layer with its own weight copy
+(327 MB of packed weights per step, so every step streams its weights from HBM;
+no L2 flush is needed). Each call quantises the token per absmax, runs the
+ternary GEMV and dequantises to bf16. The step is captured once in a CUDA graph
+and replayed.
+
+Extras on the same line: batched decode (M = 4, 8, 16), prefill int8 TOPS
+(M = 512, 2048, 4096), the 100B-class bandwidth case, the 30-layer FFN chain,
+the roofline of the dominant kernel, the end-to-end number through the public
+API with host buffers, the CPU oracle baseline and the SM clocks.
+
+Multi-GPU: one process per GPU (torchrun); every rank runs the same independent
+decode step on its own weights (weak scaling, no data-path collective); the
+time is the max over ranks.
+
+--impl reference times the CPU oracle (plain C) on a bounded sample of the same
+workload on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "W1.58A8 BitLinear: decode GEMV HBM GB/s (% peak); prefill int8 TOPS (% peak)"
+DECODE_SHAPES = [(2560, 2560), (2560, 640), (2560, 6912), (6912, 2560)]  # (K, N)
+LAYERS = 30
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+INT8_PER_BF16 = 2.0  # nominal dense int8 (= fp8) rate over dense bf16 on B200
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def dist_env():
+    return (int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)),
+            int(os.environ.get("LOCAL_RANK", 0)))
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason sampling during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.file = None
+
+    def start(self):
+        try:
+            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.file, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.file.flush()
+        self.file.seek(0)
+        rows = [ln.strip().split(",") for ln in self.file.read().splitlines() if ln.strip()]
+        self.file.close()
+        os.unlink(self.file.name)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            r = [c.strip() for c in r]
+            if len(r) < 9:
+                continue
+            try:
+                sm.append(float(r[1]))
+                mx = float(r[2])
+            except ValueError:
+                continue
+            for name, v in zip(names, r[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- ours
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import bitlinear_w1_a8_02_b200 as bl
+    from bitlinear_w1_a8_02_b200 import synth
+
+    rank, world, local = dist_env()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    peaks, peak_kind = load_peaks()
+    hbm_peak = float(peaks["hbm_gbs"])
+    int8_peak = float(peaks["bf16_tflops"]) * INT8_PER_BF16
+    int8_peak_sust = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])) * INT8_PER_BF16
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(v: float) -> float:
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    # ---- decode weights: 30 copies of each of the four shapes, packed on device
+    weights = []  # weights[layer][shape] = (Wp, gamma)
+    for layer in range(LAYERS):
+        row = []
+        for si, (K, N) in enumerate(DECODE_SHAPES):
+            W = synth.weights(N, K, synth.SIGMA_2B, synth.weight_seed(si, layer) + 7919 * rank,
+                              device=dev)
+            row.append(bl.pack_weights(W))
+            del W
+        weights.append(row)
+    xs = [synth.activations(1, K, seed=1, outliers=True, device=dev) for K, _ in DECODE_SHAPES]
+    ys = [torch.empty((1, N), dtype=torch.bfloat16, device=dev) for _, N in DECODE_SHAPES]
+    ws = torch.empty(max(bl.workspace_bytes(bl.BL_OP_FORWARD, 16, N, K) for K, N in DECODE_SHAPES),
+                     dtype=torch.uint8, device=dev)
+    step_bytes = LAYERS * sum(K * N // 4 for K, N in DECODE_SHAPES)
+    kernels_per_call = 2  # act-quant + GEMV
+
+    def step():
+        for layer in range(LAYERS):
+            for si in range(len(DECODE_SHAPES)):
+                Wp, g = weights[layer][si]
+                bl.forward(Wp, g, xs[si], out=ys[si], ws=ws)
+
+    torch.cuda.synchronize()
+    stream = torch.cuda.Stream(device=dev)
+    with torch.cuda.stream(stream):
+        step()  # warm the code paths before capture
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        step()
+    torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        graph.replay()
+    torch.cuda.synchronize()
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize()
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    cur = torch.cuda.current_stream(dev)
+    ev0.record(cur)
+    for _ in range(args.steps):
+        graph.replay()
+    ev1.record(cur)
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    ms_total = max_over_ranks(ev0.elapsed_time(ev1))
+    ms_step = ms_total / args.steps
+    value = world * step_bytes * args.steps / (ms_total * 1e-3) / 1e9
+
+    # ---- dominant kernel: per-call device time of the decode forward
+    # (act-quant + GEMV), CUDA events on the launching stream, eager, one step.
+    evs = []
+    torch.cuda.synchronize()
+    for layer in range(LAYERS):
+        for si in range(len(DECODE_SHAPES)):
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            Wp, g = weights[layer][si]
+            a.record(cur)
+            bl.forward(Wp, g, xs[si], out=ys[si], ws=ws)
+            b.record(cur)
+            evs.append((a, b, DECODE_SHAPES[si]))
+    torch.cuda.synchronize()
+    call_ms = sum(a.elapsed_time(b) for a, b, _ in evs)
+    call_bytes = sum(K * N // 4 for _, _, (K, N) in evs)
+    achieved = call_bytes / (call_ms * 1e-3) / 1e9
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
+                "frac": round(achieved / hbm_peak, 4), "traffic": None,
+                "kernel": "act_quant_vec_kernel<PLANES> + gemv_mma_kernel<1> (one forward call)",
+                "peak_kind": peak_kind}
+
+    extras = {}
+    if rank == 0 and not args.no_extras:
+        extras = run_extras(args, bl, synth, dev, hbm_peak, int8_peak)
+
+    # ---- end to end through the public API with host buffers
+    e2e = run_e2e(args, bl, dev, graph, xs, ys, step_bytes, world, barrier, max_over_ranks)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(weights, xs, bl, budget_s=args.cpu_seconds)
+
+    del graph
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
+        "data": "synthetic (seeded N(0,0.02^2) weights, N(0,1) activations with 1% x20 outlier channels)",
+        "config": {"workload": "decode_2b: M=1, (K,N) in {(2560,2560),(2560,640),(2560,6912),(6912,2560)}, "
+                               "30 layer copies each, 120 BitLinear calls per step",
+                   "M": 1, "layers": LAYERS, "calls_per_step": LAYERS * len(DECODE_SHAPES),
+                   "packed_bytes_per_step": step_bytes,
+                   "l2": "inputs larger than L2: 327 MB of packed weights per step vs 126 MB L2",
+                   "launch": "cuda_graph replay of the 120 calls", "parallelism": f"replicas x{world}"},
+        "hbm_frac": round(value / world / hbm_peak, 4),
+        "roofline": roofline,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": args.steps * LAYERS * len(DECODE_SHAPES) * kernels_per_call,
+        "clocks": clk,
+        "peaks": {"hbm_gbs": hbm_peak, "int8_tops_burst": int8_peak, "int8_tops_sustained": int8_peak_sust,
+                  "kind": peak_kind + " (int8 = bf16 x 2, the nominal dense ratio)"},
+        "extras": extras,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def time_graph(torch, fn, reps: int, warm: int = 3):
+    """Capture fn in a CUDA graph; return mean ms per replay (events)."""
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        fn()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        fn()
+    for _ in range(warm):
+        g.replay()
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(reps):
+        g.replay()
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / reps
+    del g
+    return ms
+
+
+def run_extras(args, bl, synth, dev, hbm_peak, int8_peak):
+    import torch
+
+    out = {}
+    # batched decode and prefill at the 2B FFN shapes (3 rotating copies > L2 at M<=16)
+    shapes = [(2560, 6912), (6912, 2560)]
+    packs = {}
+    for si, (K, N) in enumerate(shapes):
+        packs[(K, N)] = [bl.pack_weights(synth.weights(N, K, synth.SIGMA_2B, 50 + 10 * si + c, device=dev))
+                         for c in range(8)]
+    batched = {}
+    for M in (4, 8, 16):
+        per = {}
+        for K, N in shapes:
+            x = synth.activations(M, K, seed=M, device=dev)
+            y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+            ws = torch.empty(bl.workspace_bytes(bl.BL_OP_FORWARD, M, N, K), dtype=torch.uint8, device=dev)
+            cp = packs[(K, N)]
+
+            def fn():
+                for Wp, g in cp:
+                    bl.forward(Wp, g, x, out=y, ws=ws)
+            ms = time_graph(torch, fn, reps=20) / len(cp)
+            per[f"{K}x{N}"] = {"us_per_call": round(ms * 1e3, 2),
+                               "gbs": round(K * N / 4 / (ms * 1e-3) / 1e9, 1)}
+        batched[f"M{M}"] = per
+    out["batched_decode_2b"] = batched
+
+    prefill = {}
+    for M in (512, 2048, 4096):
+        per = {}
+        for K, N in shapes:
+            x = synth.activations(M, K, seed=M, device=dev)
+            y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+            ws = torch.empty(bl.workspace_bytes(bl.BL_OP_FORWARD, M, N, K), dtype=torch.uint8, device=dev)
+            Wp, g = packs[(K, N)][0]
+
+            def fn():
+                bl.forward(Wp, g, x, out=y, ws=ws)
+            ms = time_graph(torch, fn, reps=10)
+            tops = 2.0 * M * N * K / (ms * 1e-3) / 1e12
+            per[f"{K}x{N}"] = {"ms": round(ms, 4), "tops": round(tops, 1),
+                               "frac_int8_peak": round(tops / int8_peak, 4)}
+        prefill[f"M{M}"] = per
+    out["prefill_2b"] = prefill
+    del packs
+
+    # 100B-class bandwidth stress: M = 1 and 16, two copies per shape (235 MB > L2)
+    big = {}
+    for K, N in ((8192, 28672), (28672, 8192)):
+        cps = [bl.pack_weights(synth.weights(N, K, synth.SIGMA_100B, 90 + c, device=dev)) for c in range(2)]
+        torch.cuda.empty_cache()
+        for M in (1, 16):
+            x = synth.activations(M, K, seed=M, device=dev)
+            y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+            ws = torch.empty(bl.workspace_bytes(bl.BL_OP_FORWARD, M, N, K), dtype=torch.uint8, device=dev)
+
+            def fn():
+                for Wp, g in cps:
+                    bl.forward(Wp, g, x, out=y, ws=ws)
+            ms = time_graph(torch, fn, reps=10) / len(cps)
+            gbs = K * N / 4 / (ms * 1e-3) / 1e9
+            big[f"{K}x{N}_M{M}"] = {"us_per_call": round(ms * 1e3, 2), "gbs": round(gbs, 1),
+                                    "hbm_frac": round(gbs / hbm_peak, 4)}
+        del cps
+    out["stress_100b"] = big
+
+    # FFN chain: 30 layers, d=2560, f=6912, residual add
+    d, f = 2560, 6912
+    layers = []
+    for layer in range(LAYERS):
+        sg, su, sd = synth.ffn_layer_seeds(layer)
+        layers.append([bl.pack_weights(synth.weights(N, K, synth.SIGMA_2B, seed, device=dev))
+                       for N, K, seed in ((f, d, sg), (f, d, su), (d, f, sd))])
+    ffn = {}
+    for M in (1, 512):
+        h0 = synth.activations(M, d, seed=1, outliers=False, device=dev)
+        bufs = [torch.empty_like(h0), torch.empty_like(h0)]
+        ws = torch.empty(bl.workspace_bytes(bl.BL_OP_FFN, M, f, d), dtype=torch.uint8, device=dev)
+
+        def fn():
+            h = h0
+            for li, (g_, u_, d_) in enumerate(layers):
+                o = bufs[li % 2]
+                bl.ffn(g_[0], g_[1], u_[0], u_[1], d_[0], d_[1], h, residual=h, out=o, ws=ws)
+                h = o
+        ms = time_graph(torch, fn, reps=5)
+        wbytes = LAYERS * 3 * d * f / 4
+        ent = {"ms_30_layers": round(ms, 4), "packed_gbs": round(wbytes / (ms * 1e-3) / 1e9, 1)}
+        if M > 1:
+            tops = 2.0 * M * 3 * d * f * LAYERS / (ms * 1e-3) / 1e12
+            ent["tops"] = round(tops, 1)
+            ent["frac_int8_peak"] = round(tops / int8_peak, 4)
+        ffn[f"M{M}"] = ent
+    out["ffn_2b_30_layers"] = ffn
+    del layers
+    torch.cuda.empty_cache()
+    return out
+
+
+def run_e2e(args, bl, dev, graph, xs, ys, step_bytes, world, barrier, max_over_ranks):
+    """Each step: pinned host -> device copy of the step's activations, the
+    captured public-API calls, device -> host copy of the step's outputs."""
+    import torch
+
+    h_in = [x.detach().cpu().pin_memory() for x in xs]
+    h_out = [torch.empty(y.shape, dtype=y.dtype).pin_memory() for y in ys]
+    h2d = sum(t.numel() * t.element_size() for t in h_in)
+    d2h = sum(t.numel() * t.element_size() for t in h_out)
+    cur = torch.cuda.current_stream(dev)
+
+    def one():
+        for hx, dx in zip(h_in, xs):
+            dx.copy_(hx, non_blocking=True)
+        graph.replay()
+        for hy, dy in zip(h_out, ys):
+            hy.copy_(dy, non_blocking=True)
+
+    for _ in range(args.warmup):
+        one()
+    torch.cuda.synchronize()
+    barrier()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(cur)
+    for _ in range(args.steps):
+        one()
+    b.record(cur)
+    torch.cuda.synchronize()
+    barrier()
+    ms = max_over_ranks(a.elapsed_time(b))
+    value = world * step_bytes * args.steps / (ms * 1e-3) / 1e9
+    return {"value": round(value, 1), "unit": "GB/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "ms_per_step": round(ms / args.steps, 5)}
+
+
+def cpu_baseline(weights, xs, bl, budget_s: float):
+    """The oracle (as it stands) on a bounded sample of the decode step: whole
+    layers of the four shapes, one after another, until the budget is spent."""
+    import numpy as np
+
+    import oracle
+
+    bits = [x.cpu().view(__import__("torch").int16).numpy().view(np.uint16) for x in xs]
+    host = [[(Wp.cpu().numpy(), float(g.cpu().item())) for Wp, g in row] for row in weights]
+    done_bytes, n_layers = 0, 0
+    t0 = time.perf_counter()
+    for row in host:
+        for (Wp, g), xb in zip(row, bits):
+            oracle.forward(Wp, g, xb)
+            done_bytes += Wp.size
+        n_layers += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    return {"value": round(done_bytes / dt / 1e9, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "sample": f"{n_layers} of 30 layers of the decode step (4 shapes each, M=1), "
+                      f"{done_bytes} packed bytes in {dt:.2f} s"}
+
+
+# ----------------------------------------------------------------------------- reference arm
+
+def run_reference(args):
+    """The CPU oracle on the same workload: each step is a bounded sample (one
+    layer of the four decode shapes, M=1); value in packed GB/s."""
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    import numpy as np
+    import torch
+
+    import oracle
+    from bitlinear_w1_a8_02_b200 import synth
+
+    def bits(t):
+        return t.contiguous().view(torch.int16).numpy().view(np.uint16)
+
+    packed = []
+    for si, (K, N) in enumerate(DECODE_SHAPES):
+        W = synth.weights(N, K, synth.SIGMA_2B, synth.weight_seed(si, 0))
+        packed.append(oracle.pack_weights(bits(W)))
+    xs = [bits(synth.activations(1, K, seed=1, outliers=True)) for K, _ in DECODE_SHAPES]
+    step_bytes = sum(Wp.size for Wp, _ in packed)
+
+    def step():
+        for (Wp, g), x in zip(packed, xs):
+            oracle.forward(Wp, g, x)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = time.perf_counter() - t0
+    value = step_bytes * args.steps / dt / 1e9
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    sample = "one layer of the four decode shapes per step (M=1), of the 30-layer step"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
+        "data": "synthetic",
+        "config": {"workload": "decode_2b: M=1, (K,N) in {(2560,2560),(2560,640),(2560,6912),(6912,2560)}",
+                   "M": 1, "sample": sample},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-extras", action="store_true", help="skip the secondary workloads")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

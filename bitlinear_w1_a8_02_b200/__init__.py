@@ -1,0 +1,11 @@
+"""BitLinear W1.58A8 forward (BitNet b1.58) for B200 (sm_100a).
+
+The computation lives in ``libbitlinear.so`` (hand-written CUDA behind the C ABI
+of ``include/bitlinear.h``); this package is its Python binding plus the seeded
+synthetic input generators in ``synth``.
+"""
+from .binding import (  # noqa: F401
+    BL_BF16, BL_FP32, BL_OK, BL_OP_FFN, BL_OP_FORWARD, BL_OP_PACK, BL_OP_VALIDATE, LIB_PATH,
+    SIGNATURES, STATUS_NAMES, BitLinearError, ffn, forward, get_device_error, lib, pack_weights,
+    quant_act, validate_packed, workspace_bytes,
+)

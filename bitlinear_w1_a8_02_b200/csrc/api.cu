@@ -1,0 +1,267 @@
+// C ABI of the BitLinear W1.58A8 library (declared in include/bitlinear.h).
+//
+// Each entry point validates its arguments on the host, carves its workspace,
+// and launches kernels on the caller's stream. Nothing here allocates device
+// memory, synchronises (except where the header says so) or lets a C++
+// exception escape.
+#include <bitlinear.h>
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+#define BL_API extern "C" __attribute__((visibility("default")))
+
+namespace {
+
+constexpr int64_t kMaxM = 65535;           // tokens per call (grid.y of the per-token kernels)
+constexpr int64_t kMaxK = 262144;          // keeps the field-scaled int32 accumulators exact
+constexpr int64_t kMaxN = int64_t(1) << 24;
+constexpr size_t kWsAlign = 256;
+
+inline size_t align_up(size_t v) { return (v + kWsAlign - 1) / kWsAlign * kWsAlign; }
+inline bool aligned(const void* p, size_t a) { return (uintptr_t)p % a == 0; }
+
+// Workspace carving -----------------------------------------------------------
+struct ForwardWs {
+    size_t xq, scale, xsum, total;
+};
+inline ForwardWs forward_ws(int64_t M, int64_t K) {
+    ForwardWs w;
+    w.xq = 0;
+    w.scale = align_up((size_t)(M * K));
+    w.xsum = w.scale + align_up((size_t)M * 4);
+    w.total = w.xsum + align_up((size_t)M * 4);
+    return w;
+}
+
+struct FfnWs {
+    size_t xq, scale, xsum, g, u, q2, s2, xsum2, total;
+};
+inline FfnWs ffn_ws(int64_t M, int64_t f, int64_t d) {
+    FfnWs w;
+    w.xq = 0;
+    w.scale = align_up((size_t)(M * d));
+    w.xsum = w.scale + align_up((size_t)M * 4);
+    w.g = w.xsum + align_up((size_t)M * 4);
+    w.u = w.g + align_up((size_t)(M * f) * 4);
+    w.q2 = w.u + align_up((size_t)(M * f) * 4);
+    w.s2 = w.q2 + align_up((size_t)(M * f));
+    w.xsum2 = w.s2 + align_up((size_t)M * 4);
+    w.total = w.xsum2 + align_up((size_t)M * 4);
+    return w;
+}
+
+inline size_t pack_ws(int64_t N, int64_t K) {
+    return align_up((size_t)bl::absmean_blocks(N * K) * sizeof(double));
+}
+
+// Device check: the kernels are built for sm_100a only.
+bl_status check_device() {
+    static int cached[64];  // 0 unknown, 1 ok, 2 unsupported
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) {
+        cudaGetLastError();
+        return BL_ERR_UNSUPPORTED;
+    }
+    if (dev < 64 && cached[dev]) return cached[dev] == 1 ? BL_OK : BL_ERR_UNSUPPORTED;
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) {
+        cudaGetLastError();
+        return BL_ERR_UNSUPPORTED;
+    }
+    const bool ok = (major == 10 && minor == 0);
+    if (dev < 64) cached[dev] = ok ? 1 : 2;
+    return ok ? BL_OK : BL_ERR_UNSUPPORTED;
+}
+
+inline bl_status cuda_status(cudaError_t e) { return e == cudaSuccess ? BL_OK : BL_ERR_CUDA; }
+
+#define BL_TRY(expr)                                  \
+    do {                                              \
+        cudaError_t _e = (expr);                      \
+        if (_e != cudaSuccess) return BL_ERR_CUDA;    \
+    } while (0)
+
+bl_status check_ws(const void* ws, size_t ws_bytes, size_t need) {
+    if (need == 0) return BL_OK;
+    if (!ws) return BL_ERR_NULL;
+    if (!aligned(ws, kWsAlign)) return BL_ERR_ALIGN;
+    if (ws_bytes < need) return BL_ERR_WORKSPACE;
+    return BL_OK;
+}
+
+// Whether the streaming GEMV can read these packed weights.
+inline bool gemv_fast(const uint8_t* Wp, int64_t N, int64_t K) {
+    return bl::gemv_fast_ok(N, K) && aligned(Wp, 16);
+}
+
+// One BitLinear projection of already-quantised codes `xq` (layout chosen by
+// the caller through `fast`).
+bl_status project(bool fast, const uint8_t* Wp, const float* gamma, int64_t N, int64_t K,
+                  const int8_t* xq, const float* scale, const int32_t* xsum, int64_t M,
+                  const bl::GemvOut& out, cudaStream_t s) {
+    if (fast) return cuda_status(bl::launch_gemv(Wp, gamma, N, K, xq, scale, xsum, M, out, s));
+    return cuda_status(bl::launch_gemv_generic(Wp, gamma, N, K, xq, scale, M, out, s));
+}
+
+}  // namespace
+
+// ----------------------------------------------------------------------------
+BL_API const char* bitlinear_status_string(bl_status st) {
+    switch (st) {
+        case BL_OK: return "BL_OK";
+        case BL_ERR_NULL: return "BL_ERR_NULL: a required pointer is NULL";
+        case BL_ERR_SHAPE: return "BL_ERR_SHAPE: invalid or unsupported sizes";
+        case BL_ERR_ALIGN: return "BL_ERR_ALIGN: misaligned pointer";
+        case BL_ERR_DTYPE: return "BL_ERR_DTYPE: unknown dtype";
+        case BL_ERR_WORKSPACE: return "BL_ERR_WORKSPACE: workspace too small";
+        case BL_ERR_UNSUPPORTED: return "BL_ERR_UNSUPPORTED: needs an sm_100 (B200) device";
+        case BL_ERR_CUDA: return "BL_ERR_CUDA: a CUDA call or launch failed";
+        case BL_ERR_TIMEOUT: return "BL_ERR_TIMEOUT: a bounded wait in a kernel gave up";
+        case BL_ERR_BAD_CODE: return "BL_ERR_BAD_CODE: packed weights hold the invalid code 3";
+    }
+    return "unknown bl_status";
+}
+
+BL_API size_t bitlinear_workspace_bytes(int op, int64_t M, int64_t N, int64_t K) {
+    if (M < 0 || N < 0 || K < 0) return 0;
+    switch (op) {
+        case BL_OP_PACK: return pack_ws(N, K);
+        case BL_OP_FORWARD: return forward_ws(M, K).total;
+        case BL_OP_FFN: return ffn_ws(M, N, K).total;
+        case BL_OP_VALIDATE: return kWsAlign;
+        default: return 0;
+    }
+}
+
+BL_API bl_status bitlinear_pack_weights(const void* W, int wdt, int64_t N, int64_t K, uint8_t* Wp,
+                                        float* gamma, void* ws, size_t ws_bytes,
+                                        bl_stream_t stream) {
+    if (wdt != BL_BF16 && wdt != BL_FP32) return BL_ERR_DTYPE;
+    if (N < 1 || K < 4 || K % 4 != 0 || N > kMaxN || K > kMaxK) return BL_ERR_SHAPE;
+    if (!W || !Wp || !gamma) return BL_ERR_NULL;
+    if (!aligned(W, 16) || !aligned(gamma, 4)) return BL_ERR_ALIGN;
+    if (bl_status st = check_ws(ws, ws_bytes, pack_ws(N, K))) return st;
+    if (bl_status st = check_device()) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    const bool fp32 = wdt == BL_FP32;
+    BL_TRY(bl::launch_absmean(W, fp32, N * K, (double*)ws, gamma, s));
+    BL_TRY(bl::launch_ternary_pack(W, fp32, N, K, gamma, Wp, s));
+    return BL_OK;
+}
+
+BL_API bl_status bitlinear_quant_act(const uint16_t* x, int64_t M, int64_t K, int8_t* xq,
+                                     float* scale, int32_t* xsum, bl_stream_t stream) {
+    if (M < 0 || M > kMaxM || K < 4 || K % 4 != 0 || K > kMaxK) return BL_ERR_SHAPE;
+    if (M == 0) return BL_OK;
+    if (!x || !xq || !scale) return BL_ERR_NULL;
+    if (!aligned(x, 2) || !aligned(scale, 4) || (xsum && !aligned(xsum, 4))) return BL_ERR_ALIGN;
+    if (bl_status st = check_device()) return st;
+    return cuda_status(
+        bl::launch_act_quant(x, M, K, bl::XQ_NATURAL, xq, scale, xsum, (cudaStream_t)stream));
+}
+
+BL_API bl_status bitlinear_forward(const uint8_t* Wp, const float* gamma, int64_t N, int64_t K,
+                                   const uint16_t* x, int64_t M, const uint16_t* residual,
+                                   uint16_t* y, int32_t* acc, void* ws, size_t ws_bytes,
+                                   bl_stream_t stream) {
+    if (M < 0 || M > kMaxM || N < 0 || N > kMaxN || K < 4 || K % 4 != 0 || K > kMaxK)
+        return BL_ERR_SHAPE;
+    if (M == 0 || N == 0) return BL_OK;
+    if (!Wp || !gamma || !x || !y) return BL_ERR_NULL;
+    if (!aligned(gamma, 4) || !aligned(x, 2) || !aligned(y, 2) || (residual && !aligned(residual, 2)) ||
+        (acc && !aligned(acc, 4)))
+        return BL_ERR_ALIGN;
+    const ForwardWs w = forward_ws(M, K);
+    if (bl_status st = check_ws(ws, ws_bytes, w.total)) return st;
+    if (bl_status st = check_device()) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    char* base = (char*)ws;
+    int8_t* xq = (int8_t*)(base + w.xq);
+    float* scale = (float*)(base + w.scale);
+    int32_t* xsum = (int32_t*)(base + w.xsum);
+
+    const bool fast = gemv_fast(Wp, N, K);
+    BL_TRY(bl::launch_act_quant(x, M, K, fast ? bl::XQ_PLANES : bl::XQ_NATURAL, xq, scale, xsum, s));
+    bl::GemvOut out;
+    out.y = y;
+    out.residual = residual;
+    out.acc = acc;
+    return project(fast, Wp, gamma, N, K, xq, scale, xsum, M, out, s);
+}
+
+BL_API bl_status bitlinear_ffn(const uint8_t* Wg, const float* gg, const uint8_t* Wu,
+                               const float* gu, const uint8_t* Wd, const float* gd, int64_t d,
+                               int64_t f, const uint16_t* x, int64_t M, const uint16_t* residual,
+                               uint16_t* y, void* ws, size_t ws_bytes, bl_stream_t stream) {
+    if (M < 0 || M > kMaxM || d < 4 || d % 4 != 0 || f < 4 || f % 4 != 0 || d > kMaxK ||
+        f > kMaxK)
+        return BL_ERR_SHAPE;
+    if (M == 0) return BL_OK;
+    if (!Wg || !gg || !Wu || !gu || !Wd || !gd || !x || !y) return BL_ERR_NULL;
+    if (!aligned(gg, 4) || !aligned(gu, 4) || !aligned(gd, 4) || !aligned(x, 2) || !aligned(y, 2) ||
+        (residual && !aligned(residual, 2)))
+        return BL_ERR_ALIGN;
+    const FfnWs w = ffn_ws(M, f, d);
+    if (bl_status st = check_ws(ws, ws_bytes, w.total)) return st;
+    if (bl_status st = check_device()) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    char* base = (char*)ws;
+    int8_t* xq = (int8_t*)(base + w.xq);
+    float* scale = (float*)(base + w.scale);
+    int32_t* xsum = (int32_t*)(base + w.xsum);
+    float* g = (float*)(base + w.g);
+    float* u = (float*)(base + w.u);
+    int8_t* q2 = (int8_t*)(base + w.q2);
+    float* s2 = (float*)(base + w.s2);
+    int32_t* xsum2 = (int32_t*)(base + w.xsum2);
+
+    const bool fast_up = gemv_fast(Wg, f, d) && gemv_fast(Wu, f, d);
+    const bool fast_down = gemv_fast(Wd, d, f);
+    BL_TRY(bl::launch_act_quant(x, M, d, fast_up ? bl::XQ_PLANES : bl::XQ_NATURAL, xq, scale, xsum, s));
+    bl::GemvOut og;
+    og.y32 = g;
+    if (bl_status st = project(fast_up, Wg, gg, f, d, xq, scale, xsum, M, og, s)) return st;
+    bl::GemvOut ou;
+    ou.y32 = u;
+    if (bl_status st = project(fast_up, Wu, gu, f, d, xq, scale, xsum, M, ou, s)) return st;
+    BL_TRY(bl::launch_ffn_finalise(g, u, M, f, fast_down ? bl::XQ_PLANES : bl::XQ_NATURAL, q2, s2,
+                                   xsum2, s));
+    bl::GemvOut od;
+    od.y = y;
+    od.residual = residual;
+    return project(fast_down, Wd, gd, d, f, q2, s2, xsum2, M, od, s);
+}
+
+BL_API bl_status bitlinear_validate_packed(const uint8_t* Wp, int64_t N, int64_t K,
+                                           int64_t* bad_count, void* ws, size_t ws_bytes,
+                                           bl_stream_t stream) {
+    if (N < 0 || K < 0 || K % 4 != 0) return BL_ERR_SHAPE;
+    if (bad_count) *bad_count = 0;
+    if (N == 0 || K == 0) return BL_OK;
+    if (!Wp) return BL_ERR_NULL;
+    if (bl_status st = check_ws(ws, ws_bytes, kWsAlign)) return st;
+    if (bl_status st = check_device()) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    unsigned long long* cnt = (unsigned long long*)ws;
+    BL_TRY(cudaMemsetAsync(cnt, 0, sizeof(*cnt), s));
+    BL_TRY(bl::launch_count_bad_codes(Wp, N * (K / 4), cnt, s));
+    unsigned long long host = 0;
+    BL_TRY(cudaMemcpyAsync(&host, cnt, sizeof(host), cudaMemcpyDeviceToHost, s));
+    BL_TRY(cudaStreamSynchronize(s));
+    if (bad_count) *bad_count = (int64_t)host;
+    return host ? BL_ERR_BAD_CODE : BL_OK;
+}
+
+BL_API bl_status bitlinear_get_device_error(bl_stream_t stream) {
+    if (bl_status st = check_device()) return st;
+    if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return BL_ERR_CUDA;
+    if (cudaGetLastError() != cudaSuccess) return BL_ERR_CUDA;
+    unsigned v = 0;
+    if (bl::read_and_clear_device_error(&v) != cudaSuccess) return BL_ERR_CUDA;
+    return v ? BL_ERR_TIMEOUT : BL_OK;
+}

@@ -1,0 +1,53 @@
+// Host-side launchers of the library's kernels (internal; the public
+// interface is include/bitlinear.h). Each returns the cudaError_t of its launch.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace bl {
+
+// ---- weight packing (pack.cu)
+// Per-block fp64 partial sums of |W| into partial[0 .. absmean_blocks(n)-1].
+int absmean_blocks(int64_t n);
+cudaError_t launch_absmean(const void* W, bool fp32, int64_t n, double* partial, float* gamma,
+                           cudaStream_t s);
+cudaError_t launch_ternary_pack(const void* W, bool fp32, int64_t N, int64_t K, const float* gamma,
+                                uint8_t* Wp, cudaStream_t s);
+cudaError_t launch_count_bad_codes(const uint8_t* Wp, int64_t nbytes, unsigned long long* count,
+                                   cudaStream_t s);
+
+// ---- activation quantisation (actquant.cu); layout is an XqLayout
+cudaError_t launch_act_quant(const uint16_t* x, int64_t M, int64_t K, int layout, int8_t* xq,
+                             float* scale, int32_t* xsum, cudaStream_t s);
+
+// ---- decode GEMV (gemv.cu)
+// Output modes: bf16 y (+ residual, + int32 acc dump) or fp32 dequantised y32.
+struct GemvOut {
+    uint16_t* y = nullptr;              // [M, N] bf16 bits
+    const uint16_t* residual = nullptr; // [M, N] bf16 bits or null
+    int32_t* acc = nullptr;             // [M, N] or null
+    float* y32 = nullptr;               // [M, N] fp32 (used instead of y when set)
+};
+// Xp: PLANES layout codes for M tokens; requires K % 256 == 0 and 16-byte aligned Wp, Xp.
+bool gemv_fast_ok(int64_t N, int64_t K);
+cudaError_t launch_gemv(const uint8_t* Wp, const float* gamma, int64_t N, int64_t K,
+                        const int8_t* Xp, const float* scale, const int32_t* xsum, int64_t M,
+                        const GemvOut& out, cudaStream_t s);
+// Any K % 4 == 0: NATURAL layout codes, one warp per output.
+cudaError_t launch_gemv_generic(const uint8_t* Wp, const float* gamma, int64_t N, int64_t K,
+                                const int8_t* Xn, const float* scale, int64_t M,
+                                const GemvOut& out, cudaStream_t s);
+
+// ---- FFN glue (ffn.cu)
+// h = relu(g)^2 * u; hn = subln(h); q2, s2, xsum2 = quant(hn) in `layout`.
+cudaError_t launch_ffn_finalise(const float* g, const float* u, int64_t M, int64_t f, int layout,
+                                int8_t* q2, float* s2, int32_t* xsum2, cudaStream_t s);
+
+// ---- device error word: set by bounded waits inside kernels that give up.
+// Address of the current device's word (for kernels), and a host read that
+// also clears it.
+cudaError_t device_error_word(unsigned int** ptr);
+cudaError_t read_and_clear_device_error(unsigned int* value);
+
+}  // namespace bl

@@ -1,0 +1,182 @@
+/*
+ * bitlinear.h -- C ABI of the B200 (sm_100a) BitLinear W1.58A8 library.
+ *
+ * The operation is the BitLinear forward of BitNet b1.58: ternary weights from
+ * absmean quantisation packed four per byte, activations quantised per token to
+ * int8 by absmax, an exact integer contraction, and a dequantisation to bf16.
+ * Sources: "BitNet b1.58 2B4T Technical Report" paper card (ai-papers.xuzou.cn),
+ * sections "Method Adaptation" (absmean ternary weights, per-token absmax int8
+ * activations, subln, ReLU^2, no bias, four ternary weights per int8 value in
+ * HBM, pack-store-load-unpack-compute kernel), "Compute Setup" (packed 1.58-bit
+ * weights for inference, a custom W1.58A8 CUDA kernel) and "Bottleneck" (no
+ * library kernel serves W1.58A8); the fishai news digest of the same report
+ * (news.fishai.com.cn/news/3455510), list of the BitLinear layer's parts.
+ *
+ * Conventions shared by every call:
+ *   - All tensor pointers are DEVICE pointers, allocated and owned by the caller.
+ *     The library allocates no device memory in any call.
+ *   - bf16 tensors are passed as their 16-bit patterns (uint16_t).
+ *   - Matrices are row-major. W is [N, K] (out x in, as nn.Linear); x is [M, K];
+ *     y and acc are [M, N].
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL is the legacy
+ *     default stream). Arguments are validated on the host before anything is
+ *     launched; on an error nothing is launched and the status says why.
+ *   - No call synchronises the stream, except bitlinear_validate_packed and
+ *     bitlinear_get_device_error, which say so.
+ *   - No C++ exception crosses this boundary. A failed launch returns BL_ERR_CUDA.
+ *   - Calls on different streams may overlap only if their workspaces differ.
+ *
+ * Packed weight format (this library's reading; the pages only say "four ternary
+ * weights in one 8-bit value"): Wp is [N, K/4] uint8, row-major. Byte j of row n
+ * holds weights k = 4j .. 4j+3; weight 4j+i is stored in bits 2i..2i+1 as the
+ * code q+1 in {0, 1, 2} (q in {-1, 0, +1}). Code 3 is invalid.
+ *
+ * Arithmetic (every step is one IEEE fp32 operation, round to nearest even, with
+ * no fused multiply-add, unless noted):
+ *   gamma = fp32( sum_{n,k} |W[n,k]| / (N*K) )      sum and division in fp64
+ *   Wq    = clip(rint(W / (gamma + 1e-5)), -1, 1)
+ *   s_m   = 127 / max(max_k |x[m,k]|, 1e-5)
+ *   xq    = clip(rint(x * s_m), -128, 127)
+ *   acc   = sum_k Wq[n,k] * xq[m,k]                 exact int32
+ *   y     = bf16( float(acc) * (gamma / s_m) )      [+ float(residual) before bf16]
+ */
+#ifndef BITLINEAR_H
+#define BITLINEAR_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t, declared here so this header needs no CUDA headers. */
+typedef struct CUstream_st* bl_stream_t;
+
+typedef enum {
+    BL_OK = 0,
+    BL_ERR_NULL = 1,        /* a required pointer is NULL */
+    BL_ERR_SHAPE = 2,       /* a size is negative, zero where it may not be, K % 4 != 0, or too large */
+    BL_ERR_ALIGN = 3,       /* a pointer is not aligned as the call requires */
+    BL_ERR_DTYPE = 4,       /* unknown bl_dtype */
+    BL_ERR_WORKSPACE = 5,   /* workspace smaller than bitlinear_workspace_bytes() */
+    BL_ERR_UNSUPPORTED = 6, /* valid arguments this build does not handle (e.g. no sm_100 device) */
+    BL_ERR_CUDA = 7,        /* a CUDA call or launch failed */
+    BL_ERR_TIMEOUT = 8,     /* a bounded wait inside a kernel gave up (see bitlinear_get_device_error) */
+    BL_ERR_BAD_CODE = 9     /* packed weights hold the invalid code 3 */
+} bl_status;
+
+typedef enum { BL_BF16 = 0, BL_FP32 = 1 } bl_dtype;
+
+/* Operation ids for bitlinear_workspace_bytes. */
+typedef enum {
+    BL_OP_PACK = 0,     /* sizes: N, K of the weight */
+    BL_OP_FORWARD = 1,  /* sizes: M, N, K */
+    BL_OP_FFN = 2,      /* sizes: M, N = f (hidden), K = d (model width) */
+    BL_OP_VALIDATE = 3  /* sizes ignored */
+} bl_op;
+
+/* Human-readable name of a status. Never NULL; host only. */
+const char* bitlinear_status_string(bl_status status);
+
+/* Bytes of workspace `op` needs for the given sizes (0 for an invalid op).
+ * Host only, no CUDA call. The workspace must be 256-byte aligned. */
+size_t bitlinear_workspace_bytes(int op, int64_t M, int64_t N, int64_t K);
+
+/*
+ * Absmean ternary quantisation and packing of one weight tensor (one-time work).
+ * Paper card, "Method Adaptation": weights quantised with absmean onto {-1, 0, +1}
+ * in the forward pass, four ternary weights packed into one 8-bit value in HBM.
+ *
+ *   W      [N, K] device, bf16 bits (wdt = BL_BF16) or fp32 (BL_FP32); 16-byte aligned
+ *   N, K   N >= 1, K >= 4, K % 4 == 0, N*K < 2^40
+ *   Wp     [N, K/4] device uint8 output (format above); 16-byte aligned
+ *   gamma  [1] device fp32 output: mean |W| (the per-tensor absmean scale)
+ *   ws     device workspace of bitlinear_workspace_bytes(BL_OP_PACK, 0, N, K) bytes
+ * Deterministic: the fp64 sum runs in a fixed order for given N, K.
+ */
+bl_status bitlinear_pack_weights(const void* W, int wdt, int64_t N, int64_t K,
+                                 uint8_t* Wp, float* gamma,
+                                 void* ws, size_t ws_bytes, bl_stream_t stream);
+
+/*
+ * Per-token absmax quantisation of activations to int8.
+ * Paper card, "Method Adaptation": activations quantised per token with absmax
+ * to 8-bit integers.
+ *
+ *   x      [M, K] device bf16 bits; 16-byte aligned
+ *   M, K   M >= 0 (M == 0 is a no-op), K >= 4, K % 4 == 0
+ *   xq     [M, K] device int8 output, row-major; 16-byte aligned
+ *   scale  [M] device fp32 output: s_m = 127 / max(absmax_m, 1e-5)
+ *   xsum   [M] device int32 output: sum_k xq[m,k]; may be NULL
+ */
+bl_status bitlinear_quant_act(const uint16_t* x, int64_t M, int64_t K,
+                              int8_t* xq, float* scale, int32_t* xsum, bl_stream_t stream);
+
+/*
+ * One BitLinear forward: quantise x per token, contract with the packed ternary
+ * weights, dequantise to bf16. Dig news article on the release, section 2:
+ * nn.Linear replaced by BitLinear; paper card, "Method Adaptation": packed int8
+ * weights loaded to on-chip memory, unpacked right before the matmul, multiplied
+ * with int8 activations. No bias.
+ *
+ *   Wp        [N, K/4] device packed weights; 16-byte aligned
+ *   gamma     [1] device fp32 (as written by bitlinear_pack_weights)
+ *   N, K      N >= 0, K >= 4, K % 4 == 0
+ *   x         [M, K] device bf16 bits; 16-byte aligned
+ *   M         M >= 0; M == 0 or N == 0 launches nothing
+ *   residual  [M, N] device bf16 bits added before the final rounding; may be NULL
+ *   y         [M, N] device bf16 bits output; 4-byte aligned
+ *   acc       [M, N] device int32 output of the exact accumulator; may be NULL
+ *   ws        device workspace of bitlinear_workspace_bytes(BL_OP_FORWARD, M, N, K) bytes
+ * Kernel choice: M <= 16 streams the packed weights once through a
+ * bandwidth-bound GEMV; larger M runs the tensor-core GEMM when the shape allows
+ * it (N % 256 == 0 and K % 128 == 0), else a batched GEMV. Every path gives the same bits.
+ */
+bl_status bitlinear_forward(const uint8_t* Wp, const float* gamma, int64_t N, int64_t K,
+                            const uint16_t* x, int64_t M, const uint16_t* residual,
+                            uint16_t* y, int32_t* acc,
+                            void* ws, size_t ws_bytes, bl_stream_t stream);
+
+/*
+ * One FFN sub-layer of BitNet b1.58 (fishai digest: ReLU^2 in the FFN, subln;
+ * paper card, "Method Adaptation": subln, ReLU^2 feed-forward, no bias):
+ *   xq, s   = quant(x)                       x [M, d]
+ *   g, u    = deq(Wg . xq), deq(Wu . xq)     fp32, [M, f]
+ *   h       = max(g, 0)^2 * u
+ *   hn      = h / sqrt(mean_j h^2 + 1e-5)    unit-weight RMSNorm; sum in fp64
+ *   q2, s2  = quant(hn)
+ *   y       = bf16(residual + deq(Wd . q2))  y [M, d]; residual may be NULL
+ *   Wg, Wu  [f, d/4] packed; gg, gu [1] device fp32
+ *   Wd      [d, f/4] packed; gd [1] device fp32
+ *   d, f    multiples of 4
+ *   ws      bitlinear_workspace_bytes(BL_OP_FFN, M, f, d) bytes
+ * Alignment as bitlinear_forward.
+ */
+bl_status bitlinear_ffn(const uint8_t* Wg, const float* gg, const uint8_t* Wu, const float* gu,
+                        const uint8_t* Wd, const float* gd, int64_t d, int64_t f,
+                        const uint16_t* x, int64_t M, const uint16_t* residual, uint16_t* y,
+                        void* ws, size_t ws_bytes, bl_stream_t stream);
+
+/*
+ * Check packed weights for the invalid code 3. SYNCHRONISES `stream`.
+ * Returns BL_OK when every code is valid, BL_ERR_BAD_CODE otherwise; the number
+ * of invalid codes is written to *bad_count (host pointer, may be NULL).
+ *   ws  bitlinear_workspace_bytes(BL_OP_VALIDATE, 0, 0, 0) bytes of device memory
+ */
+bl_status bitlinear_validate_packed(const uint8_t* Wp, int64_t N, int64_t K, int64_t* bad_count,
+                                    void* ws, size_t ws_bytes, bl_stream_t stream);
+
+/*
+ * SYNCHRONISES `stream`, then reports BL_ERR_CUDA for a pending CUDA error, or
+ * BL_ERR_TIMEOUT when a bounded wait inside one of this library's kernels gave up
+ * since the last call on this device (the kernel that gave up wrote no output it
+ * could not finish and returned); the timeout flag is cleared by this call.
+ */
+bl_status bitlinear_get_device_error(bl_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BITLINEAR_H */

@@ -1,0 +1,146 @@
+"""The C ABI library: it loads, exports every declared symbol, and rejects bad
+arguments on the host before touching a GPU (CPU only; no compute calls)."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+import bitlinear_w1_a8_02_b200 as bl
+from bitlinear_w1_a8_02_b200 import binding
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "bitlinear.h")
+
+# bl_status codes, as include/bitlinear.h numbers them
+OK, NULL, SHAPE, ALIGN, DTYPE, WS, UNSUP = 0, 1, 2, 3, 4, 5, 6
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(bitlinear_\w+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol():
+    names = declared_functions()
+    assert len(names) >= 8
+    L = bl.lib()
+    for n in names:
+        assert hasattr(L, n), n
+    assert set(names) == set(binding.SIGNATURES)
+
+
+def test_library_exports_nothing_else():
+    out = os.popen(f"nm -D --defined-only {bl.LIB_PATH}").read()
+    exported = {ln.split()[-1] for ln in out.splitlines() if " T " in ln}
+    ours = {n for n in exported if n.startswith("bitlinear_")}
+    assert ours == set(declared_functions())
+
+
+def test_status_strings():
+    L = bl.lib()
+    for code, name in binding.STATUS_NAMES.items():
+        s = L.bitlinear_status_string(code).decode()
+        assert s.startswith(name), (code, s)
+    assert L.bitlinear_status_string(1234).decode() == "unknown bl_status"
+
+
+def test_workspace_sizes():
+    L = bl.lib()
+    f = L.bitlinear_workspace_bytes
+    assert f(bl.BL_OP_FORWARD, 1, 2560, 2560) >= 2560 + 8
+    assert f(bl.BL_OP_FORWARD, 16, 6912, 2560) >= 16 * 2560
+    assert f(bl.BL_OP_FFN, 512, 6912, 2560) >= 512 * 6912 * 9
+    assert f(bl.BL_OP_PACK, 0, 512, 256) >= 8
+    assert f(bl.BL_OP_VALIDATE, 0, 0, 0) == 256
+    assert f(99, 1, 1, 4) == 0
+    assert f(bl.BL_OP_FORWARD, -1, 1, 4) == 0
+    for op in (bl.BL_OP_FORWARD, bl.BL_OP_FFN):
+        assert f(op, 1, 2560, 2560) % 256 == 0
+
+
+# Fake, never-dereferenced addresses: every call below must fail host-side
+# validation before any CUDA call.
+A = 0x10000  # 64 KiB aligned
+P = ctypes.c_void_p
+
+
+def test_host_validation_forward():
+    L = bl.lib()
+    F = L.bitlinear_forward
+    ws_need = L.bitlinear_workspace_bytes(bl.BL_OP_FORWARD, 1, 512, 256)
+    args = dict(Wp=A, g=A, N=512, K=256, x=A, M=1, res=None, y=A, acc=None, ws=A, wsb=ws_need)
+
+    def call(**kw):
+        a = dict(args, **kw)
+        return F(P(a["Wp"]), P(a["g"]), a["N"], a["K"], P(a["x"]), a["M"], P(a["res"]), P(a["y"]),
+                 P(a["acc"]), P(a["ws"]), a["wsb"], None)
+
+    assert call(K=258) == SHAPE
+    assert call(K=0) == SHAPE
+    assert call(M=-1) == SHAPE
+    assert call(N=-3) == SHAPE
+    assert call(M=70000) == SHAPE
+    assert call(K=1 << 20) == SHAPE
+    assert call(M=0) == OK          # empty: nothing to do
+    assert call(N=0) == OK
+    assert call(Wp=None) == NULL
+    assert call(x=None) == NULL
+    assert call(y=None) == NULL
+    assert call(g=None) == NULL
+    assert call(g=A + 2) == ALIGN
+    assert call(y=A + 1) == ALIGN
+    assert call(acc=A + 2) == ALIGN
+    assert call(ws=A + 16) == ALIGN
+    assert call(ws=None) == NULL
+    assert call(wsb=ws_need - 1) == WS
+
+
+def test_host_validation_pack_quant_ffn_validate():
+    L = bl.lib()
+    need = L.bitlinear_workspace_bytes(bl.BL_OP_PACK, 0, 8, 16)
+    pk = L.bitlinear_pack_weights
+    assert pk(P(A), 7, 8, 16, P(A), P(A), P(A), need, None) == DTYPE
+    assert pk(P(A), bl.BL_BF16, 0, 16, P(A), P(A), P(A), need, None) == SHAPE
+    assert pk(P(A), bl.BL_BF16, 8, 18, P(A), P(A), P(A), need, None) == SHAPE
+    assert pk(None, bl.BL_BF16, 8, 16, P(A), P(A), P(A), need, None) == NULL
+    assert pk(P(A + 8), bl.BL_BF16, 8, 16, P(A), P(A), P(A), need, None) == ALIGN
+    assert pk(P(A), bl.BL_BF16, 8, 16, P(A), P(A), P(A), need - 1, None) == WS
+
+    q = L.bitlinear_quant_act
+    assert q(P(A), 2, 6, P(A), P(A), None, None) == SHAPE
+    assert q(P(A), 0, 8, None, None, None, None) == OK
+    assert q(None, 2, 8, P(A), P(A), None, None) == NULL
+    assert q(P(A), 2, 8, P(A), P(A + 1), None, None) == ALIGN
+
+    ffn = L.bitlinear_ffn
+    need = L.bitlinear_workspace_bytes(bl.BL_OP_FFN, 1, 32, 16)
+    base = [P(A)] * 6
+    assert ffn(*base, 16, 30, P(A), 1, None, P(A), P(A), need, None) == SHAPE
+    assert ffn(*base, 16, 32, P(A), 0, None, P(A), P(A), need, None) == OK
+    assert ffn(*base[:5], None, 16, 32, P(A), 1, None, P(A), P(A), need, None) == NULL
+    assert ffn(*base, 16, 32, P(A), 1, None, P(A), P(A), need - 1, None) == WS
+
+    v = L.bitlinear_validate_packed
+    cnt = ctypes.c_int64(-1)
+    assert v(P(A), 4, 6, ctypes.byref(cnt), P(A), 256, None) == SHAPE
+    assert v(P(A), 0, 16, ctypes.byref(cnt), P(A), 256, None) == OK and cnt.value == 0
+    assert v(None, 4, 16, None, P(A), 256, None) == NULL
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device answer")
+def test_valid_call_without_device_is_unsupported():
+    L = bl.lib()
+    need = L.bitlinear_workspace_bytes(bl.BL_OP_FORWARD, 1, 512, 256)
+    st = L.bitlinear_forward(P(A), P(A), 512, 256, P(A), 1, None, P(A), None, P(A), need, None)
+    assert st == UNSUP
+    assert L.bitlinear_get_device_error(None) == UNSUP
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(binding, "_lib", None)
+    monkeypatch.setattr(binding, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(ImportError):
+        binding.lib()

@@ -1,0 +1,249 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle.
+
+Integers (packed bytes, gamma bits, activation codes, scales, accumulators) must
+match bit for bit; bf16 outputs must meet the 2^-8 relative bar and, because
+every fp32 step is a unique IEEE result in both implementations, also match bit
+for bit. Full-size workloads compare sampled rows and tokens, each computed by
+the oracle on the same inputs.
+"""
+import numpy as np
+import pytest
+import torch
+
+import bitlinear_w1_a8_02_b200 as bl
+import oracle
+from bitlinear_w1_a8_02_b200 import synth
+from gpu_util import assert_bf16_close, assert_bf16_exact, bits, np_, sample_indices
+
+pytestmark = pytest.mark.gpu
+
+
+def make_weights(N, K, sigma, seed, dtype="bf16"):
+    return synth.weights(N, K, sigma, seed, dtype=dtype)
+
+
+def pack_both(W_cpu: torch.Tensor, dev):
+    """Pack on the GPU and in the oracle; assert identical bytes and gamma."""
+    Wp, gamma = bl.pack_weights(W_cpu.to(dev))
+    if W_cpu.dtype == torch.bfloat16:
+        Wp_ref, g_ref = oracle.pack_weights(bits(W_cpu))
+    else:
+        Wp_ref, g_ref = oracle.pack_weights(np_(W_cpu))
+    assert np_(gamma)[0].view(np.uint32) == np.float32(g_ref).view(np.uint32), "gamma bits"
+    assert np.array_equal(np_(Wp), Wp_ref), "packed bytes"
+    return Wp, gamma, Wp_ref, g_ref
+
+
+def check_forward_full(Wp, gamma, Wp_ref, g_ref, x_cpu, dev, residual=None):
+    y, acc = bl.forward(Wp, gamma, x_cpu.to(dev), residual=None if residual is None else residual.to(dev),
+                        want_acc=True)
+    ref = oracle.forward(Wp_ref, g_ref, bits(x_cpu), residual=None if residual is None else bits(residual))
+    assert np.array_equal(np_(acc), ref["acc"]), "int32 accumulators"
+    assert_bf16_close(bits(y), ref["y"])
+    assert_bf16_exact(bits(y), ref["y"])
+
+
+def check_forward_sampled(Wp, gamma, Wp_ref, g_ref, x_cpu, dev, rows, toks):
+    y, acc = bl.forward(Wp, gamma, x_cpu.to(dev), want_acc=True)
+    ref = oracle.forward(Wp_ref[rows], g_ref, bits(x_cpu[toks]))
+    got_acc = np_(acc)[np.ix_(toks, rows)]
+    assert np.array_equal(got_acc, ref["acc"]), "int32 accumulators (sampled)"
+    got_y = bits(y)[np.ix_(toks, rows)]
+    assert_bf16_close(got_y, ref["y"])
+    assert_bf16_exact(got_y, ref["y"])
+
+
+# ----------------------------------------------------------------------------- packing
+
+@pytest.mark.parametrize("N,K,dtype", [(512, 256, "fp32"), (2560, 2560, "bf16"), (640, 2560, "bf16"),
+                                       (6912, 2560, "bf16"), (2560, 6912, "bf16"), (136, 196, "bf16"),
+                                       (1, 4, "fp32"), (3, 12, "bf16")])
+def test_pack_parity(cuda_device, N, K, dtype):
+    pack_both(make_weights(N, K, 0.02, seed=N + K, dtype=dtype), cuda_device)
+
+
+def test_pack_parity_100b_shape(cuda_device):
+    W = make_weights(8192, 28672, synth.SIGMA_100B, seed=77)
+    Wp, gamma, Wp_ref, _ = pack_both(W, cuda_device)
+    assert bl.validate_packed(Wp) == 0
+
+
+def test_validate_packed_counts_bad_codes(cuda_device):
+    Wp, _ = bl.pack_weights(make_weights(64, 256, 0.02, seed=3).to(cuda_device))
+    assert bl.validate_packed(Wp) == 0
+    Wp[3, 5] = 0xFF   # four invalid codes
+    Wp[10, 0] = 0x57  # one invalid code (field 0 = 3)
+    assert bl.validate_packed(Wp) == 5
+
+
+# ----------------------------------------------------------------------------- act-quant
+
+@pytest.mark.parametrize("M,K", [(1, 256), (7, 2560), (33, 6912), (4, 260), (2, 4), (5, 28672)])
+def test_quant_act_parity(cuda_device, M, K):
+    x = synth.activations(M, K, seed=M * 7 + K, outliers=True)
+    if M > 2:
+        x[1] = 0
+        x[2] = x[2] * 1e-7
+    xq, s, xs = bl.quant_act(x.to(cuda_device))
+    rq, rs, rxs = oracle.quant_act(bits(x))
+    assert np.array_equal(np_(xq), rq)
+    assert np.array_equal(np_(s).view(np.uint32), rs.view(np.uint32))
+    assert np.array_equal(np_(xs), rxs)
+
+
+def test_quant_act_empty(cuda_device):
+    x = torch.empty((0, 256), dtype=torch.bfloat16, device=cuda_device)
+    xq, s, xs = bl.quant_act(x)
+    assert xq.shape == (0, 256)
+
+
+# ----------------------------------------------------------------------------- forward
+
+def test_forward_single_fp32_weights(cuda_device):
+    """The small case: M=1, K=256, N=512, fp32 W ~ N(0, 0.02^2), x ~ N(0, 1), seed 0."""
+    W = make_weights(512, 256, 0.02, seed=0, dtype="fp32")
+    x = synth.activations(1, 256, seed=0, outliers=False)
+    Wp, gamma, Wp_ref, g_ref = pack_both(W, cuda_device)
+    check_forward_full(Wp, gamma, Wp_ref, g_ref, x, cuda_device)
+
+
+@pytest.mark.parametrize("K,N", [(2560, 2560), (2560, 640), (2560, 6912), (6912, 2560)])
+def test_forward_decode_2b(cuda_device, K, N):
+    W = make_weights(N, K, 0.02, seed=1000 + K + N)
+    Wp, gamma, Wp_ref, g_ref = pack_both(W, cuda_device)
+    x = synth.activations(1, K, seed=1, outliers=True)
+    check_forward_full(Wp, gamma, Wp_ref, g_ref, x, cuda_device)
+
+
+@pytest.mark.parametrize("M", [2, 4, 8, 9, 16])
+@pytest.mark.parametrize("K,N", [(2560, 6912), (6912, 2560)])
+def test_forward_batched_decode(cuda_device, K, N, M):
+    W = make_weights(N, K, 0.02, seed=2000 + K + N)
+    Wp, gamma, Wp_ref, g_ref = pack_both(W, cuda_device)
+    x = synth.activations(M, K, seed=M, outliers=True)
+    check_forward_full(Wp, gamma, Wp_ref, g_ref, x, cuda_device)
+
+
+@pytest.mark.parametrize("M", [17, 512, 2048, 4096])
+@pytest.mark.parametrize("K,N", [(2560, 6912), (6912, 2560)])
+def test_forward_prefill_sampled(cuda_device, K, N, M):
+    W = make_weights(N, K, 0.02, seed=3000 + K + N)
+    Wp, gamma, Wp_ref, g_ref = pack_both(W, cuda_device)
+    x = synth.activations(M, K, seed=M + 5, outliers=True)
+    rows = sample_indices(N, 96, seed=M)
+    toks = sample_indices(M, 12, seed=M + 1)
+    check_forward_sampled(Wp, gamma, Wp_ref, g_ref, x, cuda_device, rows, toks)
+
+
+@pytest.mark.parametrize("M", [1, 16, 2048])
+@pytest.mark.parametrize("K,N", [(8192, 28672), (28672, 8192)])
+def test_forward_100b_sampled(cuda_device, K, N, M):
+    W = make_weights(N, K, synth.SIGMA_100B, seed=4000 + K % 1000)
+    Wp, gamma, Wp_ref, g_ref = pack_both(W, cuda_device)
+    x = synth.activations(M, K, seed=M + 9, outliers=True)
+    rows = sample_indices(N, 64, seed=M + 2)
+    toks = sample_indices(M, 8, seed=M + 3)
+    check_forward_sampled(Wp, gamma, Wp_ref, g_ref, x, cuda_device, rows, toks)
+
+
+@pytest.mark.parametrize("M,N,K", [(17, 136, 192), (3, 17, 256), (1, 1, 4), (5, 33, 260),
+                                   (16, 130, 512), (20, 100, 1024)])
+def test_forward_ragged_shapes(cuda_device, M, N, K):
+    W = make_weights(N, K, 0.02, seed=M + N + K)
+    Wp, gamma, Wp_ref, g_ref = pack_both(W, cuda_device)
+    x = synth.activations(M, K, seed=K, outliers=True)
+    check_forward_full(Wp, gamma, Wp_ref, g_ref, x, cuda_device)
+
+
+def test_forward_residual_and_degenerate_tokens(cuda_device):
+    K, N, M = 2560, 640, 6
+    W = make_weights(N, K, 0.02, seed=5)
+    Wp, gamma, Wp_ref, g_ref = pack_both(W, cuda_device)
+    x = synth.activations(M, K, seed=6, outliers=True)
+    x[0] = 0                      # all-zero token
+    x[1] = x[1] * 1e-8            # below the absmax floor
+    x[2, :] = 0
+    x[2, 7] = 3.0                 # a single non-zero channel
+    res = synth.activations(M, N, seed=8, outliers=False)
+    check_forward_full(Wp, gamma, Wp_ref, g_ref, x, cuda_device, residual=res)
+
+
+def test_forward_empty(cuda_device):
+    Wp, gamma = bl.pack_weights(make_weights(64, 256, 0.02, seed=1).to(cuda_device))
+    x = torch.empty((0, 256), dtype=torch.bfloat16, device=cuda_device)
+    y = bl.forward(Wp, gamma, x)
+    assert y.shape == (0, 64)
+
+
+def test_forward_is_deterministic(cuda_device):
+    W = make_weights(6912, 2560, 0.02, seed=9).to(cuda_device)
+    Wp, gamma = bl.pack_weights(W)
+    Wp2, gamma2 = bl.pack_weights(W)
+    assert torch.equal(Wp, Wp2) and torch.equal(gamma, gamma2)
+    for M in (1, 16, 512):
+        x = synth.activations(M, 2560, seed=M).to(cuda_device)
+        y1, a1 = bl.forward(Wp, gamma, x, want_acc=True)
+        y2, a2 = bl.forward(Wp, gamma, x, want_acc=True)
+        assert torch.equal(y1, y2) and torch.equal(a1, a2)
+
+
+def test_device_error_clean(cuda_device):
+    assert bl.get_device_error() == 0
+
+
+# ----------------------------------------------------------------------------- FFN
+
+def ffn_weights(layer, d, f, dev):
+    sg, su, sd = synth.ffn_layer_seeds(layer)
+    out = []
+    for N, K, seed in ((f, d, sg), (f, d, su), (d, f, sd)):
+        W = make_weights(N, K, synth.SIGMA_2B, seed)
+        Wp, gamma, Wp_ref, g_ref = pack_both(W, dev)
+        out.append((Wp, gamma, Wp_ref, g_ref))
+    return out
+
+
+def test_ffn_chain_decode_teacher_forced(cuda_device):
+    """30 layers at d=2560, f=6912, M=1. Each layer's GPU input is fed to the
+    oracle, so every layer is compared exactly; the chain is also run end to end."""
+    d, f, L = 2560, 6912, 30
+    h = synth.activations(1, d, seed=1, outliers=False)
+    h_dev = h.to(cuda_device)
+    h_ref = bits(h)
+    for layer in range(L):
+        (Wg, gg, Wgr, ggr), (Wu, gu, Wur, gur), (Wd, gd, Wdr, gdr) = ffn_weights(layer, d, f, cuda_device)
+        y_dev = bl.ffn(Wg, gg, Wu, gu, Wd, gd, h_dev, residual=h_dev)
+        ref = oracle.ffn_layer(Wgr, ggr, Wur, gur, Wdr, gdr, bits(h_dev), residual=bits(h_dev))
+        assert_bf16_close(bits(y_dev), ref["y"], f"layer {layer}")
+        assert_bf16_exact(bits(y_dev), ref["y"], f"layer {layer}")
+        chain = oracle.ffn_layer(Wgr, ggr, Wur, gur, Wdr, gdr, h_ref, residual=h_ref)
+        h_ref = chain["y"]
+        h_dev = y_dev
+    # end to end: the exact per-layer parity makes the chains identical
+    assert_bf16_exact(bits(h_dev), h_ref, "30-layer chain")
+
+
+def test_ffn_prefill_sampled_tokens(cuda_device):
+    d, f, M = 2560, 6912, 512
+    h = synth.activations(M, d, seed=2, outliers=False)
+    h_dev = h.to(cuda_device)
+    toks = sample_indices(M, 6, seed=4)
+    for layer in range(3):
+        (Wg, gg, Wgr, ggr), (Wu, gu, Wur, gur), (Wd, gd, Wdr, gdr) = ffn_weights(layer, d, f, cuda_device)
+        y_dev = bl.ffn(Wg, gg, Wu, gu, Wd, gd, h_dev, residual=h_dev)
+        xin = bits(h_dev)[toks]
+        ref = oracle.ffn_layer(Wgr, ggr, Wur, gur, Wdr, gdr, xin, residual=xin)
+        got = bits(y_dev)[toks]
+        assert_bf16_close(got, ref["y"], f"layer {layer}")
+        assert_bf16_exact(got, ref["y"], f"layer {layer}")
+        h_dev = y_dev
+
+
+def test_ffn_small_ragged(cuda_device):
+    d, f, M = 64, 200, 3
+    Wg, Wu, Wd = (make_weights(f, d, 0.02, 1), make_weights(f, d, 0.02, 2), make_weights(d, f, 0.02, 3))
+    P = [pack_both(W, cuda_device) for W in (Wg, Wu, Wd)]
+    x = synth.activations(M, d, seed=3, outliers=True)
+    y = bl.ffn(P[0][0], P[0][1], P[1][0], P[1][1], P[2][0], P[2][1], x.to(cuda_device))
+    ref = oracle.ffn_layer(P[0][2], P[0][3], P[1][2], P[1][3], P[2][2], P[2][3], bits(x))
+    assert_bf16_exact(bits(y), ref["y"])
