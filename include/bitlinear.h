@@ -159,6 +159,33 @@ bl_status bitlinear_ffn(const uint8_t* Wg, const float* gg, const uint8_t* Wu, c
                         void* ws, size_t ws_bytes, bl_stream_t stream);
 
 /*
+ * bitlinear_forward without a workspace, for callers that cannot allocate.
+ * The pages have no counterpart of this call; it exists for deployment.
+ *
+ * Some callers cannot call cudaMalloc where they run a layer: a plugin inside an
+ * engine that reserved all device memory at start-up and allows no allocation
+ * afterwards, or a latency-critical loop in which an allocation would implicitly
+ * synchronise the device. They may also have no workspace buffer to pass. This
+ * call computes exactly what bitlinear_forward computes (same kernels, same bits)
+ * but keeps its scratch in a fixed 1 MiB array inside the library's own device
+ * memory, which every GPU that loads the library holds until the process exits.
+ *
+ *   Arguments as bitlinear_forward, minus ws / ws_bytes.
+ *   Limit: the scratch must hold the activation codes plus two per-token words:
+ *          round256(M*K) + 2*round256(4*M) <= 1048576 bytes (for example M <= 16 at
+ *          K <= 28672). Larger sizes return BL_ERR_WORKSPACE and launch nothing.
+ *   No call allocates device memory or calls an allocating library routine.
+ *   The first call on each device looks up the array's device address
+ *   (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   Every call on a device shares the one array, which keeps the last call's
+ *   contents (nothing in it needs to start at zero). Calls that can overlap on
+ *   the GPU (other streams, unordered host threads) race on it: order them.
+ */
+bl_status bitlinear_forward_noalloc(const uint8_t* Wp, const float* gamma, int64_t N, int64_t K,
+                                    const uint16_t* x, int64_t M, const uint16_t* residual,
+                                    uint16_t* y, int32_t* acc, bl_stream_t stream);
+
+/*
  * Check packed weights for the invalid code 3. SYNCHRONISES `stream`.
  * Returns BL_OK when every code is valid, BL_ERR_BAD_CODE otherwise; the number
  * of invalid codes is written to *bad_count (host pointer, may be NULL).
