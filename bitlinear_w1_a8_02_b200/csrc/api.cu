@@ -94,18 +94,35 @@ bl_status check_ws(const void* ws, size_t ws_bytes, size_t need) {
     return BL_OK;
 }
 
-// Whether the streaming GEMV can read these packed weights.
-inline bool gemv_fast(const uint8_t* Wp, int64_t N, int64_t K) {
-    return bl::gemv_fast_ok(N, K) && aligned(Wp, 16);
+// Which kernel runs a projection, and the activation-code layout it reads.
+enum class Path { GemvFast, GemvGeneric, GemmTc };
+
+// `x` is the bf16 input the codes are made from (the fast quantiser reads it
+// 16 bytes at a time); null when the codes come from the FFN glue kernel.
+inline Path choose_path(const uint8_t* Wp, int64_t N, int64_t K, int64_t M, const void* xq,
+                        const void* x) {
+    if (x && !aligned(x, 16)) return Path::GemvGeneric;
+    if (M > 16 && bl::gemm_tc_ok(N, K, Wp, xq)) return Path::GemmTc;
+    if (bl::gemv_fast_ok(N, K) && aligned(Wp, 16)) return Path::GemvFast;
+    return Path::GemvGeneric;
 }
 
-// One BitLinear projection of already-quantised codes `xq` (layout chosen by
-// the caller through `fast`).
-bl_status project(bool fast, const uint8_t* Wp, const float* gamma, int64_t N, int64_t K,
+inline int layout_of(Path p) {
+    return p == Path::GemmTc ? bl::XQ_G16T : p == Path::GemvFast ? bl::XQ_PLANES : bl::XQ_NATURAL;
+}
+
+// One BitLinear projection of already-quantised codes `xq` (in layout_of(path)).
+bl_status project(Path path, const uint8_t* Wp, const float* gamma, int64_t N, int64_t K,
                   const int8_t* xq, const float* scale, const int32_t* xsum, int64_t M,
                   const bl::GemvOut& out, cudaStream_t s) {
-    if (fast) return cuda_status(bl::launch_gemv(Wp, gamma, N, K, xq, scale, xsum, M, out, s));
-    return cuda_status(bl::launch_gemv_generic(Wp, gamma, N, K, xq, scale, M, out, s));
+    switch (path) {
+        case Path::GemmTc:
+            return cuda_status(bl::launch_gemm_tc(Wp, gamma, N, K, xq, scale, xsum, M, out, s));
+        case Path::GemvFast:
+            return cuda_status(bl::launch_gemv(Wp, gamma, N, K, xq, scale, xsum, M, out, s));
+        default:
+            return cuda_status(bl::launch_gemv_generic(Wp, gamma, N, K, xq, scale, M, out, s));
+    }
 }
 
 }  // namespace
@@ -185,13 +202,13 @@ BL_API bl_status bitlinear_forward(const uint8_t* Wp, const float* gamma, int64_
     float* scale = (float*)(base + w.scale);
     int32_t* xsum = (int32_t*)(base + w.xsum);
 
-    const bool fast = gemv_fast(Wp, N, K);
-    BL_TRY(bl::launch_act_quant(x, M, K, fast ? bl::XQ_PLANES : bl::XQ_NATURAL, xq, scale, xsum, s));
+    const Path path = choose_path(Wp, N, K, M, xq, x);
+    BL_TRY(bl::launch_act_quant(x, M, K, layout_of(path), xq, scale, xsum, s));
     bl::GemvOut out;
     out.y = y;
     out.residual = residual;
     out.acc = acc;
-    return project(fast, Wp, gamma, N, K, xq, scale, xsum, M, out, s);
+    return project(path, Wp, gamma, N, K, xq, scale, xsum, M, out, s);
 }
 
 BL_API bl_status bitlinear_ffn(const uint8_t* Wg, const float* gg, const uint8_t* Wu,
@@ -220,21 +237,22 @@ BL_API bl_status bitlinear_ffn(const uint8_t* Wg, const float* gg, const uint8_t
     float* s2 = (float*)(base + w.s2);
     int32_t* xsum2 = (int32_t*)(base + w.xsum2);
 
-    const bool fast_up = gemv_fast(Wg, f, d) && gemv_fast(Wu, f, d);
-    const bool fast_down = gemv_fast(Wd, d, f);
-    BL_TRY(bl::launch_act_quant(x, M, d, fast_up ? bl::XQ_PLANES : bl::XQ_NATURAL, xq, scale, xsum, s));
+    // gate and up share one quantisation of x, so they must share a path
+    Path up = choose_path(Wg, f, d, M, xq, x);
+    if (choose_path(Wu, f, d, M, xq, x) != up) up = Path::GemvGeneric;
+    const Path down = choose_path(Wd, d, f, M, q2, nullptr);
+    BL_TRY(bl::launch_act_quant(x, M, d, layout_of(up), xq, scale, xsum, s));
     bl::GemvOut og;
     og.y32 = g;
-    if (bl_status st = project(fast_up, Wg, gg, f, d, xq, scale, xsum, M, og, s)) return st;
+    if (bl_status st = project(up, Wg, gg, f, d, xq, scale, xsum, M, og, s)) return st;
     bl::GemvOut ou;
     ou.y32 = u;
-    if (bl_status st = project(fast_up, Wu, gu, f, d, xq, scale, xsum, M, ou, s)) return st;
-    BL_TRY(bl::launch_ffn_finalise(g, u, M, f, fast_down ? bl::XQ_PLANES : bl::XQ_NATURAL, q2, s2,
-                                   xsum2, s));
+    if (bl_status st = project(up, Wu, gu, f, d, xq, scale, xsum, M, ou, s)) return st;
+    BL_TRY(bl::launch_ffn_finalise(g, u, M, f, layout_of(down), q2, s2, xsum2, s));
     bl::GemvOut od;
     od.y = y;
     od.residual = residual;
-    return project(fast_down, Wd, gd, d, f, q2, s2, xsum2, M, od, s);
+    return project(down, Wd, gd, d, f, q2, s2, xsum2, M, od, s);
 }
 
 BL_API bl_status bitlinear_validate_packed(const uint8_t* Wp, int64_t N, int64_t K,

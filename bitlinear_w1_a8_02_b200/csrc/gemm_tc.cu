@@ -1,0 +1,336 @@
+// Prefill GEMM on the 5th-generation tensor cores (tcgen05, sm_100a):
+//   acc[m, n] = sum_k Wq[n, k] * xq[m, k],   M > 16 tokens.
+//
+// Paper card "BitNet b1.58 2B4T Technical Report", "Method Adaptation": packed
+// int8 weights are loaded into on-chip memory and unpacked right before the
+// int8 matmul (pack-store-load-unpack-compute). On B200 this becomes:
+//   TMA:     packed weight tile [256 rows x 32 bytes] and activation-code tile
+//            [128 tokens x 128 codes] -> shared memory (one mbarrier per stage);
+//   unpack:  four warps turn every packed 32-bit word into 16 code bytes
+//            (three shifts and four ANDs) and store them straight into the
+//            128-byte-swizzled K-major operand layout the tensor core reads;
+//   MMA:     one thread issues tcgen05.mma kind::i8 (A = codes s8, B = weight
+//            codes u8 in {0,1,2}) into a 128 x 256 int32 accumulator in TMEM;
+//   epilogue: the same four warps read TMEM (tcgen05.ld), subtract the code
+//            offset (sum_k xq), dequantise and store bf16 / fp32 / int32.
+// The activation codes are in the G16T layout (each 16-code group stored as a
+// transposed 4x4 byte block), which is exactly the order a packed word unpacks
+// into, so no byte shuffling is needed anywhere.
+//
+// Every mbarrier wait is bounded (1 s); a wait that gives up sets the device
+// error word (reported as BL_ERR_TIMEOUT), lets the CTA drain and returns.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "tc_ptx.cuh"
+
+namespace bl {
+namespace {
+
+constexpr int BM = 128;            // tokens per tile (TMEM lanes)
+constexpr int BN = 256;            // weight rows per tile (TMEM columns)
+constexpr int BK = 128;            // codes per k-block (one 128-byte swizzle row)
+constexpr int STAGES = 3;
+constexpr int A_BYTES = BM * BK;        // 16 KiB activation codes
+constexpr int BU_BYTES = BN * BK;       // 32 KiB unpacked weight codes
+constexpr int BP_BYTES = BN * BK / 4;   //  8 KiB packed weights
+constexpr int THREADS = 192;            // warp 0 TMA, warp 1 MMA, warps 2-5 unpack + epilogue
+constexpr int UNPACK_THREADS = 128;
+constexpr uint32_t TMEM_COLS = 256;
+constexpr uint64_t WAIT_LIMIT_NS = 1000000000ull;
+constexpr size_t SMEM_BYTES = 1024 /*alignment slack*/ + STAGES * (A_BYTES + BU_BYTES + BP_BYTES) +
+                              256 /*barriers*/;
+
+static_assert(BN * BK / 4 / 4 % UNPACK_THREADS == 0, "unpack work must split evenly");
+
+__device__ __forceinline__ bool aligned16(const void* p) {
+    return (reinterpret_cast<uintptr_t>(p) & 15u) == 0;
+}
+
+__device__ __forceinline__ void report_timeout(unsigned* err, int* abort_flag) {
+    atomicOr(err, 1u);
+    atomicExch(abort_flag, 1);
+}
+
+__global__ void __launch_bounds__(THREADS, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   int M, int N, int K, const float* __restrict__ gamma_p,
+                   const float* __restrict__ scale, const int32_t* __restrict__ xsum, GemvOut out,
+                   unsigned* err) {
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ uint32_t tmem_base_sh;
+    __shared__ int abort_sh;
+
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~static_cast<uintptr_t>(1023));
+    uint8_t* sA = smem;
+    uint8_t* sBu = sA + STAGES * A_BYTES;
+    uint8_t* sBp = sBu + STAGES * BU_BYTES;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sBp + STAGES * BP_BYTES);
+    // bars[0..S): TMA landed; [S..2S): unpacked; [2S..3S): stage free; [3S]: accumulator done
+    auto full = [&](int s) { return tc::smem_u32(bars + s); };
+    auto ready = [&](int s) { return tc::smem_u32(bars + STAGES + s); };
+    auto empty = [&](int s) { return tc::smem_u32(bars + 2 * STAGES + s); };
+    const uint32_t accf = tc::smem_u32(bars + 3 * STAGES);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int n0 = blockIdx.x * BN, m0 = blockIdx.y * BM;
+    const int nkb = (K + BK - 1) / BK;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            tc::mbar_init(full(s), 1);
+            tc::mbar_init(ready(s), UNPACK_THREADS);
+            tc::mbar_init(empty(s), 1);
+        }
+        tc::mbar_init(accf, 1);
+        abort_sh = 0;
+        tc::fence_mbar_init();
+    }
+    if (warp == 1) {
+        tc::tmem_alloc(tc::smem_u32(&tmem_base_sh), TMEM_COLS);
+        tc::tmem_relinquish();
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = tmem_base_sh;
+
+    if (warp == 0) {
+        // ---------------------------------------------------------- TMA producer
+        if (lane == 0) {
+            tc::prefetch_tmap(&tmA);
+            tc::prefetch_tmap(&tmB);
+            int issued = 0;
+            for (int kb = 0; kb < nkb; ++kb) {
+                const int s = kb % STAGES;
+                const uint32_t ph = (kb / STAGES) & 1;
+                if (kb >= STAGES && !tc::mbar_wait(empty(s), ph ^ 1, WAIT_LIMIT_NS)) {
+                    report_timeout(err, &abort_sh);
+                    break;
+                }
+                if (*(volatile int*)&abort_sh) break;
+                tc::mbar_arrive_expect_tx(full(s), A_BYTES + BP_BYTES);
+                tc::tma_load_2d(tc::smem_u32(sA + s * A_BYTES), &tmA, kb * BK, m0, full(s));
+                tc::tma_load_2d(tc::smem_u32(sBp + s * BP_BYTES), &tmB, kb * (BK / 4), n0, full(s));
+                issued = kb + 1;
+            }
+            if (*(volatile int*)&abort_sh) {
+                // drain: let the copies still in flight land before the CTA exits
+                for (int kb = issued - STAGES < 0 ? 0 : issued - STAGES; kb < issued; ++kb)
+                    tc::mbar_wait(full(kb % STAGES), (kb / STAGES) & 1, WAIT_LIMIT_NS);
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc = tc::idesc_i8_s8u8(BM, BN);
+            for (int kb = 0; kb < nkb; ++kb) {
+                const int s = kb % STAGES;
+                const uint32_t ph = (kb / STAGES) & 1;
+                if (!tc::mbar_wait(ready(s), ph, WAIT_LIMIT_NS) ||
+                    !tc::mbar_wait(full(s), ph, WAIT_LIMIT_NS)) {
+                    report_timeout(err, &abort_sh);
+                    break;
+                }
+                tc::fence_after_sync();
+                const uint64_t ad = tc::desc_kmajor_sw128(tc::smem_u32(sA + s * A_BYTES));
+                const uint64_t bd = tc::desc_kmajor_sw128(tc::smem_u32(sBu + s * BU_BYTES));
+#pragma unroll
+                for (int kk = 0; kk < BK / 32; ++kk)  // K = 32 bytes per MMA: +2 in 16-byte units
+                    tc::mma_i8(tmem, ad + 2 * kk, bd + 2 * kk, idesc, (kb | kk) != 0);
+                tc::mma_commit(empty(s));
+            }
+            tc::mma_commit(accf);
+        }
+    } else {
+        // ---------------------------------------------------------- unpack
+        const int ut = threadIdx.x - 64;
+        bool ok = true;
+        for (int kb = 0; kb < nkb; ++kb) {
+            const int s = kb % STAGES;
+            const uint32_t ph = (kb / STAGES) & 1;
+            if (!tc::mbar_wait(full(s), ph, WAIT_LIMIT_NS)) {
+                report_timeout(err, &abort_sh);
+                ok = false;
+                break;
+            }
+            const uint32_t* bp = reinterpret_cast<const uint32_t*>(sBp + s * BP_BYTES);
+            uint8_t* bu = sBu + s * BU_BYTES;
+#pragma unroll
+            for (int i = 0; i < BN * 8 / UNPACK_THREADS; ++i) {
+                const int w = ut + UNPACK_THREADS * i;  // packed word w: row n, word j
+                const int n = w >> 3, j = w & 7;
+                const uint32_t word = bp[w];
+                uint4 v;
+                v.x = word & 0x03030303u;
+                v.y = (word >> 2) & 0x03030303u;
+                v.z = (word >> 4) & 0x03030303u;
+                v.w = (word >> 6) & 0x03030303u;
+                *reinterpret_cast<uint4*>(bu + (n >> 3) * 1024 + (n & 7) * 128 + ((j ^ (n & 7)) << 4)) = v;
+            }
+            tc::fence_proxy_async_smem();
+            tc::mbar_arrive(ready(s));
+        }
+        // ---------------------------------------------------------- epilogue
+        if (ok && !tc::mbar_wait(accf, 0, WAIT_LIMIT_NS)) {
+            report_timeout(err, &abort_sh);
+            ok = false;
+        }
+        ok = __all_sync(0xffffffffu, ok);  // tcgen05.ld below is warp-collective
+        tc::fence_after_sync();
+        const int q = warp & 3;  // TMEM lane quarter this warp may read
+        const int m = m0 + q * 32 + lane;
+        const bool mv = ok && m < M;
+        const float deq = mv ? __fdiv_rn(*gamma_p, scale[m]) : 0.0f;
+        const int xs = mv ? xsum[m] : 0;
+        const bool vec = (N % 8 == 0) && aligned16(out.y) && aligned16(out.y32) &&
+                         aligned16(out.residual) && aligned16(out.acc);
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+            uint32_t v[32];
+            if (ok) {
+                tc::tmem_ld_32x32(tmem + (static_cast<uint32_t>(q * 32) << 16) + c * 32, v);
+                tc::tmem_ld_wait();
+            }
+            const int nb = n0 + c * 32;
+            if (!mv || nb >= N) continue;
+            const size_t o = static_cast<size_t>(m) * N + nb;
+            if (vec && nb + 32 <= N) {
+                if (out.y32) {
+#pragma unroll
+                    for (int j = 0; j < 32; j += 4) {
+                        float4 f;
+                        f.x = dequant(static_cast<int>(v[j]) - xs, deq);
+                        f.y = dequant(static_cast<int>(v[j + 1]) - xs, deq);
+                        f.z = dequant(static_cast<int>(v[j + 2]) - xs, deq);
+                        f.w = dequant(static_cast<int>(v[j + 3]) - xs, deq);
+                        *reinterpret_cast<float4*>(out.y32 + o + j) = f;
+                    }
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 32; j += 8) {
+                        uint32_t pk[4];
+                        uint4 r = make_uint4(0, 0, 0, 0);
+                        if (out.residual) r = *reinterpret_cast<const uint4*>(out.residual + o + j);
+                        const uint32_t rr[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            float lo = dequant(static_cast<int>(v[j + 2 * e]) - xs, deq);
+                            float hi = dequant(static_cast<int>(v[j + 2 * e + 1]) - xs, deq);
+                            if (out.residual) {
+                                lo = __fadd_rn(bf16_bits_to_f32(rr[e] & 0xffffu), lo);
+                                hi = __fadd_rn(bf16_bits_to_f32(rr[e] >> 16), hi);
+                            }
+                            pk[e] = f32_to_bf16_bits(lo) | (static_cast<uint32_t>(f32_to_bf16_bits(hi)) << 16);
+                        }
+                        *reinterpret_cast<uint4*>(out.y + o + j) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                    }
+                }
+                if (out.acc) {
+#pragma unroll
+                    for (int j = 0; j < 32; j += 4)
+                        *reinterpret_cast<int4*>(out.acc + o + j) =
+                            make_int4(static_cast<int>(v[j]) - xs, static_cast<int>(v[j + 1]) - xs,
+                                      static_cast<int>(v[j + 2]) - xs, static_cast<int>(v[j + 3]) - xs);
+                }
+            } else {
+                for (int j = 0; j < 32 && nb + j < N; ++j) {
+                    const int a = static_cast<int>(v[j]) - xs;
+                    float f = dequant(a, deq);
+                    if (out.y32) {
+                        out.y32[o + j] = f;
+                    } else {
+                        if (out.residual) f = __fadd_rn(bf16_bits_to_f32(out.residual[o + j]), f);
+                        out.y[o + j] = f32_to_bf16_bits(f);
+                    }
+                    if (out.acc) out.acc[o + j] = a;
+                }
+            }
+        }
+    }
+
+    // ---------------------------------------------------------- teardown
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 1) {
+        if (lane == 0 && abort_sh) tc::mbar_wait(accf, 0, WAIT_LIMIT_NS);  // no MMA still writing TMEM
+        __syncwarp();
+        tc::fence_after_sync();
+        tc::tmem_dealloc(tmem, TMEM_COLS);
+    }
+}
+
+// ---------------------------------------------------------------- host side
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+        else
+            cudaGetLastError();
+    }
+    return fn;
+}
+
+// 2-D uint8 tensor map over [rows, cols] (cols contiguous), box [box_rows, box_cols].
+bool make_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows,
+              uint32_t box_cols, bool swizzle128) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {cols};
+    const cuuint32_t box[2] = {box_cols, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+bool gemm_tc_ok(int64_t N, int64_t K, const void* Wp, const void* xq) {
+    return N >= 1 && K % 64 == 0 && reinterpret_cast<uintptr_t>(Wp) % 16 == 0 &&
+           reinterpret_cast<uintptr_t>(xq) % 16 == 0;
+}
+
+cudaError_t launch_gemm_tc(const uint8_t* Wp, const float* gamma, int64_t N, int64_t K,
+                           const int8_t* xq_g16t, const float* scale, const int32_t* xsum, int64_t M,
+                           const GemvOut& out, cudaStream_t s) {
+    if (M == 0 || N == 0) return cudaSuccess;
+    CUtensorMap mapA, mapB;
+    if (!make_map(&mapA, xq_g16t, (uint64_t)M, (uint64_t)K, BM, BK, true) ||
+        !make_map(&mapB, Wp, (uint64_t)N, (uint64_t)(K / 4), BN, BK / 4, false))
+        return cudaErrorInvalidValue;
+    unsigned* err = nullptr;
+    cudaError_t e = device_error_word(&err);
+    if (e != cudaSuccess) return e;
+    static bool attr_set[64];
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 64 && !attr_set[dev]) {
+        e = cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        attr_set[dev] = true;
+    }
+    const dim3 grid((unsigned)((N + BN - 1) / BN), (unsigned)((M + BM - 1) / BM));
+    gemm_tc_kernel<<<grid, THREADS, SMEM_BYTES, s>>>(mapA, mapB, (int)M, (int)N, (int)K, gamma, scale,
+                                                     xsum, out, err);
+    return cudaGetLastError();
+}
+
+}  // namespace bl

@@ -155,6 +155,31 @@ def test_forward_ragged_shapes(cuda_device, M, N, K):
     check_forward_full(Wp, gamma, Wp_ref, g_ref, x, cuda_device)
 
 
+@pytest.mark.parametrize("M,N,K", [(129, 257, 64), (300, 512, 320), (33, 1000, 2560),
+                                   (4096, 256, 128), (17, 8, 64)])
+def test_forward_tensor_core_tails(cuda_device, M, N, K):
+    """M > 16 runs the tcgen05 GEMM: token, row and k-block tails, N not a
+    multiple of the 256-row tile, K not a multiple of the 128-code k-block."""
+    W = make_weights(N, K, 0.02, seed=M + 3 * N + K)
+    Wp, gamma, Wp_ref, g_ref = pack_both(W, cuda_device)
+    x = synth.activations(M, K, seed=N, outliers=True)
+    res = synth.activations(M, N, seed=K, outliers=False)
+    check_forward_full(Wp, gamma, Wp_ref, g_ref, x, cuda_device)
+    check_forward_full(Wp, gamma, Wp_ref, g_ref, x, cuda_device, residual=res)
+
+
+def test_forward_misaligned_input_takes_generic_path(cuda_device):
+    K, N, M = 256, 64, 20
+    W = make_weights(N, K, 0.02, seed=21)
+    Wp, gamma, Wp_ref, g_ref = pack_both(W, cuda_device)
+    xb = synth.activations(M, K + 1, seed=22, outliers=True)
+    x_dev = xb.to(cuda_device).reshape(-1)[1:1 + M * K].view(M, K)  # 2-byte aligned only
+    y, acc = bl.forward(Wp, gamma, x_dev, want_acc=True)
+    ref = oracle.forward(Wp_ref, g_ref, bits(x_dev))
+    assert np.array_equal(np_(acc), ref["acc"])
+    assert_bf16_exact(bits(y), ref["y"])
+
+
 def test_forward_residual_and_degenerate_tokens(cuda_device):
     K, N, M = 2560, 640, 6
     W = make_weights(N, K, 0.02, seed=5)
