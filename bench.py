@@ -497,6 +497,37 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+PROFILE_CASES = {
+    # name: (K, N, M) of one forward call; used for ncu captures of one kernel
+    "gemv_2b": (2560, 6912, 1),
+    "gemv_2b_m16": (2560, 6912, 16),
+    "gemv_100b": (8192, 28672, 1),
+    "gemm_2b": (2560, 6912, 4096),
+    "gemm_2b_down": (6912, 2560, 4096),
+}
+
+
+def run_profile_case(name: str, reps: int):
+    """Run one forward call `reps` times (after packing); for ncu -k/-s/-c."""
+    import torch
+
+    import bitlinear_w1_a8_02_b200 as bl
+    from bitlinear_w1_a8_02_b200 import synth
+
+    K, N, M = PROFILE_CASES[name]
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    sigma = synth.SIGMA_100B if K * N > 10 ** 8 else synth.SIGMA_2B
+    Wp, g = bl.pack_weights(synth.weights(N, K, sigma, seed=1, device=dev))
+    x = synth.activations(M, K, seed=2, device=dev)
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(bl.workspace_bytes(bl.BL_OP_FORWARD, M, N, K), dtype=torch.uint8, device=dev)
+    for _ in range(reps):
+        bl.forward(Wp, g, x, out=y, ws=ws)
+    torch.cuda.synchronize()
+    print(f"profile case {name}: K={K} N={N} M={M}, {reps} calls", flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -506,7 +537,13 @@ def main():
     ap.add_argument("--no-extras", action="store_true", help="skip the secondary workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--profile-case", choices=sorted(PROFILE_CASES),
+                    help="run one forward call repeatedly for an ncu capture, then exit")
+    ap.add_argument("--reps", type=int, default=5)
     args = ap.parse_args()
+    if args.profile_case:
+        run_profile_case(args.profile_case, args.reps)
+        return
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     if args.impl == "reference":

@@ -30,21 +30,30 @@
 namespace bl {
 namespace {
 
-constexpr int BM = 128;            // tokens per tile (TMEM lanes)
-constexpr int BN = 256;            // weight rows per tile (TMEM columns)
-constexpr int BK = 128;            // codes per k-block (one 128-byte swizzle row)
-constexpr int STAGES = 3;
-constexpr int A_BYTES = BM * BK;        // 16 KiB activation codes
-constexpr int BU_BYTES = BN * BK;       // 32 KiB unpacked weight codes
-constexpr int BP_BYTES = BN * BK / 4;   //  8 KiB packed weights
-constexpr int THREADS = 192;            // warp 0 TMA, warp 1 MMA, warps 2-5 unpack + epilogue
-constexpr int UNPACK_THREADS = 128;
-constexpr uint32_t TMEM_COLS = 256;
+constexpr int BM = 128;               // tokens per tile (TMEM lanes)
+constexpr int BN = 256;               // weight rows per tile (TMEM columns per accumulator)
+constexpr int BK = 128;               // codes per k-block (one 128-byte swizzle row)
+constexpr int TSTAGES = 6;            // TMA ring: activation codes + packed weights
+constexpr int USTAGES = 2;            // unpacked weight-code ring
+constexpr int A_BYTES = BM * BK;      // 16 KiB activation codes
+constexpr int P_BYTES = BN * BK / 4;  //  8 KiB packed weights
+constexpr int U_BYTES = BN * BK;      // 32 KiB unpacked weight codes
+#ifndef BL_GEMM_UNPACK_WARPS
+#define BL_GEMM_UNPACK_WARPS 4
+#endif
+constexpr int UNPACK_WARPS = BL_GEMM_UNPACK_WARPS;
+constexpr int UNPACK_THREADS = 32 * UNPACK_WARPS;
+constexpr int EPI_THREADS = 128;
+constexpr int THREADS = 64 + UNPACK_THREADS + EPI_THREADS;  // TMA, MMA, unpack, epilogue warps
+constexpr int UNPACK_VEC = BN * BK / 4 / 16 / UNPACK_THREADS;  // 16-byte packed groups per thread
+constexpr uint32_t TMEM_COLS = 2 * BN;  // two accumulators: epilogue of tile t overlaps tile t+1
 constexpr uint64_t WAIT_LIMIT_NS = 1000000000ull;
-constexpr size_t SMEM_BYTES = 1024 /*alignment slack*/ + STAGES * (A_BYTES + BU_BYTES + BP_BYTES) +
-                              256 /*barriers*/;
+constexpr int NUM_BARS = 2 * TSTAGES + 2 * USTAGES + 4;
+constexpr size_t SMEM_BYTES =
+    1024 /*alignment slack*/ + TSTAGES * (A_BYTES + P_BYTES) + USTAGES * U_BYTES + NUM_BARS * 8;
 
-static_assert(BN * BK / 4 / 4 % UNPACK_THREADS == 0, "unpack work must split evenly");
+static_assert(BN * BK / 4 / 16 % UNPACK_THREADS == 0, "unpack work must split evenly");
+static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 
 __device__ __forceinline__ bool aligned16(const void* p) {
     return (reinterpret_cast<uintptr_t>(p) & 15u) == 0;
@@ -55,6 +64,70 @@ __device__ __forceinline__ void report_timeout(unsigned* err, int* abort_flag) {
     atomicExch(abort_flag, 1);
 }
 
+__device__ __forceinline__ bool aborted(const int* abort_flag) {
+    return *reinterpret_cast<const volatile int*>(abort_flag) != 0;
+}
+
+// Dequantise and store 32 consecutive outputs of one row (one TMEM load).
+__device__ __forceinline__ void store_row_chunk(const uint32_t (&v)[32], int xs, float deq, int nb,
+                                                int N, size_t o, const GemvOut& out, bool vec) {
+    if (vec && nb + 32 <= N) {
+        if (out.y32) {
+#pragma unroll
+            for (int j = 0; j < 32; j += 4) {
+                float4 f;
+                f.x = dequant(static_cast<int>(v[j]) - xs, deq);
+                f.y = dequant(static_cast<int>(v[j + 1]) - xs, deq);
+                f.z = dequant(static_cast<int>(v[j + 2]) - xs, deq);
+                f.w = dequant(static_cast<int>(v[j + 3]) - xs, deq);
+                *reinterpret_cast<float4*>(out.y32 + o + j) = f;
+            }
+        } else {
+#pragma unroll
+            for (int j = 0; j < 32; j += 8) {
+                uint4 r = make_uint4(0, 0, 0, 0);
+                if (out.residual) r = *reinterpret_cast<const uint4*>(out.residual + o + j);
+                const uint32_t rr[4] = {r.x, r.y, r.z, r.w};
+                uint32_t pk[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    float lo = dequant(static_cast<int>(v[j + 2 * e]) - xs, deq);
+                    float hi = dequant(static_cast<int>(v[j + 2 * e + 1]) - xs, deq);
+                    if (out.residual) {
+                        lo = __fadd_rn(bf16_bits_to_f32(rr[e] & 0xffffu), lo);
+                        hi = __fadd_rn(bf16_bits_to_f32(rr[e] >> 16), hi);
+                    }
+                    pk[e] = f32_to_bf16_bits(lo) | (static_cast<uint32_t>(f32_to_bf16_bits(hi)) << 16);
+                }
+                *reinterpret_cast<uint4*>(out.y + o + j) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            }
+        }
+        if (out.acc) {
+#pragma unroll
+            for (int j = 0; j < 32; j += 4)
+                *reinterpret_cast<int4*>(out.acc + o + j) =
+                    make_int4(static_cast<int>(v[j]) - xs, static_cast<int>(v[j + 1]) - xs,
+                              static_cast<int>(v[j + 2]) - xs, static_cast<int>(v[j + 3]) - xs);
+        }
+    } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+            if (nb + j >= N) break;
+            const int a = static_cast<int>(v[j]) - xs;
+            float f = dequant(a, deq);
+            if (out.y32) {
+                out.y32[o + j] = f;
+            } else {
+                if (out.residual) f = __fadd_rn(bf16_bits_to_f32(out.residual[o + j]), f);
+                out.y[o + j] = f32_to_bf16_bits(f);
+            }
+            if (out.acc) out.acc[o + j] = a;
+        }
+    }
+}
+
+// Persistent CTAs walk the (m-tile, n-tile) grid with n fastest, so the CTAs in
+// flight share activation tiles and the whole packed weight stays in L2.
 __global__ void __launch_bounds__(THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    int M, int N, int K, const float* __restrict__ gamma_p,
@@ -66,27 +139,36 @@ __global__ void __launch_bounds__(THREADS, 1)
 
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
-    uint8_t* sA = smem;
-    uint8_t* sBu = sA + STAGES * A_BYTES;
-    uint8_t* sBp = sBu + STAGES * BU_BYTES;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(sBp + STAGES * BP_BYTES);
-    // bars[0..S): TMA landed; [S..2S): unpacked; [2S..3S): stage free; [3S]: accumulator done
-    auto full = [&](int s) { return tc::smem_u32(bars + s); };
-    auto ready = [&](int s) { return tc::smem_u32(bars + STAGES + s); };
-    auto empty = [&](int s) { return tc::smem_u32(bars + 2 * STAGES + s); };
-    const uint32_t accf = tc::smem_u32(bars + 3 * STAGES);
+    uint8_t* sA = smem;                         // TSTAGES x A_BYTES
+    uint8_t* sU = sA + TSTAGES * A_BYTES;       // USTAGES x U_BYTES
+    uint8_t* sP = sU + USTAGES * U_BYTES;       // TSTAGES x P_BYTES
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sP + TSTAGES * P_BYTES);
+    auto bar = [&](int i) { return tc::smem_u32(bars + i); };
+    auto tfull = [&](int s) { return bar(s); };                              // TMA landed
+    auto tempty = [&](int s) { return bar(TSTAGES + s); };                   // MMA done with it
+    auto ufull = [&](int u) { return bar(2 * TSTAGES + u); };                // unpacked
+    auto uempty = [&](int u) { return bar(2 * TSTAGES + USTAGES + u); };     // MMA done with it
+    auto afull = [&](int a) { return bar(2 * TSTAGES + 2 * USTAGES + a); };  // accumulator ready
+    auto aempty = [&](int a) { return bar(2 * TSTAGES + 2 * USTAGES + 2 + a); };  // drained
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int n0 = blockIdx.x * BN, m0 = blockIdx.y * BM;
+    const int n_tiles = (N + BN - 1) / BN;
+    const int num_tiles = n_tiles * ((M + BM - 1) / BM);
     const int nkb = (K + BK - 1) / BK;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < STAGES; ++s) {
-            tc::mbar_init(full(s), 1);
-            tc::mbar_init(ready(s), UNPACK_THREADS);
-            tc::mbar_init(empty(s), 1);
+        for (int s = 0; s < TSTAGES; ++s) {
+            tc::mbar_init(tfull(s), 1);
+            tc::mbar_init(tempty(s), 1);
         }
-        tc::mbar_init(accf, 1);
+        for (int u = 0; u < USTAGES; ++u) {
+            tc::mbar_init(ufull(u), UNPACK_THREADS);
+            tc::mbar_init(uempty(u), 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            tc::mbar_init(afull(a), 1);
+            tc::mbar_init(aempty(a), EPI_THREADS);
+        }
         abort_sh = 0;
         tc::fence_mbar_init();
     }
@@ -100,164 +182,157 @@ __global__ void __launch_bounds__(THREADS, 1)
     const uint32_t tmem = tmem_base_sh;
 
     if (warp == 0) {
-        // ---------------------------------------------------------- TMA producer
+        // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
             tc::prefetch_tmap(&tmA);
             tc::prefetch_tmap(&tmB);
-            int issued = 0;
-            for (int kb = 0; kb < nkb; ++kb) {
-                const int s = kb % STAGES;
-                const uint32_t ph = (kb / STAGES) & 1;
-                if (kb >= STAGES && !tc::mbar_wait(empty(s), ph ^ 1, WAIT_LIMIT_NS)) {
-                    report_timeout(err, &abort_sh);
-                    break;
+            uint32_t g = 0;
+            for (int tile = blockIdx.x; tile < num_tiles && !aborted(&abort_sh); tile += gridDim.x) {
+                const int m0 = (tile / n_tiles) * BM, n0 = (tile % n_tiles) * BN;
+                for (int kb = 0; kb < nkb; ++kb, ++g) {
+                    const int s = g % TSTAGES;
+                    if (g >= TSTAGES &&
+                        !tc::mbar_wait(tempty(s), ((g / TSTAGES) - 1) & 1, WAIT_LIMIT_NS)) {
+                        report_timeout(err, &abort_sh);
+                        break;
+                    }
+                    tc::mbar_arrive_expect_tx(tfull(s), A_BYTES + P_BYTES);
+                    tc::tma_load_2d(tc::smem_u32(sA + s * A_BYTES), &tmA, kb * BK, m0, tfull(s));
+                    tc::tma_load_2d(tc::smem_u32(sP + s * P_BYTES), &tmB, kb * (BK / 4), n0, tfull(s));
                 }
-                if (*(volatile int*)&abort_sh) break;
-                tc::mbar_arrive_expect_tx(full(s), A_BYTES + BP_BYTES);
-                tc::tma_load_2d(tc::smem_u32(sA + s * A_BYTES), &tmA, kb * BK, m0, full(s));
-                tc::tma_load_2d(tc::smem_u32(sBp + s * BP_BYTES), &tmB, kb * (BK / 4), n0, full(s));
-                issued = kb + 1;
             }
-            if (*(volatile int*)&abort_sh) {
-                // drain: let the copies still in flight land before the CTA exits
-                for (int kb = issued - STAGES < 0 ? 0 : issued - STAGES; kb < issued; ++kb)
-                    tc::mbar_wait(full(kb % STAGES), (kb / STAGES) & 1, WAIT_LIMIT_NS);
+            if (aborted(&abort_sh)) {
+                // let the copies still in flight land before the CTA exits
+                const uint32_t first = g > TSTAGES ? g - TSTAGES : 0;
+                for (uint32_t h = first; h < g; ++h)
+                    tc::mbar_wait(tfull(h % TSTAGES), (h / TSTAGES) & 1, WAIT_LIMIT_NS);
             }
         }
     } else if (warp == 1) {
-        // ---------------------------------------------------------- MMA issuer
+        // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             constexpr uint32_t idesc = tc::idesc_i8_s8u8(BM, BN);
-            for (int kb = 0; kb < nkb; ++kb) {
-                const int s = kb % STAGES;
-                const uint32_t ph = (kb / STAGES) & 1;
-                if (!tc::mbar_wait(ready(s), ph, WAIT_LIMIT_NS) ||
-                    !tc::mbar_wait(full(s), ph, WAIT_LIMIT_NS)) {
+            uint32_t g = 0, t = 0;
+            for (int tile = blockIdx.x; tile < num_tiles && !aborted(&abort_sh);
+                 tile += gridDim.x, ++t) {
+                const int a = t & 1;
+                if (t >= 2 && !tc::mbar_wait(aempty(a), ((t >> 1) - 1) & 1, WAIT_LIMIT_NS)) {
                     report_timeout(err, &abort_sh);
                     break;
                 }
                 tc::fence_after_sync();
-                const uint64_t ad = tc::desc_kmajor_sw128(tc::smem_u32(sA + s * A_BYTES));
-                const uint64_t bd = tc::desc_kmajor_sw128(tc::smem_u32(sBu + s * BU_BYTES));
+                const uint32_t d = tmem + a * BN;
+                bool ok = true;
+                for (int kb = 0; kb < nkb; ++kb, ++g) {
+                    const int s = g % TSTAGES, u = g % USTAGES;
+                    if (!tc::mbar_wait(ufull(u), (g / USTAGES) & 1, WAIT_LIMIT_NS) ||
+                        !tc::mbar_wait(tfull(s), (g / TSTAGES) & 1, WAIT_LIMIT_NS)) {
+                        report_timeout(err, &abort_sh);
+                        ok = false;
+                        break;
+                    }
+                    tc::fence_after_sync();
+                    const uint64_t ad = tc::desc_kmajor_sw128(tc::smem_u32(sA + s * A_BYTES));
+                    const uint64_t bd = tc::desc_kmajor_sw128(tc::smem_u32(sU + u * U_BYTES));
 #pragma unroll
-                for (int kk = 0; kk < BK / 32; ++kk)  // K = 32 bytes per MMA: +2 in 16-byte units
-                    tc::mma_i8(tmem, ad + 2 * kk, bd + 2 * kk, idesc, (kb | kk) != 0);
-                tc::mma_commit(empty(s));
+                    for (int kk = 0; kk < BK / 32; ++kk)  // 32 bytes of K per MMA: +2 in 16-byte units
+                        tc::mma_i8(d, ad + 2 * kk, bd + 2 * kk, idesc, (kb | kk) != 0);
+                    tc::mma_commit(tempty(s));
+                    tc::mma_commit(uempty(u));
+                }
+                if (!ok) break;
+                tc::mma_commit(afull(a));
             }
-            tc::mma_commit(accf);
+        }
+    } else if (warp < 2 + UNPACK_WARPS) {
+        // ------------------------------------------------------------ unpack
+        const int ut = threadIdx.x - 64;
+        uint32_t g = 0;
+        for (int tile = blockIdx.x; tile < num_tiles && !aborted(&abort_sh); tile += gridDim.x) {
+            bool ok = true;
+            for (int kb = 0; kb < nkb; ++kb, ++g) {
+                const int s = g % TSTAGES, u = g % USTAGES;
+                if (!tc::mbar_wait(tfull(s), (g / TSTAGES) & 1, WAIT_LIMIT_NS) ||
+                    (g >= USTAGES &&
+                     !tc::mbar_wait(uempty(u), ((g / USTAGES) - 1) & 1, WAIT_LIMIT_NS))) {
+                    report_timeout(err, &abort_sh);
+                    ok = false;
+                    break;
+                }
+                // Each thread owns UNPACK_VEC 16-byte groups of packed words; all of them are
+                // loaded before any store so the shared-memory latencies overlap. Group q
+                // holds words 4(q&1)..4(q&1)+3 of row q/2; the 16 codes of word j of row n
+                // go to 16-byte chunk j of that row, at swizzle position j ^ (n % 8).
+                const uint4* bp4 = reinterpret_cast<const uint4*>(sP + s * P_BYTES);
+                uint8_t* bu = sU + u * U_BYTES;
+                uint4 pw[UNPACK_VEC];
+#pragma unroll
+                for (int i = 0; i < UNPACK_VEC; ++i) pw[i] = bp4[ut + UNPACK_THREADS * i];
+#pragma unroll
+                for (int i = 0; i < UNPACK_VEC; ++i) {
+                    const int qg = ut + UNPACK_THREADS * i;
+                    const int n = qg >> 1, r = n & 7;
+                    uint8_t* rowp = bu + (n >> 3) * 1024 + r * 128;
+                    const uint32_t words[4] = {pw[i].x, pw[i].y, pw[i].z, pw[i].w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int j = 4 * (qg & 1) + e;
+                        const uint32_t wd = words[e];
+                        uint4 v;
+                        v.x = wd & 0x03030303u;
+                        v.y = (wd >> 2) & 0x03030303u;
+                        v.z = (wd >> 4) & 0x03030303u;
+                        v.w = (wd >> 6) & 0x03030303u;
+                        *reinterpret_cast<uint4*>(rowp + ((j ^ r) << 4)) = v;
+                    }
+                }
+                tc::fence_proxy_async_smem();
+                tc::mbar_arrive(ufull(u));
+            }
+            if (!ok) break;
         }
     } else {
-        // ---------------------------------------------------------- unpack
-        const int ut = threadIdx.x - 64;
-        bool ok = true;
-        for (int kb = 0; kb < nkb; ++kb) {
-            const int s = kb % STAGES;
-            const uint32_t ph = (kb / STAGES) & 1;
-            if (!tc::mbar_wait(full(s), ph, WAIT_LIMIT_NS)) {
-                report_timeout(err, &abort_sh);
-                ok = false;
-                break;
-            }
-            const uint32_t* bp = reinterpret_cast<const uint32_t*>(sBp + s * BP_BYTES);
-            uint8_t* bu = sBu + s * BU_BYTES;
-#pragma unroll
-            for (int i = 0; i < BN * 8 / UNPACK_THREADS; ++i) {
-                const int w = ut + UNPACK_THREADS * i;  // packed word w: row n, word j
-                const int n = w >> 3, j = w & 7;
-                const uint32_t word = bp[w];
-                uint4 v;
-                v.x = word & 0x03030303u;
-                v.y = (word >> 2) & 0x03030303u;
-                v.z = (word >> 4) & 0x03030303u;
-                v.w = (word >> 6) & 0x03030303u;
-                *reinterpret_cast<uint4*>(bu + (n >> 3) * 1024 + (n & 7) * 128 + ((j ^ (n & 7)) << 4)) = v;
-            }
-            tc::fence_proxy_async_smem();
-            tc::mbar_arrive(ready(s));
-        }
-        // ---------------------------------------------------------- epilogue
-        if (ok && !tc::mbar_wait(accf, 0, WAIT_LIMIT_NS)) {
-            report_timeout(err, &abort_sh);
-            ok = false;
-        }
-        ok = __all_sync(0xffffffffu, ok);  // tcgen05.ld below is warp-collective
-        tc::fence_after_sync();
-        const int q = warp & 3;  // TMEM lane quarter this warp may read
-        const int m = m0 + q * 32 + lane;
-        const bool mv = ok && m < M;
-        const float deq = mv ? __fdiv_rn(*gamma_p, scale[m]) : 0.0f;
-        const int xs = mv ? xsum[m] : 0;
+        // ------------------------------------------------------------ epilogue
+        const int q = warp & 3;  // the TMEM lane quarter this warp may read
+        const float gamma = *gamma_p;
         const bool vec = (N % 8 == 0) && aligned16(out.y) && aligned16(out.y32) &&
                          aligned16(out.residual) && aligned16(out.acc);
+        uint32_t t = 0;
+        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++t) {
+            const int a = t & 1;
+            bool ok = !aborted(&abort_sh) && tc::mbar_wait(afull(a), (t >> 1) & 1, WAIT_LIMIT_NS);
+            if (!__all_sync(0xffffffffu, ok)) {  // tcgen05.ld below is warp-collective
+                report_timeout(err, &abort_sh);
+                break;
+            }
+            tc::fence_after_sync();
+            const int m0 = (tile / n_tiles) * BM, n0 = (tile % n_tiles) * BN;
+            const int m = m0 + q * 32 + lane;
+            const bool mv = m < M;
+            const float deq = mv ? __fdiv_rn(gamma, scale[m]) : 0.0f;
+            const int xs = mv ? xsum[m] : 0;
 #pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
-            uint32_t v[32];
-            if (ok) {
-                tc::tmem_ld_32x32(tmem + (static_cast<uint32_t>(q * 32) << 16) + c * 32, v);
+            for (int c = 0; c < BN / 32; ++c) {
+                uint32_t v[32];
+                tc::tmem_ld_32x32(tmem + (static_cast<uint32_t>(q * 32) << 16) + a * BN + c * 32, v);
                 tc::tmem_ld_wait();
+                const int nb = n0 + c * 32;
+                if (mv && nb < N) store_row_chunk(v, xs, deq, nb, N, static_cast<size_t>(m) * N + nb, out, vec);
             }
-            const int nb = n0 + c * 32;
-            if (!mv || nb >= N) continue;
-            const size_t o = static_cast<size_t>(m) * N + nb;
-            if (vec && nb + 32 <= N) {
-                if (out.y32) {
-#pragma unroll
-                    for (int j = 0; j < 32; j += 4) {
-                        float4 f;
-                        f.x = dequant(static_cast<int>(v[j]) - xs, deq);
-                        f.y = dequant(static_cast<int>(v[j + 1]) - xs, deq);
-                        f.z = dequant(static_cast<int>(v[j + 2]) - xs, deq);
-                        f.w = dequant(static_cast<int>(v[j + 3]) - xs, deq);
-                        *reinterpret_cast<float4*>(out.y32 + o + j) = f;
-                    }
-                } else {
-#pragma unroll
-                    for (int j = 0; j < 32; j += 8) {
-                        uint32_t pk[4];
-                        uint4 r = make_uint4(0, 0, 0, 0);
-                        if (out.residual) r = *reinterpret_cast<const uint4*>(out.residual + o + j);
-                        const uint32_t rr[4] = {r.x, r.y, r.z, r.w};
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            float lo = dequant(static_cast<int>(v[j + 2 * e]) - xs, deq);
-                            float hi = dequant(static_cast<int>(v[j + 2 * e + 1]) - xs, deq);
-                            if (out.residual) {
-                                lo = __fadd_rn(bf16_bits_to_f32(rr[e] & 0xffffu), lo);
-                                hi = __fadd_rn(bf16_bits_to_f32(rr[e] >> 16), hi);
-                            }
-                            pk[e] = f32_to_bf16_bits(lo) | (static_cast<uint32_t>(f32_to_bf16_bits(hi)) << 16);
-                        }
-                        *reinterpret_cast<uint4*>(out.y + o + j) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                    }
-                }
-                if (out.acc) {
-#pragma unroll
-                    for (int j = 0; j < 32; j += 4)
-                        *reinterpret_cast<int4*>(out.acc + o + j) =
-                            make_int4(static_cast<int>(v[j]) - xs, static_cast<int>(v[j + 1]) - xs,
-                                      static_cast<int>(v[j + 2]) - xs, static_cast<int>(v[j + 3]) - xs);
-                }
-            } else {
-                for (int j = 0; j < 32 && nb + j < N; ++j) {
-                    const int a = static_cast<int>(v[j]) - xs;
-                    float f = dequant(a, deq);
-                    if (out.y32) {
-                        out.y32[o + j] = f;
-                    } else {
-                        if (out.residual) f = __fadd_rn(bf16_bits_to_f32(out.residual[o + j]), f);
-                        out.y[o + j] = f32_to_bf16_bits(f);
-                    }
-                    if (out.acc) out.acc[o + j] = a;
-                }
-            }
+            tc::fence_before_sync();
+            tc::mbar_arrive(aempty(a));
         }
     }
 
-    // ---------------------------------------------------------- teardown
+    // ------------------------------------------------------------ teardown
     tc::fence_before_sync();
     __syncthreads();
     if (warp == 1) {
-        if (lane == 0 && abort_sh) tc::mbar_wait(accf, 0, WAIT_LIMIT_NS);  // no MMA still writing TMEM
+        if (lane == 0 && abort_sh) {
+            // no MMA may still be writing TMEM when it is released
+            tc::mma_commit(afull(0));
+            tc::mbar_wait(afull(0), 0, WAIT_LIMIT_NS);
+        }
         __syncwarp();
         tc::fence_after_sync();
         tc::tmem_dealloc(tmem, TMEM_COLS);
@@ -327,7 +402,14 @@ cudaError_t launch_gemm_tc(const uint8_t* Wp, const float* gamma, int64_t N, int
         if (e != cudaSuccess) return e;
         attr_set[dev] = true;
     }
-    const dim3 grid((unsigned)((N + BN - 1) / BN), (unsigned)((M + BM - 1) / BM));
+    static int num_sms[64];
+    if (dev < 64 && !num_sms[dev]) {
+        e = cudaDeviceGetAttribute(&num_sms[dev], cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return e;
+    }
+    const int64_t tiles = ((N + BN - 1) / BN) * ((M + BM - 1) / BM);
+    const int sms = dev < 64 ? num_sms[dev] : 148;
+    const unsigned grid = (unsigned)(tiles < sms ? tiles : sms);
     gemm_tc_kernel<<<grid, THREADS, SMEM_BYTES, s>>>(mapA, mapB, (int)M, (int)N, (int)K, gamma, scale,
                                                      xsum, out, err);
     return cudaGetLastError();
