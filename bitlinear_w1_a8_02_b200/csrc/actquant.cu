@@ -50,6 +50,8 @@ __global__ void __launch_bounds__(kThreads) act_quant_vec_kernel(const uint16_t*
                                                                   int32_t* __restrict__ xsum) {
     __shared__ float fscratch[kWarps];
     __shared__ int iscratch[kWarps];
+    grid_dependency_wait();
+    grid_dependents_launch();
     const int m = blockIdx.x;
     const uint4* xr = reinterpret_cast<const uint4*>(x + (size_t)m * K);
     const int nvec = K / 8;
@@ -108,6 +110,8 @@ __global__ void __launch_bounds__(kThreads) act_quant_scalar_kernel(const uint16
                                                                      int32_t* __restrict__ xsum) {
     __shared__ float fscratch[kWarps];
     __shared__ int iscratch[kWarps];
+    grid_dependency_wait();
+    grid_dependents_launch();
     const int m = blockIdx.x;
     const uint16_t* xr = x + (size_t)m * K;
     float amax = 0.0f;
@@ -135,15 +139,17 @@ cudaError_t launch_act_quant(const uint16_t* x, int64_t M, int64_t K, int layout
     const bool vec = (K % 16 == 0) && ((uintptr_t)x % 16 == 0) && ((uintptr_t)xq % 16 == 0);
     if (!vec) {
         if (layout != XQ_NATURAL) return cudaErrorInvalidValue;
-        act_quant_scalar_kernel<<<(unsigned)M, kThreads, 0, s>>>(x, (int)K, xq, scale, xsum);
-    } else if (layout == XQ_NATURAL) {
-        act_quant_vec_kernel<XQ_NATURAL><<<(unsigned)M, kThreads, 0, s>>>(x, (int)K, xq, scale, xsum);
-    } else if (layout == XQ_PLANES) {
-        act_quant_vec_kernel<XQ_PLANES><<<(unsigned)M, kThreads, 0, s>>>(x, (int)K, xq, scale, xsum);
-    } else {
-        act_quant_vec_kernel<XQ_G16T><<<(unsigned)M, kThreads, 0, s>>>(x, (int)K, xq, scale, xsum);
+        return launch_pdl(act_quant_scalar_kernel, dim3((unsigned)M), dim3(kThreads), 0, s, x, (int)K,
+                          xq, scale, xsum);
     }
-    return cudaGetLastError();
+    if (layout == XQ_NATURAL)
+        return launch_pdl(act_quant_vec_kernel<XQ_NATURAL>, dim3((unsigned)M), dim3(kThreads), 0, s, x,
+                          (int)K, xq, scale, xsum);
+    if (layout == XQ_PLANES)
+        return launch_pdl(act_quant_vec_kernel<XQ_PLANES>, dim3((unsigned)M), dim3(kThreads), 0, s, x,
+                          (int)K, xq, scale, xsum);
+    return launch_pdl(act_quant_vec_kernel<XQ_G16T>, dim3((unsigned)M), dim3(kThreads), 0, s, x, (int)K,
+                      xq, scale, xsum);
 }
 
 }  // namespace bl

@@ -203,11 +203,13 @@ BL_API bl_status bitlinear_forward(const uint8_t* Wp, const float* gamma, int64_
     int32_t* xsum = (int32_t*)(base + w.xsum);
 
     const Path path = choose_path(Wp, N, K, M, xq, x);
-    BL_TRY(bl::launch_act_quant(x, M, K, layout_of(path), xq, scale, xsum, s));
     bl::GemvOut out;
     out.y = y;
     out.residual = residual;
     out.acc = acc;
+    if (path == Path::GemvFast && bl::gemv_fused_ok(M, K))  // one kernel: quantise + GEMV
+        return cuda_status(bl::launch_gemv(Wp, gamma, N, K, nullptr, nullptr, nullptr, M, out, s, x));
+    BL_TRY(bl::launch_act_quant(x, M, K, layout_of(path), xq, scale, xsum, s));
     return project(path, Wp, gamma, N, K, xq, scale, xsum, M, out, s);
 }
 
@@ -241,13 +243,18 @@ BL_API bl_status bitlinear_ffn(const uint8_t* Wg, const float* gg, const uint8_t
     Path up = choose_path(Wg, f, d, M, xq, x);
     if (choose_path(Wu, f, d, M, xq, x) != up) up = Path::GemvGeneric;
     const Path down = choose_path(Wd, d, f, M, q2, nullptr);
-    BL_TRY(bl::launch_act_quant(x, M, d, layout_of(up), xq, scale, xsum, s));
     bl::GemvOut og;
     og.y32 = g;
-    if (bl_status st = project(up, Wg, gg, f, d, xq, scale, xsum, M, og, s)) return st;
     bl::GemvOut ou;
     ou.y32 = u;
-    if (bl_status st = project(up, Wu, gu, f, d, xq, scale, xsum, M, ou, s)) return st;
+    if (up == Path::GemvFast && bl::gemv_fused_ok(M, d)) {
+        BL_TRY(bl::launch_gemv(Wg, gg, f, d, nullptr, nullptr, nullptr, M, og, s, x));
+        BL_TRY(bl::launch_gemv(Wu, gu, f, d, nullptr, nullptr, nullptr, M, ou, s, x));
+    } else {
+        BL_TRY(bl::launch_act_quant(x, M, d, layout_of(up), xq, scale, xsum, s));
+        if (bl_status st = project(up, Wg, gg, f, d, xq, scale, xsum, M, og, s)) return st;
+        if (bl_status st = project(up, Wu, gu, f, d, xq, scale, xsum, M, ou, s)) return st;
+    }
     BL_TRY(bl::launch_ffn_finalise(g, u, M, f, layout_of(down), q2, s2, xsum2, s));
     bl::GemvOut od;
     od.y = y;

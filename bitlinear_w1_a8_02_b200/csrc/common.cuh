@@ -34,10 +34,18 @@ __device__ __forceinline__ uint16_t f32_to_bf16_bits(float f) {
 }
 
 // Quantise one value with scale s: clip(rint(x * s), -128, 127).
+//
+// Rounding by magic-number addition: for |v| < 2^22, fp32 v + 1.5 * 2^23 lies in
+// [2^23, 2^24), where the spacing of fp32 values is exactly 1, so the IEEE
+// round-to-nearest-even of that one addition is rint(v) (ties to even) and the
+// integer sits in the low mantissa bits: bits(v + 1.5 * 2^23) = 0x4B400000 + rint(v).
+// The per-token scale guarantees |x * s| <= 127 * (1 + 2^-23), so the bound holds
+// and the clip to [-128, 127] can never bite; it stays for non-finite inputs.
+// This avoids the reduced-rate float-to-int conversion pipe.
 __device__ __forceinline__ int quant_code(float x, float s) {
-    float r = rintf(__fmul_rn(x, s));
-    r = fminf(fmaxf(r, -128.0f), 127.0f);
-    return (int)r;
+    const float t = __fadd_rn(__fmul_rn(x, s), 12582912.0f);
+    const int q = static_cast<int>(__float_as_uint(t)) - 0x4B400000;
+    return min(max(q, -128), 127);
 }
 
 // Dequantise: y32 = float(acc) * (gamma / s).
@@ -97,6 +105,33 @@ __device__ __forceinline__ uint4 ld_stream16(const void* p) {
 // 16-byte read-only load through L1 (activation codes, reused by many warps).
 __device__ __forceinline__ uint4 ld_nc16(const void* p) {
     return __ldg(reinterpret_cast<const uint4*>(p));
+}
+
+// Programmatic dependent launch: the kernel may start while the previous kernel
+// in the stream is still running; it must call griddepcontrol.wait before it
+// reads anything that kernel may write and before its first global store.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t s, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
+__device__ __forceinline__ void grid_dependency_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+__device__ __forceinline__ void grid_dependents_launch() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 }  // namespace bl

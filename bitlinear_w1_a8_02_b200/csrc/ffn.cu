@@ -28,6 +28,8 @@ __global__ void __launch_bounds__(kThreads) ffn_finalise_kernel(const float* __r
     __shared__ double dscratch[kWarps];
     __shared__ float fscratch[kWarps];
     __shared__ int iscratch[kWarps];
+    grid_dependency_wait();
+    grid_dependents_launch();
     const int m = blockIdx.x;
     const float* gr = g + (size_t)m * f;
     const float* ur = u + (size_t)m * f;
@@ -97,8 +99,8 @@ cudaError_t launch_fin(const float* g, const float* u, int64_t M, int64_t f, int
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
     }
-    ffn_finalise_kernel<LAYOUT><<<(unsigned)M, kThreads, smem, s>>>(g, u, (int)f, q2, s2, xsum2);
-    return cudaGetLastError();
+    return launch_pdl(ffn_finalise_kernel<LAYOUT>, dim3((unsigned)M), dim3(kThreads), smem, s, g, u,
+                      (int)f, q2, s2, xsum2);
 }
 
 }  // namespace

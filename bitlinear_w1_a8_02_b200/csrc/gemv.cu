@@ -16,9 +16,21 @@
 // is laid out in PLANES (plane i holds xq[4j + i] at byte j), so a field of a
 // weight word and a word of plane i cover the same k.
 //
-// Work split: one CTA per 16 output rows (and per group of 8*NT tokens); its 8
-// warps split K in 64-byte column chunks; partial sums meet in shared memory and
-// the dequantisation epilogue is fused.
+// Work split: persistent CTAs walk tiles of 16 output rows; the 8 warps of a CTA
+// split K in 64-byte column chunks, partial sums meet in shared memory and the
+// dequantisation epilogue is fused. Each CTA asks the TMA engine to prefetch the
+// weight rows of the tiles it will reach next into L2, so DRAM streams
+// continuously while the warps work on the current tile.
+//
+// Fused activation quantisation: when the codes of all M tokens fit in shared
+// memory, each CTA quantises x itself (absmax per token, then PLANES codes into
+// shared memory), so a forward call is one kernel. Otherwise the codes come from
+// the act-quant kernel through the workspace.
+//
+// Programmatic dependent launch: before waiting for the previous kernel in the
+// stream (griddepcontrol.wait) a CTA only issues L2 prefetches of its weights,
+// which cannot observe stale data (L2 is the point of coherence); every global
+// load of other data and every store comes after the wait.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -28,6 +40,14 @@ namespace {
 constexpr int kWarps = 8;
 constexpr int kThreads = 32 * kWarps;
 constexpr int kUnroll = 4;
+constexpr int kPrefetchAhead = 2;          // tiles of lookahead per CTA
+constexpr int kFusedSmemLimit = 48 * 1024;  // codes of all tokens in shared memory
+constexpr int kFusedMaxTokens = 4;          // beyond this the separate quantiser is faster
+
+
+__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
 
 __device__ __forceinline__ void mma_u8s8(int (&d)[4], unsigned a0, unsigned a1, unsigned a2,
                                          unsigned a3, unsigned b0, unsigned b1) {
@@ -56,105 +76,290 @@ __device__ __forceinline__ void chunk_mma(int (&acc)[NT][4][4], const uint4& wa,
     }
 }
 
-template <int NT>
-__device__ __forceinline__ void load_x(uint4 (&xv)[NT][4], const int8_t* const (&xbase)[NT],
-                                       const bool (&tv)[NT], int64_t KB, int off) {
+struct GemvArgs {
+    const uint8_t* Wp;
+    const float* gamma;
+    int N, KB, M;
+    const uint16_t* x;     // bf16 input (fused quantisation)
+    const int8_t* Xp;      // PLANES codes (not fused)
+    const float* scale;    // [M] (not fused)
+    const int32_t* xsum;   // [M] (not fused)
+    GemvOut out;
+};
+
+// Byte offset of plane i of token m in the fused shared-memory code buffer. The
+// +64 per token keeps the tokens of one quarter-warp on different banks.
+__device__ __forceinline__ int smem_plane_off(int m, int i, int KB) { return m * (4 * KB + 64) + i * KB; }
+
+// Quantise the M tokens of x into shared-memory PLANES codes (all threads).
+// Thread q handles 16-element groups q, q + 256, ...; the first kRegGroups of them
+// stay in registers between the absmax pass and the code pass, so x is read once.
+constexpr int kRegGroups = 4;
+
+template <int TOK>
+__device__ __forceinline__ void fold_absmax(float (&am)[TOK], int m, uint4 v0, uint4 v1) {
+    const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+    float r = 0.0f;
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
+    for (int e = 0; e < 8; ++e) {
+        r = fmaxf(r, fabsf(__uint_as_float(w[e] << 16)));
+        r = fmaxf(r, fabsf(__uint_as_float(w[e] & 0xffff0000u)));
+    }
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-            xv[nt][i] = tv[nt] ? ld_nc16(xbase[nt] + i * KB + off) : make_uint4(0, 0, 0, 0);
+    for (int mm = 0; mm < TOK; ++mm)
+        if (mm == m) am[mm] = fmaxf(am[mm], r);
+}
+
+// Returns the sum of the 16 codes (accumulated per token by the caller).
+__device__ __forceinline__ int quantise_group(uint8_t* codes, int KB, int m, int c, uint4 v0, uint4 v1,
+                                              float s) {
+    const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+    unsigned pw[4] = {0u, 0u, 0u, 0u};
+    int sum = 0;
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+        const float f = (e & 1) ? __uint_as_float(w[e >> 1] & 0xffff0000u) : __uint_as_float(w[e >> 1] << 16);
+        const int q = quant_code(f, s);
+        sum += q;
+        pw[e & 3] |= static_cast<unsigned>(q & 255) << (8 * (e >> 2));
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) *reinterpret_cast<unsigned*>(codes + smem_plane_off(m, i, KB) + 4 * c) = pw[i];
+    return sum;
+}
+
+template <int TOK>
+__device__ __forceinline__ void add_to_token(int (&xs)[TOK], int m, int v) {
+#pragma unroll
+    for (int mm = 0; mm < TOK; ++mm)
+        if (mm == m) xs[mm] += v;
+}
+
+// Phase 1: load this thread's first kRegGroups groups of x into registers.
+struct XRegs {
+    uint4 v[kRegGroups][2];
+};
+
+__device__ __forceinline__ void fused_load(const uint16_t* __restrict__ x, int M, int KB, XRegs& xr) {
+    const int total = M * (KB / 4);
+    const uint4* xv = reinterpret_cast<const uint4*>(x);  // token m, group c at 2 * (m * groups + c)
+#pragma unroll
+    for (int j = 0; j < kRegGroups; ++j) {
+        const int q = threadIdx.x + kThreads * j;
+        if (q < total) {
+            xr.v[j][0] = xv[2 * q];
+            xr.v[j][1] = xv[2 * q + 1];
+        }
     }
 }
 
-template <int NT>
-__global__ void __launch_bounds__(kThreads) gemv_mma_kernel(
-    const uint8_t* __restrict__ Wp, const float* __restrict__ gamma_p, int N, int KB,
-    const int8_t* __restrict__ Xp, const float* __restrict__ scale, const int32_t* __restrict__ xsum,
-    int M, GemvOut out) {
-    constexpr int TOK = 8 * NT;
-    __shared__ int red[kWarps][16][TOK];
+// Phase 2: per-token absmax, scale, then PLANES codes into shared memory.
+template <int TOK>
+__device__ void fused_quantise(const uint16_t* __restrict__ x, int M, int KB, const XRegs& xr,
+                               uint8_t* codes, float* s_sh, int* xs_sh, float (*am_sh)[TOK]) {
+    const int groups = KB / 4;  // 16-element groups per token
+    const int total = M * groups;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint4* xv = reinterpret_cast<const uint4*>(x);
+    float am[TOK];
+#pragma unroll
+    for (int mm = 0; mm < TOK; ++mm) am[mm] = 0.0f;
+    for (int q = threadIdx.x + kThreads * kRegGroups; q < total; q += kThreads)
+        fold_absmax<TOK>(am, q / groups, xv[2 * q], xv[2 * q + 1]);
+#pragma unroll
+    for (int j = 0; j < kRegGroups; ++j) {
+        const int q = threadIdx.x + kThreads * j;
+        if (q < total) fold_absmax<TOK>(am, q / groups, xr.v[j][0], xr.v[j][1]);
+    }
+#pragma unroll
+    for (int mm = 0; mm < TOK; ++mm) {
+        if (mm < M) {
+            const float r = warp_max(am[mm]);
+            if (lane == 0) am_sh[warp][mm] = r;
+        }
+    }
+    if (threadIdx.x < TOK) xs_sh[threadIdx.x] = 0;
+    __syncthreads();
+    if (threadIdx.x < M) {
+        float r = am_sh[0][threadIdx.x];
+#pragma unroll
+        for (int w = 1; w < kWarps; ++w) r = fmaxf(r, am_sh[w][threadIdx.x]);
+        s_sh[threadIdx.x] = __fdiv_rn(kActRange, fmaxf(r, kActEps));
+    }
+    __syncthreads();
+    // code sums: per-thread partials per token, a warp reduction, one atomic per warp
+    int xs[TOK];
+#pragma unroll
+    for (int mm = 0; mm < TOK; ++mm) xs[mm] = 0;
+#pragma unroll
+    for (int j = 0; j < kRegGroups; ++j) {
+        const int q = threadIdx.x + kThreads * j;
+        if (q < total) {
+            const int m = q / groups;
+            add_to_token<TOK>(xs, m, quantise_group(codes, KB, m, q - m * groups, xr.v[j][0], xr.v[j][1], s_sh[m]));
+        }
+    }
+    for (int q = threadIdx.x + kThreads * kRegGroups; q < total; q += kThreads) {
+        const int m = q / groups;
+        add_to_token<TOK>(xs, m, quantise_group(codes, KB, m, q - m * groups, xv[2 * q], xv[2 * q + 1], s_sh[m]));
+    }
+#pragma unroll
+    for (int mm = 0; mm < TOK; ++mm) {
+        if (mm < M) {
+            const int r = warp_sum(xs[mm]);
+            if (lane == 0) atomicAdd(&xs_sh[mm], r);
+        }
+    }
+}
 
+template <int NT, bool FUSED>
+__global__ void __launch_bounds__(kThreads) gemv_mma_kernel(const GemvArgs a) {
+    constexpr int TOK = 8 * NT;
+    constexpr int CPP = kWarps * kUnroll;  // chunks per pass of the whole CTA
+    extern __shared__ __align__(16) uint8_t codes[];  // fused: PLANES codes of the M tokens
+    __shared__ int red[kWarps][16][TOK];
+    __shared__ float s_sh[TOK];
+    __shared__ int xs_sh[TOK];
+    __shared__ float am_sh[kWarps][TOK];
+
+    const int N = a.N, KB = a.KB;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, t = lane & 3;
-    const int n0 = blockIdx.x * 16;
-    const int tok0 = blockIdx.y * TOK;
+    const int ntiles = (N + 15) >> 4;
     const int nchunks = KB >> 6;
+    const int npass = (nchunks + CPP - 1) / CPP;
+    const int tok0 = blockIdx.y * TOK;
 
-    const int rowA = min(n0 + g, N - 1), rowB = min(n0 + g + 8, N - 1);
-    const uint8_t* pA = Wp + (size_t)rowA * KB + 16 * t;
-    const uint8_t* pB = Wp + (size_t)rowB * KB + 16 * t;
+    auto tile_prefetch = [&](int tile) {
+        const int n0 = tile * 16;
+        const int rows = min(16, N - n0);
+        prefetch_l2(a.Wp + (size_t)n0 * KB, (uint32_t)(rows * KB));
+    };
+    if (threadIdx.x == 0) {
+        for (int p = 0; p < kPrefetchAhead; ++p) {
+            const int tile = blockIdx.x + p * gridDim.x;
+            if (tile < ntiles) tile_prefetch(tile);
+        }
+    }
+    // weight registers of one pass: chunk warp + kWarps * (kUnroll * pass + u)
+    uint4 wa[kUnroll], wb[kUnroll];
+    auto issue = [&](int tile, int pass) {
+        const int n0 = tile * 16;
+        const uint8_t* pA = a.Wp + (size_t)min(n0 + g, N - 1) * KB + 16 * t;
+        const uint8_t* pB = a.Wp + (size_t)min(n0 + g + 8, N - 1) * KB + 16 * t;
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const int c = warp + kWarps * (kUnroll * pass + u);
+            if (c < nchunks) {
+                wa[u] = ld_stream16(pA + 64 * c);
+                wb[u] = ld_stream16(pB + 64 * c);
+            }
+        }
+    };
+    grid_dependents_launch();
+    grid_dependency_wait();
 
-    const int8_t* xbase[NT];
+    // x first, then the first pass of the first tile: both loads are in flight
+    // while x is quantised
+    XRegs xr;
+    if (FUSED) fused_load(a.x, a.M, KB, xr);
+    if ((int)blockIdx.x < ntiles) issue(blockIdx.x, 0);
+
+    if (FUSED) {
+        fused_quantise<TOK>(a.x, a.M, KB, xr, codes, s_sh, xs_sh, am_sh);
+    } else if (threadIdx.x < TOK && tok0 + (int)threadIdx.x < a.M) {
+        s_sh[threadIdx.x] = a.scale[tok0 + threadIdx.x];
+        xs_sh[threadIdx.x] = a.xsum[tok0 + threadIdx.x];
+    }
+    __syncthreads();
+
+    // this lane's activation operand: token 8*nt + g of the group
+    const uint8_t* xbase[NT];
     bool tv[NT];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
         const int tok = tok0 + 8 * nt + g;
-        tv[nt] = tok < M;
-        xbase[nt] = Xp + (size_t)(tv[nt] ? tok : 0) * 4 * KB + 16 * t;
+        tv[nt] = tok < a.M;
+        if (FUSED)
+            xbase[nt] = codes + smem_plane_off(tv[nt] ? tok : 0, 0, KB) + 16 * t;
+        else
+            xbase[nt] = reinterpret_cast<const uint8_t*>(a.Xp) + (size_t)(tv[nt] ? tok : 0) * 4 * KB + 16 * t;
     }
+    auto load_x = [&](uint4 (&xv)[NT][4], int off) {
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                if (!tv[nt]) {
+                    xv[nt][i] = make_uint4(0, 0, 0, 0);
+                } else if (FUSED) {
+                    xv[nt][i] = *reinterpret_cast<const uint4*>(xbase[nt] + i * KB + off);
+                } else {
+                    xv[nt][i] = ld_nc16(xbase[nt] + i * KB + off);
+                }
+            }
+    };
 
-    int acc[NT][4][4];
+    const float gamma = *a.gamma;
+    for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+        if (threadIdx.x == 0) {
+            const int ahead = tile + kPrefetchAhead * gridDim.x;
+            if (ahead < ntiles) tile_prefetch(ahead);
+        }
+        const int n0 = tile * 16;
+        int acc[NT][4][4];
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
+        for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
+            for (int i = 0; i < 4; ++i)
 #pragma unroll
-            for (int e = 0; e < 4; ++e) acc[nt][i][e] = 0;
+                for (int e = 0; e < 4; ++e) acc[nt][i][e] = 0;
 
-    int c = warp;
-    for (; c + kWarps * (kUnroll - 1) < nchunks; c += kWarps * kUnroll) {
-        uint4 wa[kUnroll], wb[kUnroll];
+        for (int pass = 0; pass < npass; ++pass) {
+            if (tile != (int)blockIdx.x || pass != 0) issue(tile, pass);
 #pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            wa[u] = ld_stream16(pA + 64 * (c + kWarps * u));
-            wb[u] = ld_stream16(pB + 64 * (c + kWarps * u));
+            for (int u = 0; u < kUnroll; ++u) {
+                const int c = warp + kWarps * (kUnroll * pass + u);
+                if (c < nchunks) {
+                    uint4 xv[NT][4];
+                    load_x(xv, 64 * c);
+                    chunk_mma<NT>(acc, wa[u], wb[u], xv);
+                }
+            }
         }
-#pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            uint4 xv[NT][4];
-            load_x<NT>(xv, xbase, tv, KB, 64 * (c + kWarps * u));
-            chunk_mma<NT>(acc, wa[u], wb[u], xv);
-        }
-    }
-    for (; c < nchunks; c += kWarps) {
-        const uint4 wa = ld_stream16(pA + 64 * c), wb = ld_stream16(pB + 64 * c);
-        uint4 xv[NT][4];
-        load_x<NT>(xv, xbase, tv, KB, 64 * c);
-        chunk_mma<NT>(acc, wa, wb, xv);
-    }
 
-    // Fold the four field accumulators; D element e sits at row g + 8*(e >> 1),
-    // token 8*nt + 2t + (e & 1).
+        // Fold the four field accumulators; D element e sits at row g + 8*(e >> 1),
+        // token 8*nt + 2t + (e & 1).
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
+        for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const int v = acc[nt][0][e] + (acc[nt][1][e] >> 2) + (acc[nt][2][e] >> 4) +
-                          (acc[nt][3][e] >> 6);
-            red[warp][g + 8 * (e >> 1)][8 * nt + 2 * t + (e & 1)] = v;
-        }
-    __syncthreads();
+            for (int e = 0; e < 4; ++e) {
+                const int v = acc[nt][0][e] + (acc[nt][1][e] >> 2) + (acc[nt][2][e] >> 4) +
+                              (acc[nt][3][e] >> 6);
+                red[warp][g + 8 * (e >> 1)][8 * nt + 2 * t + (e & 1)] = v;
+            }
+        __syncthreads();
 
-    const float gamma = *gamma_p;
-    for (int idx = threadIdx.x; idx < 16 * TOK; idx += kThreads) {
-        const int r = idx & 15, cl = idx >> 4;
-        const int n = n0 + r, m = tok0 + cl;
-        if (n >= N || m >= M) continue;
-        int sum = 0;
+        for (int idx = threadIdx.x; idx < 16 * TOK; idx += kThreads) {
+            const int r = idx & 15, cl = idx >> 4;
+            const int n = n0 + r, m = tok0 + cl;
+            if (n >= N || m >= a.M) continue;
+            int sum = 0;
 #pragma unroll
-        for (int w = 0; w < kWarps; ++w) sum += red[w][r][cl];
-        const int a = sum - xsum[m];
-        const float deq = __fdiv_rn(gamma, scale[m]);
-        float v = dequant(a, deq);
-        const size_t o = (size_t)m * N + n;
-        if (out.y32) {
-            out.y32[o] = v;
-        } else {
-            if (out.residual) v = __fadd_rn(bf16_bits_to_f32(out.residual[o]), v);
-            out.y[o] = f32_to_bf16_bits(v);
+            for (int w = 0; w < kWarps; ++w) sum += red[w][r][cl];
+            const int accv = sum - xs_sh[cl];
+            const float deq = __fdiv_rn(gamma, s_sh[cl]);
+            float v = dequant(accv, deq);
+            const size_t o = (size_t)m * N + n;
+            if (a.out.y32) {
+                a.out.y32[o] = v;
+            } else {
+                if (a.out.residual) v = __fadd_rn(bf16_bits_to_f32(a.out.residual[o]), v);
+                a.out.y[o] = f32_to_bf16_bits(v);
+            }
+            if (a.out.acc) a.out.acc[o] = accv;
         }
-        if (out.acc) out.acc[o] = a;
+        __syncthreads();
     }
 }
 
@@ -162,6 +367,7 @@ __global__ void __launch_bounds__(kThreads) gemv_mma_kernel(
 __global__ void __launch_bounds__(kThreads) gemv_generic_kernel(
     const uint8_t* __restrict__ Wp, const float* __restrict__ gamma_p, int N, int K,
     const int8_t* __restrict__ Xn, const float* __restrict__ scale, int M, GemvOut out) {
+    grid_dependency_wait();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n = blockIdx.x * kWarps + warp;
     const int m = blockIdx.y;
@@ -169,16 +375,16 @@ __global__ void __launch_bounds__(kThreads) gemv_generic_kernel(
     const int KB = K / 4;
     const uint8_t* wr = Wp + (size_t)n * KB;
     const int8_t* xr = Xn + (size_t)m * K;
-    int a = 0;
+    int acc = 0;
     for (int j = lane; j < KB; j += 32) {
         const unsigned b = wr[j];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) a += ((int)((b >> (2 * i)) & 3u) - 1) * (int)xr[4 * j + i];
+        for (int i = 0; i < 4; ++i) acc += ((int)((b >> (2 * i)) & 3u) - 1) * (int)xr[4 * j + i];
     }
-    a = warp_sum(a);
+    acc = warp_sum(acc);
     if (lane == 0) {
         const float deq = __fdiv_rn(*gamma_p, scale[m]);
-        float v = dequant(a, deq);
+        float v = dequant(acc, deq);
         const size_t o = (size_t)m * N + n;
         if (out.y32) {
             out.y32[o] = v;
@@ -186,29 +392,74 @@ __global__ void __launch_bounds__(kThreads) gemv_generic_kernel(
             if (out.residual) v = __fadd_rn(bf16_bits_to_f32(out.residual[o]), v);
             out.y[o] = f32_to_bf16_bits(v);
         }
-        if (out.acc) out.acc[o] = a;
+        if (out.acc) out.acc[o] = acc;
     }
+}
+
+int sm_count() {
+    static int cached[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    if (dev < 64 && cached[dev]) return cached[dev];
+    int n = 148;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) n = 148;
+    if (dev < 64) cached[dev] = n;
+    return n;
+}
+
+template <int NT, bool FUSED>
+cudaError_t launch_variant(const GemvArgs& a, dim3 grid, size_t smem, cudaStream_t s) {
+    auto kern = gemv_mma_kernel<NT, FUSED>;
+    if (FUSED) {
+        // static + dynamic shared memory may pass the 48 KiB default: opt in once per device
+        static bool done[64];
+        int dev = 0;
+        cudaGetDevice(&dev);
+        if (dev >= 64 || !done[dev]) {
+            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 kFusedSmemLimit);
+            if (e != cudaSuccess) return e;
+            if (dev < 64) done[dev] = true;
+        }
+    }
+    return launch_pdl(kern, grid, dim3(kThreads), smem, s, a);
 }
 
 }  // namespace
 
 bool gemv_fast_ok(int64_t N, int64_t K) { return N >= 1 && K % 256 == 0; }
 
+bool gemv_fused_ok(int64_t M, int64_t K) {
+    return M >= 1 && M <= kFusedMaxTokens && (size_t)M * (K + 64) <= (size_t)kFusedSmemLimit;
+}
+
 cudaError_t launch_gemv(const uint8_t* Wp, const float* gamma, int64_t N, int64_t K,
                         const int8_t* Xp, const float* scale, const int32_t* xsum, int64_t M,
-                        const GemvOut& out, cudaStream_t s) {
+                        const GemvOut& out, cudaStream_t s, const uint16_t* x_fused) {
     if (M == 0 || N == 0) return cudaSuccess;
-    const int KB = (int)(K / 4);
-    const unsigned gx = (unsigned)((N + 15) / 16);
-    if (M <= 8) {
-        gemv_mma_kernel<1><<<dim3(gx, 1), kThreads, 0, s>>>(Wp, gamma, (int)N, KB, Xp, scale, xsum,
-                                                            (int)M, out);
-    } else {
-        const unsigned gy = (unsigned)((M + 15) / 16);
-        gemv_mma_kernel<2><<<dim3(gx, gy), kThreads, 0, s>>>(Wp, gamma, (int)N, KB, Xp, scale, xsum,
-                                                             (int)M, out);
+    GemvArgs a;
+    a.Wp = Wp;
+    a.gamma = gamma;
+    a.N = (int)N;
+    a.KB = (int)(K / 4);
+    a.M = (int)M;
+    a.x = x_fused;
+    a.Xp = Xp;
+    a.scale = scale;
+    a.xsum = xsum;
+    a.out = out;
+    const int ntiles = (int)((N + 15) / 16);
+    // enough CTAs for every SM to hold two; each walks tiles with a grid stride
+    const int cap = 2 * sm_count();
+    const unsigned gx = (unsigned)(ntiles < cap ? ntiles : cap);
+    if (x_fused) {
+        if (!gemv_fused_ok(M, K)) return cudaErrorInvalidValue;
+        const size_t smem = (size_t)M * (K + 64);
+        if (M <= 8) return launch_variant<1, true>(a, dim3(gx, 1), smem, s);
+        return launch_variant<2, true>(a, dim3(gx, 1), smem, s);
     }
-    return cudaGetLastError();
+    if (M <= 8) return launch_variant<1, false>(a, dim3(gx, 1), 0, s);
+    return launch_variant<2, false>(a, dim3(gx, (unsigned)((M + 15) / 16)), 0, s);
 }
 
 cudaError_t launch_gemv_generic(const uint8_t* Wp, const float* gamma, int64_t N, int64_t K,
@@ -216,8 +467,8 @@ cudaError_t launch_gemv_generic(const uint8_t* Wp, const float* gamma, int64_t N
                                 const GemvOut& out, cudaStream_t s) {
     if (M == 0 || N == 0) return cudaSuccess;
     const dim3 grid((unsigned)((N + kWarps - 1) / kWarps), (unsigned)M);
-    gemv_generic_kernel<<<grid, kThreads, 0, s>>>(Wp, gamma, (int)N, (int)K, Xn, scale, (int)M, out);
-    return cudaGetLastError();
+    return launch_pdl(gemv_generic_kernel, grid, dim3(kThreads), 0, s, Wp, gamma, (int)N, (int)K, Xn,
+                      scale, (int)M, out);
 }
 
 }  // namespace bl

@@ -29,11 +29,14 @@ struct GemvOut {
     int32_t* acc = nullptr;             // [M, N] or null
     float* y32 = nullptr;               // [M, N] fp32 (used instead of y when set)
 };
-// Xp: PLANES layout codes for M tokens; requires K % 256 == 0 and 16-byte aligned Wp, Xp.
+// Requires K % 256 == 0 and 16-byte aligned Wp. Codes either come as PLANES
+// layout Xp (+ scale, xsum) from the act-quant kernel, or, when x_fused is given
+// (16-byte aligned bf16 x, gemv_fused_ok(M, K)), are computed inside the kernel.
 bool gemv_fast_ok(int64_t N, int64_t K);
+bool gemv_fused_ok(int64_t M, int64_t K);
 cudaError_t launch_gemv(const uint8_t* Wp, const float* gamma, int64_t N, int64_t K,
                         const int8_t* Xp, const float* scale, const int32_t* xsum, int64_t M,
-                        const GemvOut& out, cudaStream_t s);
+                        const GemvOut& out, cudaStream_t s, const uint16_t* x_fused = nullptr);
 // Any K % 4 == 0: NATURAL layout codes, one warp per output.
 cudaError_t launch_gemv_generic(const uint8_t* Wp, const float* gamma, int64_t N, int64_t K,
                                 const int8_t* Xn, const float* scale, int64_t M,
