@@ -40,6 +40,12 @@ sys.path.insert(0, ROOT)
 METRIC = "W1.58A8 BitLinear: decode GEMV HBM GB/s (% peak); prefill int8 TOPS (% peak)"
 DECODE_SHAPES = [(2560, 2560), (2560, 640), (2560, 6912), (6912, 2560)]  # (K, N)
 LAYERS = 30
+# DRAM bytes (read + write) per launch of the decode GEMV, averaged over the
+# step's mix of shapes: an ncu capture of the 2560 -> 6912 launch read 4,479,232
+# bytes for 4,423,680 packed bytes (x 1.0126); scaled to the mean launch of the
+# step (2,723,840 packed bytes). Set to None whenever the kernel changes until a
+# new capture is taken.
+GEMV_TRAFFIC_PER_LAUNCH = 2758050
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 INT8_PER_BF16 = 2.0  # nominal dense int8 (= fp8) rate over dense bf16 on B200
 
@@ -76,7 +82,7 @@ class ClockSampler:
             self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
+                 "--format=csv,noheader,nounits", "-lms", "50"],
                 stdout=self.file, stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
             self.proc = None
@@ -158,7 +164,7 @@ def run_ours(args):
     ws = torch.empty(max(bl.workspace_bytes(bl.BL_OP_FORWARD, 16, N, K) for K, N in DECODE_SHAPES),
                      dtype=torch.uint8, device=dev)
     step_bytes = LAYERS * sum(K * N // 4 for K, N in DECODE_SHAPES)
-    kernels_per_call = 2  # act-quant + GEMV
+    kernels_per_call = 1  # M = 1: the GEMV quantises x itself
 
     def step():
         for layer in range(LAYERS):
@@ -199,26 +205,18 @@ def run_ours(args):
     ms_step = ms_total / args.steps
     value = world * step_bytes * args.steps / (ms_total * 1e-3) / 1e9
 
-    # ---- dominant kernel: per-call device time of the decode forward
-    # (act-quant + GEMV), CUDA events on the launching stream, eager, one step.
-    evs = []
-    torch.cuda.synchronize()
-    for layer in range(LAYERS):
-        for si in range(len(DECODE_SHAPES)):
-            a = torch.cuda.Event(enable_timing=True)
-            b = torch.cuda.Event(enable_timing=True)
-            Wp, g = weights[layer][si]
-            a.record(cur)
-            bl.forward(Wp, g, xs[si], out=ys[si], ws=ws)
-            b.record(cur)
-            evs.append((a, b, DECODE_SHAPES[si]))
-    torch.cuda.synchronize()
-    call_ms = sum(a.elapsed_time(b) for a, b, _ in evs)
-    call_bytes = sum(K * N // 4 for _, _, (K, N) in evs)
-    achieved = call_bytes / (call_ms * 1e-3) / 1e9
+    # ---- dominant kernel: the decode GEMV. At M = 1 each forward call is one
+    # kernel (quantisation fused); consecutive calls overlap through programmatic
+    # dependent launch, so the average launch duration is the timed region's
+    # device time over the launches in it (CUDA events on the launching stream).
+    calls = args.steps * LAYERS * len(DECODE_SHAPES)
+    per_launch_s = (ev0.elapsed_time(ev1) * 1e-3) / calls
+    achieved = (step_bytes / (LAYERS * len(DECODE_SHAPES))) / per_launch_s / 1e9
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
-                "frac": round(achieved / hbm_peak, 4), "traffic": None,
-                "kernel": "act_quant_vec_kernel<PLANES> + gemv_mma_kernel<1> (one forward call)",
+                "frac": round(achieved / hbm_peak, 4), "traffic": GEMV_TRAFFIC_PER_LAUNCH,
+                "kernel": "gemv_mma_kernel<1,fused> (quantise + ternary GEMV + dequant, one launch per call)",
+                "us_per_launch": round(per_launch_s * 1e6, 3),
+                "bytes_per_launch": step_bytes // (LAYERS * len(DECODE_SHAPES)),
                 "peak_kind": peak_kind}
 
     extras = {}
@@ -432,18 +430,17 @@ def cpu_baseline(weights, xs, bl, budget_s: float):
     host = [[(Wp.cpu().numpy(), float(g.cpu().item())) for Wp, g in row] for row in weights]
     done_bytes, n_layers = 0, 0
     t0 = time.perf_counter()
-    for row in host:
+    while time.perf_counter() - t0 < budget_s:
+        row = host[n_layers % LAYERS]
         for (Wp, g), xb in zip(row, bits):
             oracle.forward(Wp, g, xb)
             done_bytes += Wp.size
         n_layers += 1
-        if time.perf_counter() - t0 > budget_s:
-            break
     dt = time.perf_counter() - t0
     cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
     return {"value": round(done_bytes / dt / 1e9, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
-            "sample": f"{n_layers} of 30 layers of the decode step (4 shapes each, M=1), "
-                      f"{done_bytes} packed bytes in {dt:.2f} s"}
+            "sample": f"{n_layers} layers of the decode step, cycling over its 30 layers "
+                      f"(4 shapes each, M=1): {done_bytes} packed bytes in {dt:.2f} s"}
 
 
 # ----------------------------------------------------------------------------- reference arm
@@ -531,7 +528,7 @@ def run_profile_case(name: str, reps: int):
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-extras", action="store_true", help="skip the secondary workloads")
