@@ -45,7 +45,7 @@ LAYERS = 30
 # bytes for 4,423,680 packed bytes (x 1.0126); scaled to the mean launch of the
 # step (2,723,840 packed bytes). Set to None whenever the kernel changes until a
 # new capture is taken.
-GEMV_TRAFFIC_PER_LAUNCH = 2758050
+GEMV_TRAFFIC_PER_LAUNCH = None
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 INT8_PER_BF16 = 2.0  # nominal dense int8 (= fp8) rate over dense bf16 on B200
 

@@ -33,6 +33,7 @@
 // load of other data and every store comes after the wait.
 #include "common.cuh"
 #include "kernels.h"
+#include "tc_ptx.cuh"
 
 namespace bl {
 namespace {
@@ -43,6 +44,9 @@ constexpr int kUnroll = 4;
 constexpr int kPrefetchAhead = 2;          // tiles of lookahead per CTA
 constexpr int kFusedSmemLimit = 48 * 1024;  // codes of all tokens in shared memory
 constexpr int kFusedMaxTokens = 4;          // beyond this the separate quantiser is faster
+constexpr int kStages = 2;                  // shared-memory ring of streamed weight units (2 CTAs per SM)
+constexpr int kMaxSegChunks = 32;           // at most 2 KiB of each row per unit
+constexpr uint64_t kWaitLimitNs = 1000000000ull;
 
 
 __device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
@@ -85,7 +89,14 @@ struct GemvArgs {
     const float* scale;    // [M] (not fused)
     const int32_t* xsum;   // [M] (not fused)
     GemvOut out;
+    unsigned* err;         // device error word (bounded waits that give up)
+    int seg_chunks;        // 64-byte chunks per K segment of a streamed unit
+    int pitch;             // shared-memory row pitch of a stage
+    int codes_bytes;       // fused codes area at the start of dynamic shared memory
 };
+
+// Named barrier of the eight consumer warps (the producer warp is not in it).
+__device__ __forceinline__ void consumer_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 
 // Byte offset of plane i of token m in the fused shared-memory code buffer. The
 // +64 per token keeps the tokens of one quarter-warp on different banks.
@@ -179,14 +190,14 @@ __device__ void fused_quantise(const uint16_t* __restrict__ x, int M, int KB, co
         }
     }
     if (threadIdx.x < TOK) xs_sh[threadIdx.x] = 0;
-    __syncthreads();
+    consumer_sync();
     if (threadIdx.x < M) {
         float r = am_sh[0][threadIdx.x];
 #pragma unroll
         for (int w = 1; w < kWarps; ++w) r = fmaxf(r, am_sh[w][threadIdx.x]);
         s_sh[threadIdx.x] = __fdiv_rn(kActRange, fmaxf(r, kActEps));
     }
-    __syncthreads();
+    consumer_sync();
     // code sums: per-thread partials per token, a warp reduction, one atomic per warp
     int xs[TOK];
 #pragma unroll
@@ -212,73 +223,124 @@ __device__ void fused_quantise(const uint16_t* __restrict__ x, int M, int KB, co
     }
 }
 
+// 1-D bulk copy global -> this CTA's shared memory, completion counted on `bar`.
+__device__ __forceinline__ void bulk_copy(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+        "l"(src), "r"(bytes), "r"(bar)
+        : "memory");
+}
+
+// The weight stream: a unit is one 16-row tile restricted to one K segment of
+// at most 32 chunks (2 KiB per row). The producer warp copies the unit's row
+// segments into a ring of kStages shared-memory stages; the row pitch is
+// congruent to 64 mod 128 bytes so rows g and g + 1 of a quarter-warp fall on
+// different banks.
 template <int NT, bool FUSED>
-__global__ void __launch_bounds__(kThreads) gemv_mma_kernel(const GemvArgs a) {
+__global__ void __launch_bounds__(kThreads + 32) gemv_mma_kernel(const GemvArgs a) {
     constexpr int TOK = 8 * NT;
-    constexpr int CPP = kWarps * kUnroll;  // chunks per pass of the whole CTA
-    extern __shared__ __align__(16) uint8_t codes[];  // fused: PLANES codes of the M tokens
+    extern __shared__ __align__(128) uint8_t dyn[];
     __shared__ int red[kWarps][16][TOK];
     __shared__ float s_sh[TOK];
     __shared__ int xs_sh[TOK];
     __shared__ float am_sh[kWarps][TOK];
+    __shared__ int abort_sh;
 
     const int N = a.N, KB = a.KB;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int g = lane >> 2, t = lane & 3;
     const int ntiles = (N + 15) >> 4;
     const int nchunks = KB >> 6;
-    const int npass = (nchunks + CPP - 1) / CPP;
+    const int cps = a.seg_chunks;                     // chunks per K segment
+    const int nseg = (nchunks + cps - 1) / cps;
+    const int pitch = a.pitch;
     const int tok0 = blockIdx.y * TOK;
 
-    auto tile_prefetch = [&](int tile) {
-        const int n0 = tile * 16;
-        const int rows = min(16, N - n0);
-        prefetch_l2(a.Wp + (size_t)n0 * KB, (uint32_t)(rows * KB));
-    };
-    if (threadIdx.x == 0) {
+    uint8_t* codes = dyn;                              // fused: PLANES codes of the M tokens
+    uint8_t* stages = dyn + a.codes_bytes;             // kStages x 16 rows x pitch
+    uint64_t* bars = reinterpret_cast<uint64_t*>(stages + kStages * 16 * pitch);
+    auto full = [&](int st) { return tc::smem_u32(bars + st); };
+    auto empty = [&](int st) { return tc::smem_u32(bars + kStages + st); };
+
+    if (threadIdx.x == kThreads) {
+        for (int st = 0; st < kStages; ++st) {
+            tc::mbar_init(full(st), 1);
+            tc::mbar_init(empty(st), kWarps);
+        }
+        abort_sh = 0;
+        tc::fence_mbar_init();
+        // L2 prefetch of the first tiles may run before the previous kernel ends
         for (int p = 0; p < kPrefetchAhead; ++p) {
             const int tile = blockIdx.x + p * gridDim.x;
-            if (tile < ntiles) tile_prefetch(tile);
-        }
-    }
-    // weight registers of one pass: chunk warp + kWarps * (kUnroll * pass + u)
-    uint4 wa[kUnroll], wb[kUnroll];
-    auto issue = [&](int tile, int pass) {
-        const int n0 = tile * 16;
-        const uint8_t* pA = a.Wp + (size_t)min(n0 + g, N - 1) * KB + 16 * t;
-        const uint8_t* pB = a.Wp + (size_t)min(n0 + g + 8, N - 1) * KB + 16 * t;
-#pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            const int c = warp + kWarps * (kUnroll * pass + u);
-            if (c < nchunks) {
-                wa[u] = ld_stream16(pA + 64 * c);
-                wb[u] = ld_stream16(pB + 64 * c);
+            if (tile < ntiles) {
+                const int n0 = tile * 16;
+                prefetch_l2(a.Wp + (size_t)n0 * KB, (uint32_t)(min(16, N - n0) * KB));
             }
         }
-    };
+    }
+    __syncthreads();
     grid_dependents_launch();
     grid_dependency_wait();
 
-    // x first, then the first pass of the first tile: both loads are in flight
-    // while x is quantised
-    XRegs xr;
-    if (FUSED) fused_load(a.x, a.M, KB, xr);
-    if ((int)blockIdx.x < ntiles) issue(blockIdx.x, 0);
+    if (warp == kWarps) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            uint32_t g = 0;
+            bool stop = false;
+            for (int tile = blockIdx.x; tile < ntiles && !stop; tile += gridDim.x) {
+                const int n0 = tile * 16;
+                const int rows = min(16, N - n0);
+                for (int sg = 0; sg < nseg; ++sg, ++g) {
+                    const int st = g % kStages;
+                    if (g >= kStages &&
+                        !tc::mbar_wait(empty(st), ((g / kStages) - 1) & 1, kWaitLimitNs)) {
+                        atomicOr(a.err, 1u);
+                        atomicExch(&abort_sh, 1);
+                    }
+                    if (*reinterpret_cast<volatile int*>(&abort_sh)) {
+                        stop = true;
+                        break;
+                    }
+                    const int c0 = sg * cps;
+                    const uint32_t segb = (uint32_t)(min(cps, nchunks - c0) * 64);
+                    tc::mbar_arrive_expect_tx(full(st), segb * rows);
+                    const uint32_t dst = tc::smem_u32(stages + st * 16 * pitch);
+                    for (int r = 0; r < rows; ++r)
+                        bulk_copy(dst + r * pitch, a.Wp + (size_t)(n0 + r) * KB + c0 * 64, segb, full(st));
+                }
+            }
+            if (stop) {
+                // let the copies still in flight land before this warp exits
+                const uint32_t first = g > (uint32_t)kStages ? g - kStages : 0;
+                for (uint32_t h = first; h < g; ++h)
+                    tc::mbar_wait(full(h % kStages), (h / kStages) & 1, kWaitLimitNs);
+            }
+            // otherwise every unit handed out was consumed: the consumers waited on
+            // each full barrier, so no copy is in flight when this warp exits
+        }
+        return;
+    }
 
+    // ---------------------------------------------------------------- consumers
+    const int g8 = lane >> 2, t = lane & 3;
     if (FUSED) {
+        XRegs xr;
+        fused_load(a.x, a.M, KB, xr);
         fused_quantise<TOK>(a.x, a.M, KB, xr, codes, s_sh, xs_sh, am_sh);
     } else if (threadIdx.x < TOK && tok0 + (int)threadIdx.x < a.M) {
         s_sh[threadIdx.x] = a.scale[tok0 + threadIdx.x];
         xs_sh[threadIdx.x] = a.xsum[tok0 + threadIdx.x];
     }
-    __syncthreads();
+    consumer_sync();
+    __shared__ float deq_sh[TOK];
+    if (threadIdx.x < TOK && tok0 + (int)threadIdx.x < a.M) deq_sh[threadIdx.x] = __fdiv_rn(*a.gamma, s_sh[threadIdx.x]);
+    consumer_sync();
 
-    // this lane's activation operand: token 8*nt + g of the group
+    // this lane's activation operand: token 8*nt + g8 of the group
     const uint8_t* xbase[NT];
     bool tv[NT];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
-        const int tok = tok0 + 8 * nt + g;
+        const int tok = tok0 + 8 * nt + g8;
         tv[nt] = tok < a.M;
         if (FUSED)
             xbase[nt] = codes + smem_plane_off(tv[nt] ? tok : 0, 0, KB) + 16 * t;
@@ -300,12 +362,11 @@ __global__ void __launch_bounds__(kThreads) gemv_mma_kernel(const GemvArgs a) {
             }
     };
 
-    const float gamma = *a.gamma;
+    // An abort (a bounded wait that gave up) keeps every consumer warp on the same
+    // sequence of named barriers: later waits are skipped and nothing is stored.
+    auto aborted = [&]() { return *reinterpret_cast<volatile int*>(&abort_sh) != 0; };
+    uint32_t g = 0;
     for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
-        if (threadIdx.x == 0) {
-            const int ahead = tile + kPrefetchAhead * gridDim.x;
-            if (ahead < ntiles) tile_prefetch(ahead);
-        }
         const int n0 = tile * 16;
         int acc[NT][4][4];
 #pragma unroll
@@ -315,20 +376,34 @@ __global__ void __launch_bounds__(kThreads) gemv_mma_kernel(const GemvArgs a) {
 #pragma unroll
                 for (int e = 0; e < 4; ++e) acc[nt][i][e] = 0;
 
-        for (int pass = 0; pass < npass; ++pass) {
-            if (tile != (int)blockIdx.x || pass != 0) issue(tile, pass);
+        for (int sg = 0; sg < nseg; ++sg, ++g) {
+            const int st = g % kStages;
+            if (aborted()) continue;
+            if (!tc::mbar_wait(full(st), (g / kStages) & 1, kWaitLimitNs)) {
+                atomicOr(a.err, 1u);
+                atomicExch(&abort_sh, 1);
+                continue;
+            }
+            const int c0 = sg * cps;
+            const int segc = min(cps, nchunks - c0);
+            const uint8_t* sa = stages + st * 16 * pitch + g8 * pitch + 16 * t;
+            const uint8_t* sb = sa + 8 * pitch;
 #pragma unroll
             for (int u = 0; u < kUnroll; ++u) {
-                const int c = warp + kWarps * (kUnroll * pass + u);
-                if (c < nchunks) {
+                const int cl = warp + kWarps * u;
+                if (cl < segc) {
+                    const uint4 wa = *reinterpret_cast<const uint4*>(sa + 64 * cl);
+                    const uint4 wb = *reinterpret_cast<const uint4*>(sb + 64 * cl);
                     uint4 xv[NT][4];
-                    load_x(xv, 64 * c);
-                    chunk_mma<NT>(acc, wa[u], wb[u], xv);
+                    load_x(xv, 64 * (c0 + cl));
+                    chunk_mma<NT>(acc, wa, wb, xv);
                 }
             }
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(empty(st));
         }
 
-        // Fold the four field accumulators; D element e sits at row g + 8*(e >> 1),
+        // Fold the four field accumulators; D element e sits at row g8 + 8*(e >> 1),
         // token 8*nt + 2t + (e & 1).
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
@@ -336,11 +411,12 @@ __global__ void __launch_bounds__(kThreads) gemv_mma_kernel(const GemvArgs a) {
             for (int e = 0; e < 4; ++e) {
                 const int v = acc[nt][0][e] + (acc[nt][1][e] >> 2) + (acc[nt][2][e] >> 4) +
                               (acc[nt][3][e] >> 6);
-                red[warp][g + 8 * (e >> 1)][8 * nt + 2 * t + (e & 1)] = v;
+                red[warp][g8 + 8 * (e >> 1)][8 * nt + 2 * t + (e & 1)] = v;
             }
-        __syncthreads();
+        consumer_sync();
 
-        for (int idx = threadIdx.x; idx < 16 * TOK; idx += kThreads) {
+        const bool store = !aborted();
+        for (int idx = threadIdx.x; store && idx < 16 * TOK; idx += kThreads) {
             const int r = idx & 15, cl = idx >> 4;
             const int n = n0 + r, m = tok0 + cl;
             if (n >= N || m >= a.M) continue;
@@ -348,8 +424,7 @@ __global__ void __launch_bounds__(kThreads) gemv_mma_kernel(const GemvArgs a) {
 #pragma unroll
             for (int w = 0; w < kWarps; ++w) sum += red[w][r][cl];
             const int accv = sum - xs_sh[cl];
-            const float deq = __fdiv_rn(gamma, s_sh[cl]);
-            float v = dequant(accv, deq);
+            float v = dequant(accv, deq_sh[cl]);
             const size_t o = (size_t)m * N + n;
             if (a.out.y32) {
                 a.out.y32[o] = v;
@@ -359,7 +434,7 @@ __global__ void __launch_bounds__(kThreads) gemv_mma_kernel(const GemvArgs a) {
             }
             if (a.out.acc) a.out.acc[o] = accv;
         }
-        __syncthreads();
+        consumer_sync();
     }
 }
 
@@ -410,19 +485,15 @@ int sm_count() {
 template <int NT, bool FUSED>
 cudaError_t launch_variant(const GemvArgs& a, dim3 grid, size_t smem, cudaStream_t s) {
     auto kern = gemv_mma_kernel<NT, FUSED>;
-    if (FUSED) {
-        // static + dynamic shared memory may pass the 48 KiB default: opt in once per device
-        static bool done[64];
-        int dev = 0;
-        cudaGetDevice(&dev);
-        if (dev >= 64 || !done[dev]) {
-            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 kFusedSmemLimit);
-            if (e != cudaSuccess) return e;
-            if (dev < 64) done[dev] = true;
-        }
+    static bool done[64];
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 64 || !done[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+        if (e != cudaSuccess) return e;
+        if (dev < 64) done[dev] = true;
     }
-    return launch_pdl(kern, grid, dim3(kThreads), smem, s, a);
+    return launch_pdl(kern, grid, dim3(kThreads + 32), smem, s, a);
 }
 
 }  // namespace
@@ -448,18 +519,26 @@ cudaError_t launch_gemv(const uint8_t* Wp, const float* gamma, int64_t N, int64_
     a.scale = scale;
     a.xsum = xsum;
     a.out = out;
+    cudaError_t e = device_error_word(&a.err);
+    if (e != cudaSuccess) return e;
+    // K segments of at most kMaxSegChunks chunks, as even as possible
+    const int nchunks = a.KB / 64;
+    const int nseg = (nchunks + kMaxSegChunks - 1) / kMaxSegChunks;
+    a.seg_chunks = (nchunks + nseg - 1) / nseg;
+    const int segb = a.seg_chunks * 64;
+    a.pitch = (segb % 128 == 0) ? segb + 64 : segb;  // rows g, g+1 on different banks
+    a.codes_bytes = x_fused ? (int)((M * (K + 64) + 127) / 128 * 128) : 0;
+    if (x_fused && !gemv_fused_ok(M, K)) return cudaErrorInvalidValue;
+    const size_t smem = (size_t)a.codes_bytes + (size_t)kStages * 16 * a.pitch + 2 * kStages * 8;
     const int ntiles = (int)((N + 15) / 16);
-    // enough CTAs for every SM to hold two; each walks tiles with a grid stride
-    const int cap = 2 * sm_count();
+    // as many CTAs per SM as shared memory allows (228 KiB per SM, 1 KiB reserved per CTA)
+    int per_sm = (int)((228 * 1024) / (smem + 8 * 1024 + 1024));
+    per_sm = per_sm < 1 ? 1 : per_sm > 4 ? 4 : per_sm;
+    const int cap = per_sm * sm_count();
     const unsigned gx = (unsigned)(ntiles < cap ? ntiles : cap);
-    if (x_fused) {
-        if (!gemv_fused_ok(M, K)) return cudaErrorInvalidValue;
-        const size_t smem = (size_t)M * (K + 64);
-        if (M <= 8) return launch_variant<1, true>(a, dim3(gx, 1), smem, s);
-        return launch_variant<2, true>(a, dim3(gx, 1), smem, s);
-    }
-    if (M <= 8) return launch_variant<1, false>(a, dim3(gx, 1), 0, s);
-    return launch_variant<2, false>(a, dim3(gx, (unsigned)((M + 15) / 16)), 0, s);
+    if (x_fused) return launch_variant<1, true>(a, dim3(gx, 1), smem, s);
+    if (M <= 8) return launch_variant<1, false>(a, dim3(gx, 1), smem, s);
+    return launch_variant<2, false>(a, dim3(gx, (unsigned)((M + 15) / 16)), smem, s);
 }
 
 cudaError_t launch_gemv_generic(const uint8_t* Wp, const float* gamma, int64_t N, int64_t K,
