@@ -243,6 +243,20 @@ BL_API bl_status bitlinear_ffn(const uint8_t* Wg, const float* gg, const uint8_t
     Path up = choose_path(Wg, f, d, M, xq, x);
     if (choose_path(Wu, f, d, M, xq, x) != up) up = Path::GemvGeneric;
     const Path down = choose_path(Wd, d, f, M, q2, nullptr);
+    if (up == Path::GemvFast && down == Path::GemvFast && bl::gemv_fused_ok(M, d) &&
+        bl::gemv_fused_ok(M, f)) {
+        // Two kernels: gate+up streamed together with h and its per-tile partials
+        // as output (h in the g slot, partials in the u slot), then the down
+        // projection with the RMSNorm + requantisation folded into its prologue.
+        const size_t nparts = (size_t)((f + 15) / 16);
+        double* part_ss = (double*)u;
+        float* part_max = (float*)((char*)u + align_up((size_t)M * nparts * sizeof(double)));
+        BL_TRY(bl::launch_ffn_up_fused(Wg, gg, Wu, gu, f, d, x, M, g, part_ss, part_max, s));
+        bl::GemvOut od;
+        od.y = y;
+        od.residual = residual;
+        return cuda_status(bl::launch_ffn_down_fused(Wd, gd, d, f, g, part_ss, part_max, M, od, s));
+    }
     bl::GemvOut og;
     og.y32 = g;
     bl::GemvOut ou;

@@ -93,6 +93,24 @@ struct GemvArgs {
     int seg_chunks;        // 64-byte chunks per K segment of a streamed unit
     int pitch;             // shared-memory row pitch of a stage
     int codes_bytes;       // fused codes area at the start of dynamic shared memory
+    // second weight stream (FFN up: Wp = gate, Wp2 = up; same rows, same codes)
+    const uint8_t* Wp2;
+    const float* gamma2;
+    float* h;              // FFN up output: h = relu(g)^2 * u, [M, N] fp32
+    double* part_ss;       // FFN up output: per (token, 16-row tile) sum of h^2
+    float* part_max;       // FFN up output: per (token, 16-row tile) max |h|
+    // FFN down input (SRC_H): h [M, K] fp32 and the per-tile partials of the up kernel
+    const float* hin;
+    const double* hin_ss;
+    const float* hin_max;
+    int hin_parts;         // tiles of the up projection (= ceil(K / 16))
+};
+
+// Where the activation codes of a streamed GEMV come from.
+enum GemvSrc : int {
+    SRC_CODES = 0,  // PLANES codes (+ scale, code sum) from the act-quant kernel
+    SRC_X = 1,      // bf16 x, quantised per token inside the kernel
+    SRC_H = 2,      // fp32 h of the FFN up kernel: subln RMSNorm + requant inside the kernel
 };
 
 // Named barrier of the eight consumer warps (the producer warp is not in it).
@@ -223,6 +241,79 @@ __device__ void fused_quantise(const uint16_t* __restrict__ x, int M, int KB, co
     }
 }
 
+// FFN glue inside the down projection (one token per loop step, all consumer
+// threads): r = 1 / sqrtf(float(sum_j h_j^2 / f) + eps) from the up kernel's
+// per-tile fp64 partials (summed in tile order), s2 = 127 / max(max_j |h_j r|, eps)
+// with max_j |fl(h_j r)| = fl(max_j |h_j| r) (rounding is monotonic, r > 0), then
+// PLANES codes of fl(h_j r) into shared memory.
+template <int TOK>
+__device__ void finalise_quantise(const GemvArgs& a, int KB, uint8_t* codes, float* s_sh, int* xs_sh,
+                                  float* r_sh) {
+    const int f = 4 * KB;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    __shared__ double dred[kWarps];
+    __shared__ float fred[kWarps];
+    if (threadIdx.x < TOK) xs_sh[threadIdx.x] = 0;
+    for (int m = 0; m < a.M; ++m) {
+        // fixed order: thread strides, warp butterfly, warps in index order
+        double ss = 0.0;
+        float hmax = 0.0f;
+        for (int p = threadIdx.x; p < a.hin_parts; p += kThreads) {
+            ss = __dadd_rn(ss, a.hin_ss[(size_t)m * a.hin_parts + p]);
+            hmax = fmaxf(hmax, a.hin_max[(size_t)m * a.hin_parts + p]);
+        }
+        ss = warp_sum(ss);
+        hmax = warp_max(hmax);
+        if (lane == 0) {
+            dred[warp] = ss;
+            fred[warp] = hmax;
+        }
+        consumer_sync();
+        if (threadIdx.x == 0) {
+            double tot = dred[0];
+            float mx = fred[0];
+            for (int w = 1; w < kWarps; ++w) {
+                tot = __dadd_rn(tot, dred[w]);
+                mx = fmaxf(mx, fred[w]);
+            }
+            const float ms = __double2float_rn(__ddiv_rn(tot, (double)f));
+            const float r = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, kRmsEps)));
+            r_sh[m] = r;
+            s_sh[m] = __fdiv_rn(kActRange, fmaxf(__fmul_rn(mx, r), kActEps));
+        }
+        consumer_sync();
+    }
+    const int groups = KB / 4;
+    for (int m = 0; m < a.M; ++m) {
+        const float r = r_sh[m], s = s_sh[m];
+        const float4* hr = reinterpret_cast<const float4*>(a.hin + (size_t)m * f);
+        int sum = 0;
+        for (int c = threadIdx.x; c < groups; c += kThreads) {
+            float v[16];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const float4 h4 = hr[4 * c + q];
+                v[4 * q] = h4.x;
+                v[4 * q + 1] = h4.y;
+                v[4 * q + 2] = h4.z;
+                v[4 * q + 3] = h4.w;
+            }
+            unsigned pw[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+                const int q = quant_code(__fmul_rn(v[e], r), s);
+                sum += q;
+                pw[e & 3] |= static_cast<unsigned>(q & 255) << (8 * (e >> 2));
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                *reinterpret_cast<unsigned*>(codes + smem_plane_off(m, i, KB) + 4 * c) = pw[i];
+        }
+        sum = warp_sum(sum);
+        if (lane == 0) atomicAdd(&xs_sh[m], sum);
+    }
+}
+
 // 1-D bulk copy global -> this CTA's shared memory, completion counted on `bar`.
 __device__ __forceinline__ void bulk_copy(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
     asm volatile(
@@ -236,14 +327,18 @@ __device__ __forceinline__ void bulk_copy(uint32_t dst, const void* src, uint32_
 // segments into a ring of kStages shared-memory stages; the row pitch is
 // congruent to 64 mod 128 bytes so rows g and g + 1 of a quarter-warp fall on
 // different banks.
-template <int NT, bool FUSED>
+template <int NT, int SRC, bool DUAL>
 __global__ void __launch_bounds__(kThreads + 32) gemv_mma_kernel(const GemvArgs a) {
     constexpr int TOK = 8 * NT;
+    constexpr bool FUSED = SRC != SRC_CODES;
+    constexpr int NW = DUAL ? 2 : 1;  // weight streams
     extern __shared__ __align__(128) uint8_t dyn[];
     __shared__ int red[kWarps][16][TOK];
+    __shared__ int red2[DUAL ? kWarps : 1][16][TOK];
     __shared__ float s_sh[TOK];
     __shared__ int xs_sh[TOK];
     __shared__ float am_sh[kWarps][TOK];
+    __shared__ float r_sh[TOK];
     __shared__ int abort_sh;
 
     const int N = a.N, KB = a.KB;
@@ -256,8 +351,9 @@ __global__ void __launch_bounds__(kThreads + 32) gemv_mma_kernel(const GemvArgs 
     const int tok0 = blockIdx.y * TOK;
 
     uint8_t* codes = dyn;                              // fused: PLANES codes of the M tokens
-    uint8_t* stages = dyn + a.codes_bytes;             // kStages x 16 rows x pitch
-    uint64_t* bars = reinterpret_cast<uint64_t*>(stages + kStages * 16 * pitch);
+    uint8_t* stages = dyn + a.codes_bytes;             // kStages x NW x 16 rows x pitch
+    const int stage_bytes = NW * 16 * pitch;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(stages + kStages * stage_bytes);
     auto full = [&](int st) { return tc::smem_u32(bars + st); };
     auto empty = [&](int st) { return tc::smem_u32(bars + kStages + st); };
 
@@ -274,6 +370,7 @@ __global__ void __launch_bounds__(kThreads + 32) gemv_mma_kernel(const GemvArgs 
             if (tile < ntiles) {
                 const int n0 = tile * 16;
                 prefetch_l2(a.Wp + (size_t)n0 * KB, (uint32_t)(min(16, N - n0) * KB));
+                if (DUAL) prefetch_l2(a.Wp2 + (size_t)n0 * KB, (uint32_t)(min(16, N - n0) * KB));
             }
         }
     }
@@ -302,10 +399,14 @@ __global__ void __launch_bounds__(kThreads + 32) gemv_mma_kernel(const GemvArgs 
                     }
                     const int c0 = sg * cps;
                     const uint32_t segb = (uint32_t)(min(cps, nchunks - c0) * 64);
-                    tc::mbar_arrive_expect_tx(full(st), segb * rows);
-                    const uint32_t dst = tc::smem_u32(stages + st * 16 * pitch);
+                    tc::mbar_arrive_expect_tx(full(st), segb * rows * NW);
+                    const uint32_t dst = tc::smem_u32(stages + st * stage_bytes);
                     for (int r = 0; r < rows; ++r)
                         bulk_copy(dst + r * pitch, a.Wp + (size_t)(n0 + r) * KB + c0 * 64, segb, full(st));
+                    if (DUAL)
+                        for (int r = 0; r < rows; ++r)
+                            bulk_copy(dst + (16 + r) * pitch, a.Wp2 + (size_t)(n0 + r) * KB + c0 * 64, segb,
+                                      full(st));
                 }
             }
             if (stop) {
@@ -322,17 +423,22 @@ __global__ void __launch_bounds__(kThreads + 32) gemv_mma_kernel(const GemvArgs 
 
     // ---------------------------------------------------------------- consumers
     const int g8 = lane >> 2, t = lane & 3;
-    if (FUSED) {
+    if (SRC == SRC_X) {
         XRegs xr;
         fused_load(a.x, a.M, KB, xr);
         fused_quantise<TOK>(a.x, a.M, KB, xr, codes, s_sh, xs_sh, am_sh);
+    } else if (SRC == SRC_H) {
+        finalise_quantise<TOK>(a, KB, codes, s_sh, xs_sh, r_sh);
     } else if (threadIdx.x < TOK && tok0 + (int)threadIdx.x < a.M) {
         s_sh[threadIdx.x] = a.scale[tok0 + threadIdx.x];
         xs_sh[threadIdx.x] = a.xsum[tok0 + threadIdx.x];
     }
     consumer_sync();
-    __shared__ float deq_sh[TOK];
-    if (threadIdx.x < TOK && tok0 + (int)threadIdx.x < a.M) deq_sh[threadIdx.x] = __fdiv_rn(*a.gamma, s_sh[threadIdx.x]);
+    __shared__ float deq_sh[TOK], deq2_sh[TOK];
+    if (threadIdx.x < TOK && tok0 + (int)threadIdx.x < a.M) {
+        deq_sh[threadIdx.x] = __fdiv_rn(*a.gamma, s_sh[threadIdx.x]);
+        if (DUAL) deq2_sh[threadIdx.x] = __fdiv_rn(*a.gamma2, s_sh[threadIdx.x]);
+    }
     consumer_sync();
 
     // this lane's activation operand: token 8*nt + g8 of the group
@@ -368,13 +474,21 @@ __global__ void __launch_bounds__(kThreads + 32) gemv_mma_kernel(const GemvArgs 
     uint32_t g = 0;
     for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
         const int n0 = tile * 16;
-        int acc[NT][4][4];
+        int acc[NT][4][4], acc2[NT][4][4];
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
             for (int i = 0; i < 4; ++i)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) acc[nt][i][e] = 0;
+        if constexpr (DUAL) {
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) acc2[nt][i][e] = 0;
+        }
 
         for (int sg = 0; sg < nseg; ++sg, ++g) {
             const int st = g % kStages;
@@ -386,7 +500,7 @@ __global__ void __launch_bounds__(kThreads + 32) gemv_mma_kernel(const GemvArgs 
             }
             const int c0 = sg * cps;
             const int segc = min(cps, nchunks - c0);
-            const uint8_t* sa = stages + st * 16 * pitch + g8 * pitch + 16 * t;
+            const uint8_t* sa = stages + st * stage_bytes + g8 * pitch + 16 * t;
             const uint8_t* sb = sa + 8 * pitch;
 #pragma unroll
             for (int u = 0; u < kUnroll; ++u) {
@@ -397,6 +511,11 @@ __global__ void __launch_bounds__(kThreads + 32) gemv_mma_kernel(const GemvArgs 
                     uint4 xv[NT][4];
                     load_x(xv, 64 * (c0 + cl));
                     chunk_mma<NT>(acc, wa, wb, xv);
+                    if constexpr (DUAL) {
+                        const uint4 wc = *reinterpret_cast<const uint4*>(sa + 16 * pitch + 64 * cl);
+                        const uint4 wd = *reinterpret_cast<const uint4*>(sb + 16 * pitch + 64 * cl);
+                        chunk_mma<NT>(acc2, wc, wd, xv);
+                    }
                 }
             }
             __syncwarp();
@@ -412,8 +531,50 @@ __global__ void __launch_bounds__(kThreads + 32) gemv_mma_kernel(const GemvArgs 
                 const int v = acc[nt][0][e] + (acc[nt][1][e] >> 2) + (acc[nt][2][e] >> 4) +
                               (acc[nt][3][e] >> 6);
                 red[warp][g8 + 8 * (e >> 1)][8 * nt + 2 * t + (e & 1)] = v;
+                if constexpr (DUAL) {
+                    red2[warp][g8 + 8 * (e >> 1)][8 * nt + 2 * t + (e & 1)] =
+                        acc2[nt][0][e] + (acc2[nt][1][e] >> 2) + (acc2[nt][2][e] >> 4) + (acc2[nt][3][e] >> 6);
+                }
             }
         consumer_sync();
+
+        if constexpr (DUAL) {
+            // FFN up epilogue: h = relu(g)^2 * u, plus the tile's per-token sum of
+            // h^2 (fp64, fixed butterfly order over the 16 rows) and max |h|.
+            const bool store_h = !aborted();
+            for (int idx = threadIdx.x; idx < 16 * TOK; idx += kThreads) {
+                const int r = idx & 15, cl = idx >> 4;
+                const int n = n0 + r, m = tok0 + cl;
+                const bool valid = n < N && m < a.M;
+                float hv = 0.0f;
+                if (valid) {
+                    int sg = 0, su = 0;
+#pragma unroll
+                    for (int w = 0; w < kWarps; ++w) {
+                        sg += red[w][r][cl];
+                        su += red2[w][r][cl];
+                    }
+                    const float gv = dequant(sg - xs_sh[cl], deq_sh[cl]);
+                    const float uv = dequant(su - xs_sh[cl], deq2_sh[cl]);
+                    const float tv0 = gv > 0.0f ? gv : 0.0f;
+                    hv = __fmul_rn(__fmul_rn(tv0, tv0), uv);
+                    if (store_h) a.h[(size_t)m * N + n] = hv;
+                }
+                double ss = __dmul_rn((double)hv, (double)hv);
+                float mx = fabsf(hv);
+#pragma unroll
+                for (int o = 8; o > 0; o >>= 1) {  // the 16 rows of a token are 16 adjacent lanes
+                    ss = __dadd_rn(ss, __shfl_xor_sync(0xffffffffu, ss, o));
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+                }
+                if (r == 0 && m < a.M && store_h) {
+                    a.part_ss[(size_t)m * ntiles + tile] = ss;
+                    a.part_max[(size_t)m * ntiles + tile] = mx;
+                }
+            }
+            consumer_sync();
+            continue;
+        }
 
         const bool store = !aborted();
         for (int idx = threadIdx.x; store && idx < 16 * TOK; idx += kThreads) {
@@ -482,9 +643,9 @@ int sm_count() {
     return n;
 }
 
-template <int NT, bool FUSED>
+template <int NT, int SRC, bool DUAL>
 cudaError_t launch_variant(const GemvArgs& a, dim3 grid, size_t smem, cudaStream_t s) {
-    auto kern = gemv_mma_kernel<NT, FUSED>;
+    auto kern = gemv_mma_kernel<NT, SRC, DUAL>;
     static bool done[64];
     int dev = 0;
     cudaGetDevice(&dev);
@@ -494,6 +655,45 @@ cudaError_t launch_variant(const GemvArgs& a, dim3 grid, size_t smem, cudaStream
         if (dev < 64) done[dev] = true;
     }
     return launch_pdl(kern, grid, dim3(kThreads + 32), smem, s, a);
+}
+
+// Segment plan, shared-memory size and grid of one streamed GEMV launch.
+struct StreamPlan {
+    size_t smem;
+    unsigned grid_x;
+};
+
+cudaError_t plan_stream(GemvArgs& a, int64_t N, int64_t K, int64_t M, int nw, bool codes_in_smem,
+                        StreamPlan& p) {
+    cudaError_t e = device_error_word(&a.err);
+    if (e != cudaSuccess) return e;
+    // K segments of at most kMaxSegChunks chunks, as even as possible
+    const int nchunks = (int)(K / 256);
+    const int nseg = (nchunks + kMaxSegChunks - 1) / kMaxSegChunks;
+    a.seg_chunks = (nchunks + nseg - 1) / nseg;
+    const int segb = a.seg_chunks * 64;
+    a.pitch = (segb % 128 == 0) ? segb + 64 : segb;  // rows g, g+1 on different banks
+    a.codes_bytes = codes_in_smem ? (int)((M * (K + 64) + 127) / 128 * 128) : 0;
+    p.smem = (size_t)a.codes_bytes + (size_t)kStages * nw * 16 * a.pitch + 2 * kStages * 8;
+    const int ntiles = (int)((N + 15) / 16);
+    // as many CTAs per SM as shared memory allows (228 KiB per SM, static + reserve per CTA)
+    int per_sm = (int)((228 * 1024) / (p.smem + 10 * 1024));
+    per_sm = per_sm < 1 ? 1 : per_sm > 4 ? 4 : per_sm;
+    const int cap = per_sm * sm_count();
+    p.grid_x = (unsigned)(ntiles < cap ? ntiles : cap);
+    return cudaSuccess;
+}
+
+GemvArgs base_args(const uint8_t* Wp, const float* gamma, int64_t N, int64_t K, int64_t M,
+                   const GemvOut& out) {
+    GemvArgs a = {};
+    a.Wp = Wp;
+    a.gamma = gamma;
+    a.N = (int)N;
+    a.KB = (int)(K / 4);
+    a.M = (int)M;
+    a.out = out;
+    return a;
 }
 
 }  // namespace
@@ -508,37 +708,52 @@ cudaError_t launch_gemv(const uint8_t* Wp, const float* gamma, int64_t N, int64_
                         const int8_t* Xp, const float* scale, const int32_t* xsum, int64_t M,
                         const GemvOut& out, cudaStream_t s, const uint16_t* x_fused) {
     if (M == 0 || N == 0) return cudaSuccess;
-    GemvArgs a;
-    a.Wp = Wp;
-    a.gamma = gamma;
-    a.N = (int)N;
-    a.KB = (int)(K / 4);
-    a.M = (int)M;
+    if (x_fused && !gemv_fused_ok(M, K)) return cudaErrorInvalidValue;
+    GemvArgs a = base_args(Wp, gamma, N, K, M, out);
     a.x = x_fused;
     a.Xp = Xp;
     a.scale = scale;
     a.xsum = xsum;
-    a.out = out;
-    cudaError_t e = device_error_word(&a.err);
+    StreamPlan p;
+    cudaError_t e = plan_stream(a, N, K, M, 1, x_fused != nullptr, p);
     if (e != cudaSuccess) return e;
-    // K segments of at most kMaxSegChunks chunks, as even as possible
-    const int nchunks = a.KB / 64;
-    const int nseg = (nchunks + kMaxSegChunks - 1) / kMaxSegChunks;
-    a.seg_chunks = (nchunks + nseg - 1) / nseg;
-    const int segb = a.seg_chunks * 64;
-    a.pitch = (segb % 128 == 0) ? segb + 64 : segb;  // rows g, g+1 on different banks
-    a.codes_bytes = x_fused ? (int)((M * (K + 64) + 127) / 128 * 128) : 0;
-    if (x_fused && !gemv_fused_ok(M, K)) return cudaErrorInvalidValue;
-    const size_t smem = (size_t)a.codes_bytes + (size_t)kStages * 16 * a.pitch + 2 * kStages * 8;
-    const int ntiles = (int)((N + 15) / 16);
-    // as many CTAs per SM as shared memory allows (228 KiB per SM, 1 KiB reserved per CTA)
-    int per_sm = (int)((228 * 1024) / (smem + 8 * 1024 + 1024));
-    per_sm = per_sm < 1 ? 1 : per_sm > 4 ? 4 : per_sm;
-    const int cap = per_sm * sm_count();
-    const unsigned gx = (unsigned)(ntiles < cap ? ntiles : cap);
-    if (x_fused) return launch_variant<1, true>(a, dim3(gx, 1), smem, s);
-    if (M <= 8) return launch_variant<1, false>(a, dim3(gx, 1), smem, s);
-    return launch_variant<2, false>(a, dim3(gx, (unsigned)((M + 15) / 16)), smem, s);
+    if (x_fused) return launch_variant<1, SRC_X, false>(a, dim3(p.grid_x, 1), p.smem, s);
+    if (M <= 8) return launch_variant<1, SRC_CODES, false>(a, dim3(p.grid_x, 1), p.smem, s);
+    return launch_variant<2, SRC_CODES, false>(a, dim3(p.grid_x, (unsigned)((M + 15) / 16)), p.smem, s);
+}
+
+cudaError_t launch_ffn_up_fused(const uint8_t* Wg, const float* gg, const uint8_t* Wu, const float* gu,
+                                int64_t f, int64_t d, const uint16_t* x, int64_t M, float* h,
+                                double* part_ss, float* part_max, cudaStream_t s) {
+    if (M == 0) return cudaSuccess;
+    if (!gemv_fused_ok(M, d)) return cudaErrorInvalidValue;
+    GemvArgs a = base_args(Wg, gg, f, d, M, GemvOut());
+    a.x = x;
+    a.Wp2 = Wu;
+    a.gamma2 = gu;
+    a.h = h;
+    a.part_ss = part_ss;
+    a.part_max = part_max;
+    StreamPlan p;
+    cudaError_t e = plan_stream(a, f, d, M, 2, true, p);
+    if (e != cudaSuccess) return e;
+    return launch_variant<1, SRC_X, true>(a, dim3(p.grid_x, 1), p.smem, s);
+}
+
+cudaError_t launch_ffn_down_fused(const uint8_t* Wd, const float* gd, int64_t d, int64_t f,
+                                  const float* h, const double* part_ss, const float* part_max,
+                                  int64_t M, const GemvOut& out, cudaStream_t s) {
+    if (M == 0) return cudaSuccess;
+    if (!gemv_fused_ok(M, f)) return cudaErrorInvalidValue;
+    GemvArgs a = base_args(Wd, gd, d, f, M, out);
+    a.hin = h;
+    a.hin_ss = part_ss;
+    a.hin_max = part_max;
+    a.hin_parts = (int)((f + 15) / 16);
+    StreamPlan p;
+    cudaError_t e = plan_stream(a, d, f, M, 1, true, p);
+    if (e != cudaSuccess) return e;
+    return launch_variant<1, SRC_H, false>(a, dim3(p.grid_x, 1), p.smem, s);
 }
 
 cudaError_t launch_gemv_generic(const uint8_t* Wp, const float* gamma, int64_t N, int64_t K,

@@ -37,6 +37,17 @@ bool gemv_fused_ok(int64_t M, int64_t K);
 cudaError_t launch_gemv(const uint8_t* Wp, const float* gamma, int64_t N, int64_t K,
                         const int8_t* Xp, const float* scale, const int32_t* xsum, int64_t M,
                         const GemvOut& out, cudaStream_t s, const uint16_t* x_fused = nullptr);
+// FFN sub-layer for M <= 4 tokens in two streamed kernels (K = d for the up
+// projections, f for the down one; both multiples of 256, f + 64 codes per token
+// in shared memory). up: h = relu(g)^2 * u [M, f] fp32 plus per (token, 16-row
+// tile) partials sum h^2 (fp64) and max |h| [M, ceil(f/16)]; down: subln RMSNorm
+// and requantisation of h from those partials, then the down projection.
+cudaError_t launch_ffn_up_fused(const uint8_t* Wg, const float* gg, const uint8_t* Wu, const float* gu,
+                                int64_t f, int64_t d, const uint16_t* x, int64_t M, float* h,
+                                double* part_ss, float* part_max, cudaStream_t s);
+cudaError_t launch_ffn_down_fused(const uint8_t* Wd, const float* gd, int64_t d, int64_t f,
+                                  const float* h, const double* part_ss, const float* part_max,
+                                  int64_t M, const GemvOut& out, cudaStream_t s);
 // Any K % 4 == 0: NATURAL layout codes, one warp per output.
 cudaError_t launch_gemv_generic(const uint8_t* Wp, const float* gamma, int64_t N, int64_t K,
                                 const int8_t* Xn, const float* scale, int64_t M,

@@ -264,6 +264,22 @@ def test_ffn_prefill_sampled_tokens(cuda_device):
         h_dev = y_dev
 
 
+@pytest.mark.parametrize("M", [2, 4, 8])
+def test_ffn_small_batches(cuda_device, M):
+    """M <= 4 runs the two-kernel FFN (gate+up with h partials, down with the
+    norm and requantisation folded in); M = 8 the unfused decode path."""
+    d, f = 2560, 6912
+    h = synth.activations(M, d, seed=30 + M, outliers=False)
+    h_dev = h.to(cuda_device)
+    for layer in range(2):
+        (Wg, gg, Wgr, ggr), (Wu, gu, Wur, gur), (Wd, gd, Wdr, gdr) = ffn_weights(layer + 7, d, f, cuda_device)
+        y_dev = bl.ffn(Wg, gg, Wu, gu, Wd, gd, h_dev, residual=h_dev)
+        ref = oracle.ffn_layer(Wgr, ggr, Wur, gur, Wdr, gdr, bits(h_dev), residual=bits(h_dev))
+        assert_bf16_close(bits(y_dev), ref["y"], f"M={M} layer {layer}")
+        assert_bf16_exact(bits(y_dev), ref["y"], f"M={M} layer {layer}")
+        h_dev = y_dev
+
+
 def test_ffn_small_ragged(cuda_device):
     d, f, M = 64, 200, 3
     Wg, Wu, Wd = (make_weights(f, d, 0.02, 1), make_weights(f, d, 0.02, 2), make_weights(d, f, 0.02, 3))
