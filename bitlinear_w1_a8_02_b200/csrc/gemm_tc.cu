@@ -31,13 +31,10 @@ namespace bl {
 namespace {
 
 constexpr int BM = 128;               // tokens per tile (TMEM lanes)
-constexpr int BN = 256;               // weight rows per tile (TMEM columns per accumulator)
 constexpr int BK = 128;               // codes per k-block (one 128-byte swizzle row)
 constexpr int TSTAGES = 6;            // TMA ring: activation codes + packed weights
 constexpr int USTAGES = 2;            // unpacked weight-code ring
 constexpr int A_BYTES = BM * BK;      // 16 KiB activation codes
-constexpr int P_BYTES = BN * BK / 4;  //  8 KiB packed weights
-constexpr int U_BYTES = BN * BK;      // 32 KiB unpacked weight codes
 #ifndef BL_GEMM_UNPACK_WARPS
 #define BL_GEMM_UNPACK_WARPS 4
 #endif
@@ -45,15 +42,22 @@ constexpr int UNPACK_WARPS = BL_GEMM_UNPACK_WARPS;
 constexpr int UNPACK_THREADS = 32 * UNPACK_WARPS;
 constexpr int EPI_THREADS = 128;
 constexpr int THREADS = 64 + UNPACK_THREADS + EPI_THREADS;  // TMA, MMA, unpack, epilogue warps
-constexpr int UNPACK_VEC = BN * BK / 4 / 16 / UNPACK_THREADS;  // 16-byte packed groups per thread
-constexpr uint32_t TMEM_COLS = 2 * BN;  // two accumulators: epilogue of tile t overlaps tile t+1
 constexpr uint64_t WAIT_LIMIT_NS = 1000000000ull;
 constexpr int NUM_BARS = 2 * TSTAGES + 2 * USTAGES + 4;
-constexpr size_t SMEM_BYTES =
-    1024 /*alignment slack*/ + TSTAGES * (A_BYTES + P_BYTES) + USTAGES * U_BYTES + NUM_BARS * 8;
 
-static_assert(BN * BK / 4 / 16 % UNPACK_THREADS == 0, "unpack work must split evenly");
-static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+// Sizes that follow from the tile width BN (weight rows per tile = TMEM columns
+// per accumulator): 256 normally, 128 or 64 when wider tiles cannot fill the SMs.
+template <int BN>
+struct TileCfg {
+    static constexpr int P_BYTES = BN * BK / 4;  // packed weights per k-block
+    static constexpr int U_BYTES = BN * BK;      // unpacked weight codes per k-block
+    static constexpr int UNPACK_VEC = BN * BK / 4 / 16 / UNPACK_THREADS;  // 16-byte groups per thread
+    static constexpr uint32_t TMEM_COLS = 2 * BN;  // two accumulators: epilogue of tile t overlaps t+1
+    static constexpr size_t SMEM_BYTES =
+        1024 /*alignment slack*/ + TSTAGES * (A_BYTES + P_BYTES) + USTAGES * U_BYTES + NUM_BARS * 8;
+    static_assert(BN * BK / 4 / 16 % UNPACK_THREADS == 0, "unpack work must split evenly");
+    static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+};
 
 __device__ __forceinline__ bool aligned16(const void* p) {
     return (reinterpret_cast<uintptr_t>(p) & 15u) == 0;
@@ -128,11 +132,16 @@ __device__ __forceinline__ void store_row_chunk(const uint32_t (&v)[32], int xs,
 
 // Persistent CTAs walk the (m-tile, n-tile) grid with n fastest, so the CTAs in
 // flight share activation tiles and the whole packed weight stays in L2.
+template <int BN>
 __global__ void __launch_bounds__(THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    int M, int N, int K, const float* __restrict__ gamma_p,
                    const float* __restrict__ scale, const int32_t* __restrict__ xsum, GemvOut out,
                    unsigned* err) {
+    constexpr int P_BYTES = TileCfg<BN>::P_BYTES;
+    constexpr int U_BYTES = TileCfg<BN>::U_BYTES;
+    constexpr int UNPACK_VEC = TileCfg<BN>::UNPACK_VEC;
+    constexpr uint32_t TMEM_COLS = TileCfg<BN>::TMEM_COLS;
     extern __shared__ uint8_t smem_raw[];
     __shared__ uint32_t tmem_base_sh;
     __shared__ int abort_sh;
@@ -382,10 +391,12 @@ bool gemm_tc_ok(int64_t N, int64_t K, const void* Wp, const void* xq) {
            reinterpret_cast<uintptr_t>(xq) % 16 == 0;
 }
 
-cudaError_t launch_gemm_tc(const uint8_t* Wp, const float* gamma, int64_t N, int64_t K,
-                           const int8_t* xq_g16t, const float* scale, const int32_t* xsum, int64_t M,
-                           const GemvOut& out, cudaStream_t s) {
-    if (M == 0 || N == 0) return cudaSuccess;
+namespace {
+template <int BN>
+cudaError_t launch_bn(const uint8_t* Wp, const float* gamma, int64_t N, int64_t K, const int8_t* xq_g16t,
+                      const float* scale, const int32_t* xsum, int64_t M, const GemvOut& out,
+                      cudaStream_t s, int dev, int sms) {
+    constexpr size_t smem = TileCfg<BN>::SMEM_BYTES;
     CUtensorMap mapA, mapB;
     if (!make_map(&mapA, xq_g16t, (uint64_t)M, (uint64_t)K, BM, BK, true) ||
         !make_map(&mapB, Wp, (uint64_t)N, (uint64_t)(K / 4), BN, BK / 4, false))
@@ -394,25 +405,57 @@ cudaError_t launch_gemm_tc(const uint8_t* Wp, const float* gamma, int64_t N, int
     cudaError_t e = device_error_word(&err);
     if (e != cudaSuccess) return e;
     static bool attr_set[64];
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev < 64 && !attr_set[dev]) {
-        e = cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)SMEM_BYTES);
+    if (dev >= 64 || !attr_set[dev]) {
+        e = cudaFuncSetAttribute(gemm_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        attr_set[dev] = true;
-    }
-    static int num_sms[64];
-    if (dev < 64 && !num_sms[dev]) {
-        e = cudaDeviceGetAttribute(&num_sms[dev], cudaDevAttrMultiProcessorCount, dev);
-        if (e != cudaSuccess) return e;
+        if (dev < 64) attr_set[dev] = true;
     }
     const int64_t tiles = ((N + BN - 1) / BN) * ((M + BM - 1) / BM);
-    const int sms = dev < 64 ? num_sms[dev] : 148;
     const unsigned grid = (unsigned)(tiles < sms ? tiles : sms);
-    gemm_tc_kernel<<<grid, THREADS, SMEM_BYTES, s>>>(mapA, mapB, (int)M, (int)N, (int)K, gamma, scale,
-                                                     xsum, out, err);
+    gemm_tc_kernel<BN><<<grid, THREADS, smem, s>>>(mapA, mapB, (int)M, (int)N, (int)K, gamma, scale, xsum,
+                                                   out, err);
     return cudaGetLastError();
+}
+}  // namespace
+
+// Tile width: 256 weight rows per tile unless narrower tiles finish sooner. The
+// estimate is waves x relative time of one tile; a narrower tile still loads the
+// whole activation tile and pays the same per-k-block overheads, so on B200 a
+// 128-row tile takes 0.68 and a 64-row tile 0.59 of a 256-row tile (measured).
+int gemm_tc_tile_width(int64_t M, int64_t N, int sms) {
+    const int64_t mt = (M + BM - 1) / BM;
+    const int widths[3] = {256, 128, 64};
+    const double tile_cost[3] = {1.0, 0.68, 0.59};
+    int best = 256;
+    double best_time = 0.0;
+    for (int i = 0; i < 3; ++i) {
+        const int64_t tiles = mt * ((N + widths[i] - 1) / widths[i]);
+        const double time = (double)((tiles + sms - 1) / sms) * tile_cost[i];
+        if (i == 0 || time < best_time - 1e-9) {
+            best = widths[i];
+            best_time = time;
+        }
+    }
+    return best;
+}
+
+cudaError_t launch_gemm_tc(const uint8_t* Wp, const float* gamma, int64_t N, int64_t K,
+                           const int8_t* xq_g16t, const float* scale, const int32_t* xsum, int64_t M,
+                           const GemvOut& out, cudaStream_t s) {
+    if (M == 0 || N == 0) return cudaSuccess;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    static int num_sms[64];
+    if (dev < 64 && !num_sms[dev]) {
+        cudaError_t e = cudaDeviceGetAttribute(&num_sms[dev], cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return e;
+    }
+    const int sms = dev < 64 ? num_sms[dev] : 148;
+    switch (gemm_tc_tile_width(M, N, sms)) {
+        case 64: return launch_bn<64>(Wp, gamma, N, K, xq_g16t, scale, xsum, M, out, s, dev, sms);
+        case 128: return launch_bn<128>(Wp, gamma, N, K, xq_g16t, scale, xsum, M, out, s, dev, sms);
+        default: return launch_bn<256>(Wp, gamma, N, K, xq_g16t, scale, xsum, M, out, s, dev, sms);
+    }
 }
 
 }  // namespace bl

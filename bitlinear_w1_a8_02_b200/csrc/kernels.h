@@ -57,6 +57,7 @@ cudaError_t launch_gemv_generic(const uint8_t* Wp, const float* gamma, int64_t N
 // xq_g16t: G16T layout codes for M tokens. Requires K % 64 == 0 and 16-byte
 // aligned Wp and xq_g16t (TMA); any M, N (tails are zero-filled by the TMA).
 bool gemm_tc_ok(int64_t N, int64_t K, const void* Wp, const void* xq);
+int gemm_tc_tile_width(int64_t M, int64_t N, int sms);
 cudaError_t launch_gemm_tc(const uint8_t* Wp, const float* gamma, int64_t N, int64_t K,
                            const int8_t* xq_g16t, const float* scale, const int32_t* xsum, int64_t M,
                            const GemvOut& out, cudaStream_t s);

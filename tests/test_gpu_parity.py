@@ -156,10 +156,11 @@ def test_forward_ragged_shapes(cuda_device, M, N, K):
 
 
 @pytest.mark.parametrize("M,N,K", [(129, 257, 64), (300, 512, 320), (33, 1000, 2560),
-                                   (4096, 256, 128), (17, 8, 64)])
+                                   (4096, 256, 128), (17, 8, 64), (512, 2400, 128), (64, 1000, 192)])
 def test_forward_tensor_core_tails(cuda_device, M, N, K):
     """M > 16 runs the tcgen05 GEMM: token, row and k-block tails, N not a
-    multiple of the 256-row tile, K not a multiple of the 128-code k-block."""
+    multiple of the weight-row tile, K not a multiple of the 128-code k-block.
+    The last two shapes pick the 128- and 64-row tiles."""
     W = make_weights(N, K, 0.02, seed=M + 3 * N + K)
     Wp, gamma, Wp_ref, g_ref = pack_both(W, cuda_device)
     x = synth.activations(M, K, seed=N, outliers=True)
