@@ -40,6 +40,7 @@ SIGNATURES = {
     "bitlinear_forward_noalloc": (_ST, [_P, _P, _I, _I, _P, _I, _P, _P, _P, _P]),
     "bitlinear_validate_packed": (_ST, [_P, _I, _I, _P, _P, _S, _P]),
     "bitlinear_get_device_error": (_ST, [_P]),
+    "bitlinear_selftest_timeout": (_ST, [_I, _P]),
 }
 
 

@@ -130,8 +130,9 @@ bl_status bitlinear_quant_act(const uint16_t* x, int64_t M, int64_t K,
  *   acc       [M, N] device int32 output of the exact accumulator; may be NULL
  *   ws        device workspace of bitlinear_workspace_bytes(BL_OP_FORWARD, M, N, K) bytes
  * Kernel choice: M <= 16 streams the packed weights once through a
- * bandwidth-bound GEMV; larger M runs the tensor-core GEMM when the shape allows
- * it (N % 256 == 0 and K % 128 == 0), else a batched GEMV. Every path gives the same bits.
+ * bandwidth-bound GEMV (K % 256 == 0, Wp and x 16-byte aligned); larger M runs
+ * the tensor-core GEMM (K % 64 == 0, same alignment, any N); other shapes take a
+ * generic kernel. Every path gives the same bits.
  */
 bl_status bitlinear_forward(const uint8_t* Wp, const float* gamma, int64_t N, int64_t K,
                             const uint16_t* x, int64_t M, const uint16_t* residual,
@@ -201,6 +202,17 @@ bl_status bitlinear_validate_packed(const uint8_t* Wp, int64_t N, int64_t K, int
  * could not finish and returned); the timeout flag is cleared by this call.
  */
 bl_status bitlinear_get_device_error(bl_stream_t stream);
+
+/*
+ * Self-test of the failure path (the pages have no counterpart; it exists to
+ * test this library's error reporting). Launches, on `stream`, one thread that
+ * waits with the library's bounded mbarrier wait on a barrier nothing arrives
+ * on; after limit_us microseconds (1 .. 2,000,000) the wait gives up, records a
+ * timeout in the device error word and the kernel returns normally. The next
+ * bitlinear_get_device_error on this device then reports BL_ERR_TIMEOUT (and
+ * clears it). The GPU context stays usable. Returns the launch status.
+ */
+bl_status bitlinear_selftest_timeout(int64_t limit_us, bl_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -130,6 +130,12 @@ def test_host_validation_pack_quant_ffn_validate():
     assert v(None, 4, 16, None, P(A), 256, None) == NULL
 
 
+def test_host_validation_selftest():
+    L = bl.lib()
+    assert L.bitlinear_selftest_timeout(0, None) == SHAPE
+    assert L.bitlinear_selftest_timeout(3_000_000, None) == SHAPE
+
+
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device answer")
 def test_valid_call_without_device_is_unsupported():
     L = bl.lib()

@@ -217,6 +217,21 @@ def test_device_error_clean(cuda_device):
     assert bl.get_device_error() == 0
 
 
+def test_bounded_wait_reports_timeout(cuda_device):
+    """A wait that nothing satisfies gives up after its limit, the kernel returns,
+    the host sees BL_ERR_TIMEOUT once, and the context keeps working."""
+    import ctypes
+    BL_ERR_TIMEOUT = 8
+    stream = ctypes.c_void_p(torch.cuda.current_stream(cuda_device).cuda_stream)
+    assert bl.get_device_error() == 0
+    assert bl.lib().bitlinear_selftest_timeout(20000, stream) == 0
+    assert bl.get_device_error() == BL_ERR_TIMEOUT
+    assert bl.get_device_error() == 0
+    W = make_weights(64, 256, 0.02, seed=12)
+    Wp, gamma, Wp_ref, g_ref = pack_both(W, cuda_device)
+    check_forward_full(Wp, gamma, Wp_ref, g_ref, synth.activations(2, 256, seed=13), cuda_device)
+
+
 # ----------------------------------------------------------------------------- FFN
 
 def ffn_weights(layer, d, f, dev):
