@@ -2,11 +2,12 @@
 //
 // Paper card "BitNet b1.58 2B4T Technical Report", "Method Adaptation": the
 // packed int8 weights are loaded on chip, unpacked right before the matmul and
-// multiplied with the int8 activations (pack-store-load-unpack-compute). Here
-// the packed bytes stream from HBM straight into registers (16-byte loads that
-// skip L1), are unpacked there with one AND per 4 codes, and feed int8 tensor-core
-// MMAs (m16n8k32, u8 weights x s8 activations, int32 accumulators). Nothing of the
-// weight is staged or re-read.
+// multiplied with the int8 activations (pack-store-load-unpack-compute). Here a
+// producer warp copies the packed rows with 1-D bulk copies (TMA engine) into a
+// ring of shared-memory stages; eight consumer warps read them into registers,
+// unpack there with one AND per 4 codes and feed int8 tensor-core MMAs
+// (m16n8k32, u8 weights x s8 activations, int32 accumulators). Each weight byte
+// is read from DRAM once.
 //
 // Unpacking without shifts. A packed 32-bit word holds 16 codes c = q + 1; the
 // i-th 2-bit field of its 4 bytes is (word & (0x03030303 << 2i)), i.e. the codes
@@ -16,11 +17,11 @@
 // is laid out in PLANES (plane i holds xq[4j + i] at byte j), so a field of a
 // weight word and a word of plane i cover the same k.
 //
-// Work split: persistent CTAs walk tiles of 16 output rows; the 8 warps of a CTA
-// split K in 64-byte column chunks, partial sums meet in shared memory and the
-// dequantisation epilogue is fused. Each CTA asks the TMA engine to prefetch the
-// weight rows of the tiles it will reach next into L2, so DRAM streams
-// continuously while the warps work on the current tile.
+// Work split: persistent CTAs walk units of 16 output rows x one K segment
+// (at most 2 KiB of each row); the 8 warps of a CTA split a unit in 64-byte column
+// chunks, partial sums meet in shared memory and the dequantisation epilogue is
+// fused. Before the dependency wait each CTA asks for its first tiles to be
+// prefetched into L2, so DRAM already streams while the previous kernel ends.
 //
 // Fused activation quantisation: when the codes of all M tokens fit in shared
 // memory, each CTA quantises x itself (absmax per token, then PLANES codes into
@@ -120,144 +121,132 @@ __device__ __forceinline__ void consumer_sync() { asm volatile("bar.sync 1, 256;
 // +64 per token keeps the tokens of one quarter-warp on different banks.
 __device__ __forceinline__ int smem_plane_off(int m, int i, int KB) { return m * (4 * KB + 64) + i * KB; }
 
-// Quantise the M tokens of x into shared-memory PLANES codes (all threads).
-// Thread q handles 16-element groups q, q + 256, ...; the first kRegGroups of them
-// stay in registers between the absmax pass and the code pass, so x is read once.
-constexpr int kRegGroups = 4;
+// Per-token quantisation inside the kernel. It runs once per launch from a cold
+// instruction cache, so code size rather than arithmetic sets its latency: the
+// loops stay rolled and each token costs one barrier.
 
-template <int TOK>
-__device__ __forceinline__ void fold_absmax(float (&am)[TOK], int m, uint4 v0, uint4 v1) {
-    const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-    float r = 0.0f;
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-        r = fmaxf(r, fabsf(__uint_as_float(w[e] << 16)));
-        r = fmaxf(r, fabsf(__uint_as_float(w[e] & 0xffff0000u)));
-    }
-#pragma unroll
-    for (int mm = 0; mm < TOK; ++mm)
-        if (mm == m) am[mm] = fmaxf(am[mm], r);
+__device__ __forceinline__ uint32_t bf16x2_max(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("max.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
 }
 
-// Returns the sum of the 16 codes (accumulated per token by the caller).
-__device__ __forceinline__ int quantise_group(uint8_t* codes, int KB, int m, int c, uint4 v0, uint4 v1,
-                                              float s) {
-    const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-    unsigned pw[4] = {0u, 0u, 0u, 0u};
+// max |x| over 16 bf16 values, returned as a bf16 bit pattern (sign bits cleared,
+// so the patterns order like the values).
+__device__ __forceinline__ uint32_t absmax16(uint4 v0, uint4 v1) {
+    constexpr uint32_t k = 0x7fff7fffu;
+    const uint32_t a = bf16x2_max(bf16x2_max(v0.x & k, v0.y & k), bf16x2_max(v0.z & k, v0.w & k));
+    const uint32_t b = bf16x2_max(bf16x2_max(v1.x & k, v1.y & k), bf16x2_max(v1.z & k, v1.w & k));
+    const uint32_t c = bf16x2_max(a, b);
+    return max(c & 0xffffu, c >> 16);
+}
+
+// PLANES codes of 16 consecutive elements k = 16 g + e with fp32 values f[e]:
+// code rint(f s), taken from the low byte of fl(f s) + 1.5 * 2^23. The per-token
+// scale keeps |f s| <= 127 (1 + 2^-23) for finite inputs, so the clip to
+// [-128, 127] cannot bite and is left out. Plane i receives the codes of
+// e = i, 4 + i, 8 + i, 12 + i as one word. Returns the sum of the 16 codes.
+__device__ __forceinline__ int quant_pack16(const float (&f)[16], float s, uint8_t* plane0, int KB) {
+    uint32_t u[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) u[e] = __float_as_uint(__fadd_rn(__fmul_rn(f[e], s), 12582912.0f));
     int sum = 0;
 #pragma unroll
-    for (int e = 0; e < 16; ++e) {
-        const float f = (e & 1) ? __uint_as_float(w[e >> 1] & 0xffff0000u) : __uint_as_float(w[e >> 1] << 16);
-        const int q = quant_code(f, s);
-        sum += q;
-        pw[e & 3] |= static_cast<unsigned>(q & 255) << (8 * (e >> 2));
+    for (int i = 0; i < 4; ++i) {
+        const uint32_t w = __byte_perm(__byte_perm(u[i], u[4 + i], 0x0040),
+                                       __byte_perm(u[8 + i], u[12 + i], 0x0040), 0x5410);
+        *reinterpret_cast<uint32_t*>(plane0 + i * KB) = w;
+        sum = __dp4a(static_cast<int>(w), 0x01010101, sum);
     }
-#pragma unroll
-    for (int i = 0; i < 4; ++i) *reinterpret_cast<unsigned*>(codes + smem_plane_off(m, i, KB) + 4 * c) = pw[i];
     return sum;
 }
 
-template <int TOK>
-__device__ __forceinline__ void add_to_token(int (&xs)[TOK], int m, int v) {
+__device__ __forceinline__ int quant_bf16x16(uint4 v0, uint4 v1, float s, uint8_t* plane0, int KB) {
+    const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+    float f[16];
 #pragma unroll
-    for (int mm = 0; mm < TOK; ++mm)
-        if (mm == m) xs[mm] += v;
-}
-
-// Phase 1: load this thread's first kRegGroups groups of x into registers.
-struct XRegs {
-    uint4 v[kRegGroups][2];
-};
-
-__device__ __forceinline__ void fused_load(const uint16_t* __restrict__ x, int M, int KB, XRegs& xr) {
-    const int total = M * (KB / 4);
-    const uint4* xv = reinterpret_cast<const uint4*>(x);  // token m, group c at 2 * (m * groups + c)
-#pragma unroll
-    for (int j = 0; j < kRegGroups; ++j) {
-        const int q = threadIdx.x + kThreads * j;
-        if (q < total) {
-            xr.v[j][0] = xv[2 * q];
-            xr.v[j][1] = xv[2 * q + 1];
-        }
+    for (int j = 0; j < 8; ++j) {
+        f[2 * j] = __uint_as_float(w[j] << 16);
+        f[2 * j + 1] = __uint_as_float(w[j] & 0xffff0000u);
     }
+    return quant_pack16(f, s, plane0, KB);
 }
 
-// Phase 2: per-token absmax, scale, then PLANES codes into shared memory.
-template <int TOK>
-__device__ void fused_quantise(const uint16_t* __restrict__ x, int M, int KB, const XRegs& xr,
-                               uint8_t* codes, float* s_sh, int* xs_sh, float (*am_sh)[TOK]) {
+// bf16 x [M, K] -> PLANES codes of each token in shared memory (consumer threads).
+// Per token: absmax (warp reduction, one barrier), s = 127 / max(amax, eps),
+// codes, and the code sum. Thread 0 records s and the dequantisation factors
+// gamma / s. The first 16-element group of the next token is loaded while the
+// current one is reduced.
+template <bool DUAL>
+__device__ void fused_quantise(const GemvArgs& a, int KB, uint8_t* codes, uint32_t (*am_sh)[kWarps],
+                               float* s_sh, int* xs_sh, float* deq_sh, float* deq2_sh) {
     const int groups = KB / 4;  // 16-element groups per token
-    const int total = M * groups;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const uint4* xv = reinterpret_cast<const uint4*>(x);
-    float am[TOK];
-#pragma unroll
-    for (int mm = 0; mm < TOK; ++mm) am[mm] = 0.0f;
-    for (int q = threadIdx.x + kThreads * kRegGroups; q < total; q += kThreads)
-        fold_absmax<TOK>(am, q / groups, xv[2 * q], xv[2 * q + 1]);
-#pragma unroll
-    for (int j = 0; j < kRegGroups; ++j) {
-        const int q = threadIdx.x + kThreads * j;
-        if (q < total) fold_absmax<TOK>(am, q / groups, xr.v[j][0], xr.v[j][1]);
+    const int c0 = threadIdx.x;
+    const uint4* xv = reinterpret_cast<const uint4*>(a.x);
+    float gamma = 0.0f, gamma2 = 0.0f;
+    if (threadIdx.x == 0) {
+        gamma = *a.gamma;
+        if (DUAL) gamma2 = *a.gamma2;
     }
-#pragma unroll
-    for (int mm = 0; mm < TOK; ++mm) {
-        if (mm < M) {
-            const float r = warp_max(am[mm]);
-            if (lane == 0) am_sh[warp][mm] = r;
+    uint4 n0 = make_uint4(0, 0, 0, 0), n1 = n0;
+    if (c0 < groups) {
+        n0 = xv[2 * c0];
+        n1 = xv[2 * c0 + 1];
+    }
+#pragma unroll 1
+    for (int m = 0; m < a.M; ++m) {
+        const uint4* xr = xv + (size_t)m * 2 * groups;
+        const uint4 v0 = n0, v1 = n1;
+        if (m + 1 < a.M && c0 < groups) {
+            n0 = xr[2 * groups + 2 * c0];
+            n1 = xr[2 * groups + 2 * c0 + 1];
         }
-    }
-    if (threadIdx.x < TOK) xs_sh[threadIdx.x] = 0;
-    consumer_sync();
-    if (threadIdx.x < M) {
-        float r = am_sh[0][threadIdx.x];
+        uint32_t mx = absmax16(v0, v1);  // 0 when this thread has no group
+#pragma unroll 1
+        for (int c = c0 + kThreads; c < groups; c += kThreads) mx = max(mx, absmax16(xr[2 * c], xr[2 * c + 1]));
+        mx = __reduce_max_sync(0xffffffffu, mx);
+        if (lane == 0) am_sh[m][warp] = mx;
+        consumer_sync();
+        uint32_t amb = am_sh[m][0];
 #pragma unroll
-        for (int w = 1; w < kWarps; ++w) r = fmaxf(r, am_sh[w][threadIdx.x]);
-        s_sh[threadIdx.x] = __fdiv_rn(kActRange, fmaxf(r, kActEps));
-    }
-    consumer_sync();
-    // code sums: per-thread partials per token, a warp reduction, one atomic per warp
-    int xs[TOK];
-#pragma unroll
-    for (int mm = 0; mm < TOK; ++mm) xs[mm] = 0;
-#pragma unroll
-    for (int j = 0; j < kRegGroups; ++j) {
-        const int q = threadIdx.x + kThreads * j;
-        if (q < total) {
-            const int m = q / groups;
-            add_to_token<TOK>(xs, m, quantise_group(codes, KB, m, q - m * groups, xr.v[j][0], xr.v[j][1], s_sh[m]));
-        }
-    }
-    for (int q = threadIdx.x + kThreads * kRegGroups; q < total; q += kThreads) {
-        const int m = q / groups;
-        add_to_token<TOK>(xs, m, quantise_group(codes, KB, m, q - m * groups, xv[2 * q], xv[2 * q + 1], s_sh[m]));
-    }
-#pragma unroll
-    for (int mm = 0; mm < TOK; ++mm) {
-        if (mm < M) {
-            const int r = warp_sum(xs[mm]);
-            if (lane == 0) atomicAdd(&xs_sh[mm], r);
+        for (int w = 1; w < kWarps; ++w) amb = max(amb, am_sh[m][w]);
+        const float s = __fdiv_rn(kActRange, fmaxf(__uint_as_float(amb << 16), kActEps));
+        uint8_t* plane0 = codes + smem_plane_off(m, 0, KB);
+        int sum = 0;
+        if (c0 < groups) sum = quant_bf16x16(v0, v1, s, plane0 + 4 * c0, KB);
+#pragma unroll 1
+        for (int c = c0 + kThreads; c < groups; c += kThreads)
+            sum += quant_bf16x16(xr[2 * c], xr[2 * c + 1], s, plane0 + 4 * c, KB);
+        sum = __reduce_add_sync(0xffffffffu, sum);
+        if (lane == 0) atomicAdd(&xs_sh[m], sum);
+        if (threadIdx.x == 0) {
+            s_sh[m] = s;
+            deq_sh[m] = __fdiv_rn(gamma, s);
+            if (DUAL) deq2_sh[m] = __fdiv_rn(gamma2, s);
         }
     }
 }
 
-// FFN glue inside the down projection (one token per loop step, all consumer
-// threads): r = 1 / sqrtf(float(sum_j h_j^2 / f) + eps) from the up kernel's
-// per-tile fp64 partials (summed in tile order), s2 = 127 / max(max_j |h_j r|, eps)
-// with max_j |fl(h_j r)| = fl(max_j |h_j| r) (rounding is monotonic, r > 0), then
-// PLANES codes of fl(h_j r) into shared memory.
-template <int TOK>
+// FFN glue inside the down projection (consumer threads): per token,
+// r = 1 / sqrtf(float(sum_j h_j^2 / f) + eps) from the up kernel's per-tile fp64
+// partials (fixed order: thread strides, warp butterfly, warps in index order),
+// s2 = 127 / max(max_j |h_j r|, eps) with max_j |fl(h_j r)| = fl(max_j |h_j| r)
+// (rounding is monotonic, r > 0), then PLANES codes of fl(h_j r) into shared
+// memory. Thread 0 records s2 and gamma / s2.
 __device__ void finalise_quantise(const GemvArgs& a, int KB, uint8_t* codes, float* s_sh, int* xs_sh,
-                                  float* r_sh) {
+                                  float* r_sh, float* deq_sh) {
     const int f = 4 * KB;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     __shared__ double dred[kWarps];
     __shared__ float fred[kWarps];
-    if (threadIdx.x < TOK) xs_sh[threadIdx.x] = 0;
+    float gamma = 0.0f;
+    if (threadIdx.x == 0) gamma = *a.gamma;
+#pragma unroll 1
     for (int m = 0; m < a.M; ++m) {
-        // fixed order: thread strides, warp butterfly, warps in index order
         double ss = 0.0;
         float hmax = 0.0f;
+#pragma unroll 1
         for (int p = threadIdx.x; p < a.hin_parts; p += kThreads) {
             ss = __dadd_rn(ss, a.hin_ss[(size_t)m * a.hin_parts + p]);
             hmax = fmaxf(hmax, a.hin_max[(size_t)m * a.hin_parts + p]);
@@ -272,44 +261,41 @@ __device__ void finalise_quantise(const GemvArgs& a, int KB, uint8_t* codes, flo
         if (threadIdx.x == 0) {
             double tot = dred[0];
             float mx = fred[0];
+#pragma unroll 1
             for (int w = 1; w < kWarps; ++w) {
                 tot = __dadd_rn(tot, dred[w]);
                 mx = fmaxf(mx, fred[w]);
             }
             const float ms = __double2float_rn(__ddiv_rn(tot, (double)f));
             const float r = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, kRmsEps)));
+            const float s = __fdiv_rn(kActRange, fmaxf(__fmul_rn(mx, r), kActEps));
             r_sh[m] = r;
-            s_sh[m] = __fdiv_rn(kActRange, fmaxf(__fmul_rn(mx, r), kActEps));
+            s_sh[m] = s;
+            deq_sh[m] = __fdiv_rn(gamma, s);
         }
         consumer_sync();
     }
     const int groups = KB / 4;
+#pragma unroll 1
     for (int m = 0; m < a.M; ++m) {
         const float r = r_sh[m], s = s_sh[m];
         const float4* hr = reinterpret_cast<const float4*>(a.hin + (size_t)m * f);
+        uint8_t* plane0 = codes + smem_plane_off(m, 0, KB);
         int sum = 0;
+#pragma unroll 1
         for (int c = threadIdx.x; c < groups; c += kThreads) {
             float v[16];
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 const float4 h4 = hr[4 * c + q];
-                v[4 * q] = h4.x;
-                v[4 * q + 1] = h4.y;
-                v[4 * q + 2] = h4.z;
-                v[4 * q + 3] = h4.w;
+                v[4 * q] = __fmul_rn(h4.x, r);
+                v[4 * q + 1] = __fmul_rn(h4.y, r);
+                v[4 * q + 2] = __fmul_rn(h4.z, r);
+                v[4 * q + 3] = __fmul_rn(h4.w, r);
             }
-            unsigned pw[4] = {0u, 0u, 0u, 0u};
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-                const int q = quant_code(__fmul_rn(v[e], r), s);
-                sum += q;
-                pw[e & 3] |= static_cast<unsigned>(q & 255) << (8 * (e >> 2));
-            }
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-                *reinterpret_cast<unsigned*>(codes + smem_plane_off(m, i, KB) + 4 * c) = pw[i];
+            sum += quant_pack16(v, s, plane0 + 4 * c, KB);
         }
-        sum = warp_sum(sum);
+        sum = __reduce_add_sync(0xffffffffu, sum);
         if (lane == 0) atomicAdd(&xs_sh[m], sum);
     }
 }
@@ -337,8 +323,9 @@ __global__ void __launch_bounds__(kThreads + 32) gemv_mma_kernel(const GemvArgs 
     __shared__ int red2[DUAL ? kWarps : 1][16][TOK];
     __shared__ float s_sh[TOK];
     __shared__ int xs_sh[TOK];
-    __shared__ float am_sh[kWarps][TOK];
+    __shared__ uint32_t am_sh[TOK][kWarps];
     __shared__ float r_sh[TOK];
+    __shared__ float deq_sh[TOK], deq2_sh[TOK];
     __shared__ int abort_sh;
 
     const int N = a.N, KB = a.KB;
@@ -363,6 +350,7 @@ __global__ void __launch_bounds__(kThreads + 32) gemv_mma_kernel(const GemvArgs 
             tc::mbar_init(empty(st), kWarps);
         }
         abort_sh = 0;
+        for (int m = 0; m < TOK; ++m) xs_sh[m] = 0;
         tc::fence_mbar_init();
         // L2 prefetch of the first tiles may run before the previous kernel ends
         for (int p = 0; p < kPrefetchAhead; ++p) {
@@ -424,43 +412,36 @@ __global__ void __launch_bounds__(kThreads + 32) gemv_mma_kernel(const GemvArgs 
     // ---------------------------------------------------------------- consumers
     const int g8 = lane >> 2, t = lane & 3;
     if (SRC == SRC_X) {
-        XRegs xr;
-        fused_load(a.x, a.M, KB, xr);
-        fused_quantise<TOK>(a.x, a.M, KB, xr, codes, s_sh, xs_sh, am_sh);
+        fused_quantise<DUAL>(a, KB, codes, am_sh, s_sh, xs_sh, deq_sh, deq2_sh);
     } else if (SRC == SRC_H) {
-        finalise_quantise<TOK>(a, KB, codes, s_sh, xs_sh, r_sh);
+        finalise_quantise(a, KB, codes, s_sh, xs_sh, r_sh, deq_sh);
     } else if (threadIdx.x < TOK && tok0 + (int)threadIdx.x < a.M) {
-        s_sh[threadIdx.x] = a.scale[tok0 + threadIdx.x];
+        const float s = a.scale[tok0 + threadIdx.x];
+        s_sh[threadIdx.x] = s;
         xs_sh[threadIdx.x] = a.xsum[tok0 + threadIdx.x];
+        deq_sh[threadIdx.x] = __fdiv_rn(*a.gamma, s);
     }
-    consumer_sync();
-    __shared__ float deq_sh[TOK], deq2_sh[TOK];
-    if (threadIdx.x < TOK && tok0 + (int)threadIdx.x < a.M) {
-        deq_sh[threadIdx.x] = __fdiv_rn(*a.gamma, s_sh[threadIdx.x]);
-        if (DUAL) deq2_sh[threadIdx.x] = __fdiv_rn(*a.gamma2, s_sh[threadIdx.x]);
-    }
-    consumer_sync();
+    consumer_sync();  // codes, code sums and dequantisation factors are ready
 
-    // this lane's activation operand: token 8*nt + g8 of the group
+    // this lane's activation operand: token 8*nt + g8 of the group. Lanes past the
+    // last token read token 0's codes instead: they only feed output columns that
+    // are never stored, and loading them costs less than zeroing registers.
     const uint8_t* xbase[NT];
-    bool tv[NT];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
-        const int tok = tok0 + 8 * nt + g8;
-        tv[nt] = tok < a.M;
+        int tok = tok0 + 8 * nt + g8;
+        if (tok >= a.M) tok = 0;
         if (FUSED)
-            xbase[nt] = codes + smem_plane_off(tv[nt] ? tok : 0, 0, KB) + 16 * t;
+            xbase[nt] = codes + smem_plane_off(tok, 0, KB) + 16 * t;
         else
-            xbase[nt] = reinterpret_cast<const uint8_t*>(a.Xp) + (size_t)(tv[nt] ? tok : 0) * 4 * KB + 16 * t;
+            xbase[nt] = reinterpret_cast<const uint8_t*>(a.Xp) + (size_t)tok * 4 * KB + 16 * t;
     }
     auto load_x = [&](uint4 (&xv)[NT][4], int off) {
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                if (!tv[nt]) {
-                    xv[nt][i] = make_uint4(0, 0, 0, 0);
-                } else if (FUSED) {
+                if (FUSED) {
                     xv[nt][i] = *reinterpret_cast<const uint4*>(xbase[nt] + i * KB + off);
                 } else {
                     xv[nt][i] = ld_nc16(xbase[nt] + i * KB + off);
