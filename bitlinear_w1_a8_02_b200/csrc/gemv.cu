@@ -30,8 +30,9 @@
 //
 // Programmatic dependent launch: before waiting for the previous kernel in the
 // stream (griddepcontrol.wait) a CTA only issues L2 prefetches of its weights,
-// which cannot observe stale data (L2 is the point of coherence); every global
-// load of other data and every store comes after the wait.
+// which cannot observe stale data (L2 is the point of coherence), and sets up its
+// barriers; the producer arms its first stage before it waits. Every global load
+// of other data and every store comes after the wait.
 #include "common.cuh"
 #include "kernels.h"
 #include "tc_ptx.cuh"
@@ -180,7 +181,7 @@ __device__ __forceinline__ int quant_bf16x16(uint4 v0, uint4 v1, float s, uint8_
 template <bool DUAL>
 __device__ void fused_quantise(const GemvArgs& a, int KB, uint8_t* codes, uint32_t (*am_sh)[kWarps],
                                float* s_sh, int* xs_sh, float* deq_sh, float* deq2_sh) {
-    const int groups = KB / 4;  // 16-element groups per token
+    const int M = a.M, groups = KB / 4;  // 16-element groups per token
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int c0 = threadIdx.x;
     const uint4* xv = reinterpret_cast<const uint4*>(a.x);
@@ -195,10 +196,10 @@ __device__ void fused_quantise(const GemvArgs& a, int KB, uint8_t* codes, uint32
         n1 = xv[2 * c0 + 1];
     }
 #pragma unroll 1
-    for (int m = 0; m < a.M; ++m) {
+    for (int m = 0; m < M; ++m) {
         const uint4* xr = xv + (size_t)m * 2 * groups;
         const uint4 v0 = n0, v1 = n1;
-        if (m + 1 < a.M && c0 < groups) {
+        if (m + 1 < M && c0 < groups) {
             n0 = xr[2 * groups + 2 * c0];
             n1 = xr[2 * groups + 2 * c0 + 1];
         }
@@ -314,7 +315,7 @@ __device__ __forceinline__ void bulk_copy(uint32_t dst, const void* src, uint32_
 // congruent to 64 mod 128 bytes so rows g and g + 1 of a quarter-warp fall on
 // different banks.
 template <int NT, int SRC, bool DUAL>
-__global__ void __launch_bounds__(kThreads + 32) gemv_mma_kernel(const GemvArgs a) {
+__global__ void __launch_bounds__(kThreads + 32, NT == 1 ? 3 : 2) gemv_mma_kernel(const GemvArgs a) {
     constexpr int TOK = 8 * NT;
     constexpr bool FUSED = SRC != SRC_CODES;
     constexpr int NW = DUAL ? 2 : 1;  // weight streams
@@ -364,13 +365,13 @@ __global__ void __launch_bounds__(kThreads + 32) gemv_mma_kernel(const GemvArgs 
     }
     __syncthreads();
     grid_dependents_launch();
-    grid_dependency_wait();
 
     if (warp == kWarps) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
             uint32_t g = 0;
             bool stop = false;
+            bool waited = false;
             for (int tile = blockIdx.x; tile < ntiles && !stop; tile += gridDim.x) {
                 const int n0 = tile * 16;
                 const int rows = min(16, N - n0);
@@ -388,6 +389,10 @@ __global__ void __launch_bounds__(kThreads + 32) gemv_mma_kernel(const GemvArgs 
                     const int c0 = sg * cps;
                     const uint32_t segb = (uint32_t)(min(cps, nchunks - c0) * 64);
                     tc::mbar_arrive_expect_tx(full(st), segb * rows * NW);
+                    if (!waited) {  // everything above touches shared memory only
+                        grid_dependency_wait();
+                        waited = true;
+                    }
                     const uint32_t dst = tc::smem_u32(stages + st * stage_bytes);
                     for (int r = 0; r < rows; ++r)
                         bulk_copy(dst + r * pitch, a.Wp + (size_t)(n0 + r) * KB + c0 * 64, segb, full(st));
@@ -411,17 +416,6 @@ __global__ void __launch_bounds__(kThreads + 32) gemv_mma_kernel(const GemvArgs 
 
     // ---------------------------------------------------------------- consumers
     const int g8 = lane >> 2, t = lane & 3;
-    if (SRC == SRC_X) {
-        fused_quantise<DUAL>(a, KB, codes, am_sh, s_sh, xs_sh, deq_sh, deq2_sh);
-    } else if (SRC == SRC_H) {
-        finalise_quantise(a, KB, codes, s_sh, xs_sh, r_sh, deq_sh);
-    } else if (threadIdx.x < TOK && tok0 + (int)threadIdx.x < a.M) {
-        const float s = a.scale[tok0 + threadIdx.x];
-        s_sh[threadIdx.x] = s;
-        xs_sh[threadIdx.x] = a.xsum[tok0 + threadIdx.x];
-        deq_sh[threadIdx.x] = __fdiv_rn(*a.gamma, s);
-    }
-    consumer_sync();  // codes, code sums and dequantisation factors are ready
 
     // this lane's activation operand: token 8*nt + g8 of the group. Lanes past the
     // last token read token 0's codes instead: they only feed output columns that
@@ -452,6 +446,20 @@ __global__ void __launch_bounds__(kThreads + 32) gemv_mma_kernel(const GemvArgs 
     // An abort (a bounded wait that gave up) keeps every consumer warp on the same
     // sequence of named barriers: later waits are skipped and nothing is stored.
     auto aborted = [&]() { return *reinterpret_cast<volatile int*>(&abort_sh) != 0; };
+
+    grid_dependency_wait();
+    if (SRC == SRC_X) {
+        fused_quantise<DUAL>(a, KB, codes, am_sh, s_sh, xs_sh, deq_sh, deq2_sh);
+    } else if (SRC == SRC_H) {
+        finalise_quantise(a, KB, codes, s_sh, xs_sh, r_sh, deq_sh);
+    } else if (threadIdx.x < TOK && tok0 + (int)threadIdx.x < a.M) {
+        const float s = a.scale[tok0 + threadIdx.x];
+        s_sh[threadIdx.x] = s;
+        xs_sh[threadIdx.x] = a.xsum[tok0 + threadIdx.x];
+        deq_sh[threadIdx.x] = __fdiv_rn(*a.gamma, s);
+    }
+    consumer_sync();  // codes, code sums and dequantisation factors are ready
+
     uint32_t g = 0;
     for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
         const int n0 = tile * 16;
@@ -483,7 +491,7 @@ __global__ void __launch_bounds__(kThreads + 32) gemv_mma_kernel(const GemvArgs 
             const int segc = min(cps, nchunks - c0);
             const uint8_t* sa = stages + st * stage_bytes + g8 * pitch + 16 * t;
             const uint8_t* sb = sa + 8 * pitch;
-#pragma unroll
+#pragma unroll 2
             for (int u = 0; u < kUnroll; ++u) {
                 const int cl = warp + kWarps * u;
                 if (cl < segc) {
@@ -514,15 +522,16 @@ __global__ void __launch_bounds__(kThreads + 32) gemv_mma_kernel(const GemvArgs 
                 red[warp][g8 + 8 * (e >> 1)][8 * nt + 2 * t + (e & 1)] = v;
                 if constexpr (DUAL) {
                     red2[warp][g8 + 8 * (e >> 1)][8 * nt + 2 * t + (e & 1)] =
-                        acc2[nt][0][e] + (acc2[nt][1][e] >> 2) + (acc2[nt][2][e] >> 4) + (acc2[nt][3][e] >> 6);
+                        acc2[nt][0][e] + (acc2[nt][1][e] >> 2) + (acc2[nt][2][e] >> 4) +
+                        (acc2[nt][3][e] >> 6);
                 }
             }
         consumer_sync();
 
+        const bool store = !aborted();
         if constexpr (DUAL) {
             // FFN up epilogue: h = relu(g)^2 * u, plus the tile's per-token sum of
             // h^2 (fp64, fixed butterfly order over the 16 rows) and max |h|.
-            const bool store_h = !aborted();
             for (int idx = threadIdx.x; idx < 16 * TOK; idx += kThreads) {
                 const int r = idx & 15, cl = idx >> 4;
                 const int n = n0 + r, m = tok0 + cl;
@@ -539,7 +548,7 @@ __global__ void __launch_bounds__(kThreads + 32) gemv_mma_kernel(const GemvArgs 
                     const float uv = dequant(su - xs_sh[cl], deq2_sh[cl]);
                     const float tv0 = gv > 0.0f ? gv : 0.0f;
                     hv = __fmul_rn(__fmul_rn(tv0, tv0), uv);
-                    if (store_h) a.h[(size_t)m * N + n] = hv;
+                    if (store) a.h[(size_t)m * N + n] = hv;
                 }
                 double ss = __dmul_rn((double)hv, (double)hv);
                 float mx = fabsf(hv);
@@ -548,33 +557,31 @@ __global__ void __launch_bounds__(kThreads + 32) gemv_mma_kernel(const GemvArgs 
                     ss = __dadd_rn(ss, __shfl_xor_sync(0xffffffffu, ss, o));
                     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
                 }
-                if (r == 0 && m < a.M && store_h) {
+                if (r == 0 && m < a.M && store) {
                     a.part_ss[(size_t)m * ntiles + tile] = ss;
                     a.part_max[(size_t)m * ntiles + tile] = mx;
                 }
             }
-            consumer_sync();
-            continue;
-        }
-
-        const bool store = !aborted();
-        for (int idx = threadIdx.x; store && idx < 16 * TOK; idx += kThreads) {
-            const int r = idx & 15, cl = idx >> 4;
-            const int n = n0 + r, m = tok0 + cl;
-            if (n >= N || m >= a.M) continue;
-            int sum = 0;
+        } else {
+            for (int idx = threadIdx.x; idx < 16 * TOK; idx += kThreads) {
+                const int r = idx & 15, cl = idx >> 4;
+                const int n = n0 + r, m = tok0 + cl;
+                if (n >= N || m >= a.M) continue;
+                int sum = 0;
 #pragma unroll
-            for (int w = 0; w < kWarps; ++w) sum += red[w][r][cl];
-            const int accv = sum - xs_sh[cl];
-            float v = dequant(accv, deq_sh[cl]);
-            const size_t o = (size_t)m * N + n;
-            if (a.out.y32) {
-                a.out.y32[o] = v;
-            } else {
-                if (a.out.residual) v = __fadd_rn(bf16_bits_to_f32(a.out.residual[o]), v);
-                a.out.y[o] = f32_to_bf16_bits(v);
+                for (int w = 0; w < kWarps; ++w) sum += red[w][r][cl];
+                const int accv = sum - xs_sh[cl];
+                float v = dequant(accv, deq_sh[cl]);
+                if (!store) continue;
+                const size_t o = (size_t)m * N + n;
+                if (a.out.y32) {
+                    a.out.y32[o] = v;
+                } else {
+                    if (a.out.residual) v = __fadd_rn(bf16_bits_to_f32(a.out.residual[o]), v);
+                    a.out.y[o] = f32_to_bf16_bits(v);
+                }
+                if (a.out.acc) a.out.acc[o] = accv;
             }
-            if (a.out.acc) a.out.acc[o] = accv;
         }
         consumer_sync();
     }
