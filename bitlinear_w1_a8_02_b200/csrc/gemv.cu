@@ -82,6 +82,20 @@ __device__ __forceinline__ void chunk_mma(int (&acc)[NT][4][4], const uint4& wa,
     }
 }
 
+// dp4a of the four 2-bit fields of a packed weight word (unsigned bytes code * 4^i)
+// against the four plane words of one token (signed bytes), one accumulator per field.
+__device__ __forceinline__ void dp4a_fields(int (&acc)[4], uint32_t w, const uint4& x) {
+    const uint32_t xw[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        asm("dp4a.u32.s32 %0, %1, %2, %0;" : "+r"(acc[i]) : "r"(w & (0x03030303u << (2 * i))), "r"(xw[i]));
+}
+
+// acc_u = A0 + A1 / 4 + A2 / 16 + A3 / 64; each Ai is an exact multiple of 4^i.
+__device__ __forceinline__ int fold_fields(const int (&acc)[4]) {
+    return acc[0] + (acc[1] >> 2) + (acc[2] >> 4) + (acc[3] >> 6);
+}
+
 struct GemvArgs {
     const uint8_t* Wp;
     const float* gamma;
@@ -146,22 +160,37 @@ __device__ __forceinline__ uint32_t absmax16(uint4 v0, uint4 v1) {
 // code rint(f s), taken from the low byte of fl(f s) + 1.5 * 2^23. The per-token
 // scale keeps |f s| <= 127 (1 + 2^-23) for finite inputs, so the clip to
 // [-128, 127] cannot bite and is left out. Plane i receives the codes of
-// e = i, 4 + i, 8 + i, 12 + i as one word. Returns the sum of the 16 codes.
+// e = i, 4 + i, 8 + i, 12 + i as one word, stored at plane0 + i * KB, or, in the
+// interleaved single-token layout (IL), the four plane words of group g side by
+// side at plane0 = codes + 16 g. Returns the sum of the 16 codes.
+template <bool IL>
 __device__ __forceinline__ int quant_pack16(const float (&f)[16], float s, uint8_t* plane0, int KB) {
     uint32_t u[16];
 #pragma unroll
     for (int e = 0; e < 16; ++e) u[e] = __float_as_uint(__fadd_rn(__fmul_rn(f[e], s), 12582912.0f));
+    uint32_t w[4];
     int sum = 0;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        const uint32_t w = __byte_perm(__byte_perm(u[i], u[4 + i], 0x0040),
-                                       __byte_perm(u[8 + i], u[12 + i], 0x0040), 0x5410);
-        *reinterpret_cast<uint32_t*>(plane0 + i * KB) = w;
-        sum = __dp4a(static_cast<int>(w), 0x01010101, sum);
+        w[i] = __byte_perm(__byte_perm(u[i], u[4 + i], 0x0040), __byte_perm(u[8 + i], u[12 + i], 0x0040), 0x5410);
+        sum = __dp4a(static_cast<int>(w[i]), 0x01010101, sum);
+    }
+    if (IL) {
+        *reinterpret_cast<uint4*>(plane0) = make_uint4(w[0], w[1], w[2], w[3]);
+    } else {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) *reinterpret_cast<uint32_t*>(plane0 + i * KB) = w[i];
     }
     return sum;
 }
 
+// Shared-memory address of the code words of 16-element group c of token m.
+template <bool IL>
+__device__ __forceinline__ uint8_t* group_codes(uint8_t* codes, int m, int c, int KB) {
+    return IL ? codes + 16 * c : codes + smem_plane_off(m, 0, KB) + 4 * c;
+}
+
+template <bool IL>
 __device__ __forceinline__ int quant_bf16x16(uint4 v0, uint4 v1, float s, uint8_t* plane0, int KB) {
     const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
     float f[16];
@@ -170,7 +199,7 @@ __device__ __forceinline__ int quant_bf16x16(uint4 v0, uint4 v1, float s, uint8_
         f[2 * j] = __uint_as_float(w[j] << 16);
         f[2 * j + 1] = __uint_as_float(w[j] & 0xffff0000u);
     }
-    return quant_pack16(f, s, plane0, KB);
+    return quant_pack16<IL>(f, s, plane0, KB);
 }
 
 // bf16 x [M, K] -> PLANES codes of each token in shared memory (consumer threads).
@@ -178,7 +207,7 @@ __device__ __forceinline__ int quant_bf16x16(uint4 v0, uint4 v1, float s, uint8_
 // codes, and the code sum. Thread 0 records s and the dequantisation factors
 // gamma / s. The first 16-element group of the next token is loaded while the
 // current one is reduced.
-template <bool DUAL>
+template <bool DUAL, bool IL>
 __device__ void fused_quantise(const GemvArgs& a, int KB, uint8_t* codes, uint32_t (*am_sh)[kWarps],
                                float* s_sh, int* xs_sh, float* deq_sh, float* deq2_sh) {
     const int M = a.M, groups = KB / 4;  // 16-element groups per token
@@ -213,12 +242,11 @@ __device__ void fused_quantise(const GemvArgs& a, int KB, uint8_t* codes, uint32
 #pragma unroll
         for (int w = 1; w < kWarps; ++w) amb = max(amb, am_sh[m][w]);
         const float s = __fdiv_rn(kActRange, fmaxf(__uint_as_float(amb << 16), kActEps));
-        uint8_t* plane0 = codes + smem_plane_off(m, 0, KB);
         int sum = 0;
-        if (c0 < groups) sum = quant_bf16x16(v0, v1, s, plane0 + 4 * c0, KB);
+        if (c0 < groups) sum = quant_bf16x16<IL>(v0, v1, s, group_codes<IL>(codes, m, c0, KB), KB);
 #pragma unroll 1
         for (int c = c0 + kThreads; c < groups; c += kThreads)
-            sum += quant_bf16x16(xr[2 * c], xr[2 * c + 1], s, plane0 + 4 * c, KB);
+            sum += quant_bf16x16<IL>(xr[2 * c], xr[2 * c + 1], s, group_codes<IL>(codes, m, c, KB), KB);
         sum = __reduce_add_sync(0xffffffffu, sum);
         if (lane == 0) atomicAdd(&xs_sh[m], sum);
         if (threadIdx.x == 0) {
@@ -235,6 +263,7 @@ __device__ void fused_quantise(const GemvArgs& a, int KB, uint8_t* codes, uint32
 // s2 = 127 / max(max_j |h_j r|, eps) with max_j |fl(h_j r)| = fl(max_j |h_j| r)
 // (rounding is monotonic, r > 0), then PLANES codes of fl(h_j r) into shared
 // memory. Thread 0 records s2 and gamma / s2.
+template <bool IL>
 __device__ void finalise_quantise(const GemvArgs& a, int KB, uint8_t* codes, float* s_sh, int* xs_sh,
                                   float* r_sh, float* deq_sh) {
     const int f = 4 * KB;
@@ -281,7 +310,6 @@ __device__ void finalise_quantise(const GemvArgs& a, int KB, uint8_t* codes, flo
     for (int m = 0; m < a.M; ++m) {
         const float r = r_sh[m], s = s_sh[m];
         const float4* hr = reinterpret_cast<const float4*>(a.hin + (size_t)m * f);
-        uint8_t* plane0 = codes + smem_plane_off(m, 0, KB);
         int sum = 0;
 #pragma unroll 1
         for (int c = threadIdx.x; c < groups; c += kThreads) {
@@ -294,7 +322,7 @@ __device__ void finalise_quantise(const GemvArgs& a, int KB, uint8_t* codes, flo
                 v[4 * q + 2] = __fmul_rn(h4.z, r);
                 v[4 * q + 3] = __fmul_rn(h4.w, r);
             }
-            sum += quant_pack16(v, s, plane0 + 4 * c, KB);
+            sum += quant_pack16<IL>(v, s, group_codes<IL>(codes, m, c, KB), KB);
         }
         sum = __reduce_add_sync(0xffffffffu, sum);
         if (lane == 0) atomicAdd(&xs_sh[m], sum);
@@ -314,10 +342,11 @@ __device__ __forceinline__ void bulk_copy(uint32_t dst, const void* src, uint32_
 // segments into a ring of kStages shared-memory stages; the row pitch is
 // congruent to 64 mod 128 bytes so rows g and g + 1 of a quarter-warp fall on
 // different banks.
-template <int NT, int SRC, bool DUAL>
+template <int NT, int SRC, bool DUAL, bool DP>
 __global__ void __launch_bounds__(kThreads + 32, NT == 1 ? 3 : 2) gemv_mma_kernel(const GemvArgs a) {
     constexpr int TOK = 8 * NT;
     constexpr bool FUSED = SRC != SRC_CODES;
+    static_assert(!DP || (FUSED && NT == 1), "the dp4a path reads one token's codes from shared memory");
     constexpr int NW = DUAL ? 2 : 1;  // weight streams
     extern __shared__ __align__(128) uint8_t dyn[];
     __shared__ int red[kWarps][16][TOK];
@@ -449,9 +478,9 @@ __global__ void __launch_bounds__(kThreads + 32, NT == 1 ? 3 : 2) gemv_mma_kerne
 
     grid_dependency_wait();
     if (SRC == SRC_X) {
-        fused_quantise<DUAL>(a, KB, codes, am_sh, s_sh, xs_sh, deq_sh, deq2_sh);
+        fused_quantise<DUAL, DP>(a, KB, codes, am_sh, s_sh, xs_sh, deq_sh, deq2_sh);
     } else if (SRC == SRC_H) {
-        finalise_quantise(a, KB, codes, s_sh, xs_sh, r_sh, deq_sh);
+        finalise_quantise<DP>(a, KB, codes, s_sh, xs_sh, r_sh, deq_sh);
     } else if (threadIdx.x < TOK && tok0 + (int)threadIdx.x < a.M) {
         const float s = a.scale[tok0 + threadIdx.x];
         s_sh[threadIdx.x] = s;
@@ -463,69 +492,122 @@ __global__ void __launch_bounds__(kThreads + 32, NT == 1 ? 3 : 2) gemv_mma_kerne
     uint32_t g = 0;
     for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
         const int n0 = tile * 16;
-        int acc[NT][4][4], acc2[NT][4][4];
+        if constexpr (DP) {
+            // One token: thread (row group rg, lane tl of 64) owns rows 4 rg .. 4 rg + 3
+            // of the unit and its words j = tl, tl + 64, ...; per word one dp4a per
+            // field against the interleaved plane words of the token.
+            const int rg = threadIdx.x >> 6, tl = threadIdx.x & 63;
+            int acc[4][4] = {}, acc2[DUAL ? 4 : 1][4] = {};
+            for (int sg = 0; sg < nseg; ++sg, ++g) {
+                const int st = g % kStages;
+                if (aborted()) continue;
+                if (!tc::mbar_wait(full(st), (g / kStages) & 1, kWaitLimitNs)) {
+                    atomicOr(a.err, 1u);
+                    atomicExch(&abort_sh, 1);
+                    continue;
+                }
+                const int words = min(cps, nchunks - sg * cps) * 16;
+                const uint8_t* wr = stages + st * stage_bytes + 4 * rg * pitch;
+                const uint4* xw = reinterpret_cast<const uint4*>(codes) + sg * cps * 16;
+#pragma unroll 2
+                for (int j = tl; j < words; j += 64) {
+                    const uint4 xv = xw[j];
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
+                    for (int r = 0; r < 4; ++r) {
+                        const uint32_t w = *reinterpret_cast<const uint32_t*>(wr + r * pitch + 4 * j);
+                        dp4a_fields(acc[r], w, xv);
+                        if constexpr (DUAL) {
+                            const uint32_t w2 = *reinterpret_cast<const uint32_t*>(wr + (16 + r) * pitch + 4 * j);
+                            dp4a_fields(acc2[r], w2, xv);
+                        }
+                    }
+                }
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(empty(st));
+            }
+            // fold the fields, sum the warp, and leave this warp's share of each of
+            // the 16 rows (zero for rows of the other groups) as token 0's column
+            int v[4], v2[4];
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) acc[nt][i][e] = 0;
-        if constexpr (DUAL) {
+            for (int r = 0; r < 4; ++r) {
+                v[r] = __reduce_add_sync(0xffffffffu, fold_fields(acc[r]));
+                if constexpr (DUAL) v2[r] = __reduce_add_sync(0xffffffffu, fold_fields(acc2[r]));
+            }
+            if (lane < 16) {
+                const bool mine = (lane >> 2) == rg;
+                const int q = lane & 3;
+                const int pick = q == 0 ? v[0] : q == 1 ? v[1] : q == 2 ? v[2] : v[3];
+                red[warp][lane][0] = mine ? pick : 0;
+                if constexpr (DUAL) {
+                    const int pick2 = q == 0 ? v2[0] : q == 1 ? v2[1] : q == 2 ? v2[2] : v2[3];
+                    red2[warp][lane][0] = mine ? pick2 : 0;
+                }
+            }
+        } else {
+            int acc[NT][4][4], acc2[NT][4][4];
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
                 for (int i = 0; i < 4; ++i)
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) acc2[nt][i][e] = 0;
-        }
-
-        for (int sg = 0; sg < nseg; ++sg, ++g) {
-            const int st = g % kStages;
-            if (aborted()) continue;
-            if (!tc::mbar_wait(full(st), (g / kStages) & 1, kWaitLimitNs)) {
-                atomicOr(a.err, 1u);
-                atomicExch(&abort_sh, 1);
-                continue;
+                    for (int e = 0; e < 4; ++e) acc[nt][i][e] = 0;
+            if constexpr (DUAL) {
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) acc2[nt][i][e] = 0;
             }
-            const int c0 = sg * cps;
-            const int segc = min(cps, nchunks - c0);
-            const uint8_t* sa = stages + st * stage_bytes + g8 * pitch + 16 * t;
-            const uint8_t* sb = sa + 8 * pitch;
+
+            for (int sg = 0; sg < nseg; ++sg, ++g) {
+                const int st = g % kStages;
+                if (aborted()) continue;
+                if (!tc::mbar_wait(full(st), (g / kStages) & 1, kWaitLimitNs)) {
+                    atomicOr(a.err, 1u);
+                    atomicExch(&abort_sh, 1);
+                    continue;
+                }
+                const int c0 = sg * cps;
+                const int segc = min(cps, nchunks - c0);
+                const uint8_t* sa = stages + st * stage_bytes + g8 * pitch + 16 * t;
+                const uint8_t* sb = sa + 8 * pitch;
 #pragma unroll 2
-            for (int u = 0; u < kUnroll; ++u) {
-                const int cl = warp + kWarps * u;
-                if (cl < segc) {
-                    const uint4 wa = *reinterpret_cast<const uint4*>(sa + 64 * cl);
-                    const uint4 wb = *reinterpret_cast<const uint4*>(sb + 64 * cl);
-                    uint4 xv[NT][4];
-                    load_x(xv, 64 * (c0 + cl));
-                    chunk_mma<NT>(acc, wa, wb, xv);
-                    if constexpr (DUAL) {
-                        const uint4 wc = *reinterpret_cast<const uint4*>(sa + 16 * pitch + 64 * cl);
-                        const uint4 wd = *reinterpret_cast<const uint4*>(sb + 16 * pitch + 64 * cl);
-                        chunk_mma<NT>(acc2, wc, wd, xv);
+                for (int u = 0; u < kUnroll; ++u) {
+                    const int cl = warp + kWarps * u;
+                    if (cl < segc) {
+                        const uint4 wa = *reinterpret_cast<const uint4*>(sa + 64 * cl);
+                        const uint4 wb = *reinterpret_cast<const uint4*>(sb + 64 * cl);
+                        uint4 xv[NT][4];
+                        load_x(xv, 64 * (c0 + cl));
+                        chunk_mma<NT>(acc, wa, wb, xv);
+                        if constexpr (DUAL) {
+                            const uint4 wc = *reinterpret_cast<const uint4*>(sa + 16 * pitch + 64 * cl);
+                            const uint4 wd = *reinterpret_cast<const uint4*>(sb + 16 * pitch + 64 * cl);
+                            chunk_mma<NT>(acc2, wc, wd, xv);
+                        }
                     }
                 }
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(empty(st));
             }
-            __syncwarp();
-            if (lane == 0) tc::mbar_arrive(empty(st));
-        }
 
-        // Fold the four field accumulators; D element e sits at row g8 + 8*(e >> 1),
-        // token 8*nt + 2t + (e & 1).
+            // Fold the four field accumulators; D element e sits at row g8 + 8*(e >> 1),
+            // token 8*nt + 2t + (e & 1).
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
+            for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int v = acc[nt][0][e] + (acc[nt][1][e] >> 2) + (acc[nt][2][e] >> 4) +
-                              (acc[nt][3][e] >> 6);
-                red[warp][g8 + 8 * (e >> 1)][8 * nt + 2 * t + (e & 1)] = v;
-                if constexpr (DUAL) {
-                    red2[warp][g8 + 8 * (e >> 1)][8 * nt + 2 * t + (e & 1)] =
-                        acc2[nt][0][e] + (acc2[nt][1][e] >> 2) + (acc2[nt][2][e] >> 4) +
-                        (acc2[nt][3][e] >> 6);
+                for (int e = 0; e < 4; ++e) {
+                    const int v = acc[nt][0][e] + (acc[nt][1][e] >> 2) + (acc[nt][2][e] >> 4) +
+                                  (acc[nt][3][e] >> 6);
+                    red[warp][g8 + 8 * (e >> 1)][8 * nt + 2 * t + (e & 1)] = v;
+                    if constexpr (DUAL) {
+                        red2[warp][g8 + 8 * (e >> 1)][8 * nt + 2 * t + (e & 1)] =
+                            acc2[nt][0][e] + (acc2[nt][1][e] >> 2) + (acc2[nt][2][e] >> 4) +
+                            (acc2[nt][3][e] >> 6);
+                    }
                 }
-            }
+        }
         consumer_sync();
 
         const bool store = !aborted();
@@ -631,9 +713,9 @@ int sm_count() {
     return n;
 }
 
-template <int NT, int SRC, bool DUAL>
+template <int NT, int SRC, bool DUAL, bool DP = false>
 cudaError_t launch_variant(const GemvArgs& a, dim3 grid, size_t smem, cudaStream_t s) {
-    auto kern = gemv_mma_kernel<NT, SRC, DUAL>;
+    auto kern = gemv_mma_kernel<NT, SRC, DUAL, DP>;
     static bool done[64];
     int dev = 0;
     cudaGetDevice(&dev);
@@ -643,6 +725,14 @@ cudaError_t launch_variant(const GemvArgs& a, dim3 grid, size_t smem, cudaStream
         if (dev < 64) done[dev] = true;
     }
     return launch_pdl(kern, grid, dim3(kThreads + 32), smem, s, a);
+}
+
+// Codes in shared memory: a single token takes the dp4a path (the MMA path would
+// spend 7 of its 8 token columns on padding).
+template <int SRC, bool DUAL>
+cudaError_t launch_fused(const GemvArgs& a, dim3 grid, size_t smem, cudaStream_t s) {
+    if (a.M == 1) return launch_variant<1, SRC, DUAL, true>(a, grid, smem, s);
+    return launch_variant<1, SRC, DUAL, false>(a, grid, smem, s);
 }
 
 // Segment plan, shared-memory size and grid of one streamed GEMV launch.
@@ -705,7 +795,7 @@ cudaError_t launch_gemv(const uint8_t* Wp, const float* gamma, int64_t N, int64_
     StreamPlan p;
     cudaError_t e = plan_stream(a, N, K, M, 1, x_fused != nullptr, p);
     if (e != cudaSuccess) return e;
-    if (x_fused) return launch_variant<1, SRC_X, false>(a, dim3(p.grid_x, 1), p.smem, s);
+    if (x_fused) return launch_fused<SRC_X, false>(a, dim3(p.grid_x, 1), p.smem, s);
     if (M <= 8) return launch_variant<1, SRC_CODES, false>(a, dim3(p.grid_x, 1), p.smem, s);
     return launch_variant<2, SRC_CODES, false>(a, dim3(p.grid_x, (unsigned)((M + 15) / 16)), p.smem, s);
 }
@@ -725,7 +815,7 @@ cudaError_t launch_ffn_up_fused(const uint8_t* Wg, const float* gg, const uint8_
     StreamPlan p;
     cudaError_t e = plan_stream(a, f, d, M, 2, true, p);
     if (e != cudaSuccess) return e;
-    return launch_variant<1, SRC_X, true>(a, dim3(p.grid_x, 1), p.smem, s);
+    return launch_fused<SRC_X, true>(a, dim3(p.grid_x, 1), p.smem, s);
 }
 
 cudaError_t launch_ffn_down_fused(const uint8_t* Wd, const float* gd, int64_t d, int64_t f,
@@ -741,7 +831,7 @@ cudaError_t launch_ffn_down_fused(const uint8_t* Wd, const float* gd, int64_t d,
     StreamPlan p;
     cudaError_t e = plan_stream(a, d, f, M, 1, true, p);
     if (e != cudaSuccess) return e;
-    return launch_variant<1, SRC_H, false>(a, dim3(p.grid_x, 1), p.smem, s);
+    return launch_fused<SRC_H, false>(a, dim3(p.grid_x, 1), p.smem, s);
 }
 
 cudaError_t launch_gemv_generic(const uint8_t* Wp, const float* gamma, int64_t N, int64_t K,
