@@ -25,20 +25,26 @@ inline size_t align_up(size_t v) { return (v + kWsAlign - 1) / kWsAlign * kWsAli
 inline bool aligned(const void* p, size_t a) { return (uintptr_t)p % a == 0; }
 
 // Workspace carving -----------------------------------------------------------
+// Tensor-core projections (M > 16) may split tiles across CTAs (stream-K) and
+// need scratch for the pieces; the smaller paths do not.
+inline size_t sk_bytes(int64_t M) { return M > 16 ? align_up(bl::gemm_sk_workspace_bytes(bl::device_sm_count())) : 0; }
+
 struct ForwardWs {
-    size_t xq, scale, xsum, total;
+    size_t xq, scale, xsum, sk, sk_bytes, total;
 };
 inline ForwardWs forward_ws(int64_t M, int64_t K) {
     ForwardWs w;
     w.xq = 0;
     w.scale = align_up((size_t)(M * K));
     w.xsum = w.scale + align_up((size_t)M * 4);
-    w.total = w.xsum + align_up((size_t)M * 4);
+    w.sk = w.xsum + align_up((size_t)M * 4);
+    w.sk_bytes = sk_bytes(M);
+    w.total = w.sk + w.sk_bytes;
     return w;
 }
 
 struct FfnWs {
-    size_t xq, scale, xsum, g, u, q2, s2, xsum2, total;
+    size_t xq, scale, xsum, g, u, q2, s2, xsum2, sk, sk_bytes, total;
 };
 inline FfnWs ffn_ws(int64_t M, int64_t f, int64_t d) {
     FfnWs w;
@@ -50,7 +56,9 @@ inline FfnWs ffn_ws(int64_t M, int64_t f, int64_t d) {
     w.q2 = w.u + align_up((size_t)(M * f) * 4);
     w.s2 = w.q2 + align_up((size_t)(M * f));
     w.xsum2 = w.s2 + align_up((size_t)M * 4);
-    w.total = w.xsum2 + align_up((size_t)M * 4);
+    w.sk = w.xsum2 + align_up((size_t)M * 4);
+    w.sk_bytes = sk_bytes(M);
+    w.total = w.sk + w.sk_bytes;
     return w;
 }
 
@@ -114,10 +122,11 @@ inline int layout_of(Path p) {
 // One BitLinear projection of already-quantised codes `xq` (in layout_of(path)).
 bl_status project(Path path, const uint8_t* Wp, const float* gamma, int64_t N, int64_t K,
                   const int8_t* xq, const float* scale, const int32_t* xsum, int64_t M,
-                  const bl::GemvOut& out, cudaStream_t s) {
+                  const bl::GemvOut& out, cudaStream_t s, void* sk_ws, size_t sk_ws_bytes) {
     switch (path) {
         case Path::GemmTc:
-            return cuda_status(bl::launch_gemm_tc(Wp, gamma, N, K, xq, scale, xsum, M, out, s));
+            return cuda_status(
+                bl::launch_gemm_tc(Wp, gamma, N, K, xq, scale, xsum, M, out, s, sk_ws, sk_ws_bytes));
         case Path::GemvFast:
             return cuda_status(bl::launch_gemv(Wp, gamma, N, K, xq, scale, xsum, M, out, s));
         default:
@@ -210,7 +219,7 @@ BL_API bl_status bitlinear_forward(const uint8_t* Wp, const float* gamma, int64_
     if (path == Path::GemvFast && bl::gemv_fused_ok(M, K))  // one kernel: quantise + GEMV
         return cuda_status(bl::launch_gemv(Wp, gamma, N, K, nullptr, nullptr, nullptr, M, out, s, x));
     BL_TRY(bl::launch_act_quant(x, M, K, layout_of(path), xq, scale, xsum, s));
-    return project(path, Wp, gamma, N, K, xq, scale, xsum, M, out, s);
+    return project(path, Wp, gamma, N, K, xq, scale, xsum, M, out, s, base + w.sk, w.sk_bytes);
 }
 
 BL_API bl_status bitlinear_ffn(const uint8_t* Wg, const float* gg, const uint8_t* Wu,
@@ -266,14 +275,16 @@ BL_API bl_status bitlinear_ffn(const uint8_t* Wg, const float* gg, const uint8_t
         BL_TRY(bl::launch_gemv(Wu, gu, f, d, nullptr, nullptr, nullptr, M, ou, s, x));
     } else {
         BL_TRY(bl::launch_act_quant(x, M, d, layout_of(up), xq, scale, xsum, s));
-        if (bl_status st = project(up, Wg, gg, f, d, xq, scale, xsum, M, og, s)) return st;
-        if (bl_status st = project(up, Wu, gu, f, d, xq, scale, xsum, M, ou, s)) return st;
+        if (bl_status st = project(up, Wg, gg, f, d, xq, scale, xsum, M, og, s, base + w.sk, w.sk_bytes))
+            return st;
+        if (bl_status st = project(up, Wu, gu, f, d, xq, scale, xsum, M, ou, s, base + w.sk, w.sk_bytes))
+            return st;
     }
     BL_TRY(bl::launch_ffn_finalise(g, u, M, f, layout_of(down), q2, s2, xsum2, s));
     bl::GemvOut od;
     od.y = y;
     od.residual = residual;
-    return project(down, Wd, gd, d, f, q2, s2, xsum2, M, od, s);
+    return project(down, Wd, gd, d, f, q2, s2, xsum2, M, od, s, base + w.sk, w.sk_bytes);
 }
 
 BL_API bl_status bitlinear_validate_packed(const uint8_t* Wp, int64_t N, int64_t K,

@@ -17,6 +17,14 @@
 // transposed 4x4 byte block), which is exactly the order a packed word unpacks
 // into, so no byte shuffling is needed anywhere.
 //
+// Work split: data-parallel (each persistent CTA takes whole 128 x BN tiles) or,
+// when the tiles would leave part of the last wave idle, stream-K: the k-blocks
+// of all tiles, tile after tile, are cut into one contiguous range per CTA. A
+// CTA whose range covers a whole tile finishes it as usual; a piece of a tile is
+// written as raw int32 accumulators to a per-CTA slot of the workspace, and a
+// second kernel sums the pieces of each split tile (int32, so in any order the
+// same) and runs the same epilogue. No CTA ever waits for another.
+//
 // Every mbarrier wait is bounded (1 s); a wait that gives up sets the device
 // error word (reported as BL_ERR_TIMEOUT), lets the CTA drain and returns.
 #include <cuda.h>
@@ -71,6 +79,40 @@ __device__ __forceinline__ void report_timeout(unsigned* err, int* abort_flag) {
 __device__ __forceinline__ bool aborted(const int* abort_flag) {
     return *reinterpret_cast<const volatile int*>(abort_flag) != 0;
 }
+
+// The (tile, k-block range) pieces one CTA works on, in order. Data-parallel:
+// tiles c, c + G, ... whole. Stream-K: the units [U c / G, U (c + 1) / G) of the
+// U = tiles x nkb k-blocks, tile-major.
+template <bool SK>
+struct WorkIter {
+    int nkb, num_tiles, stride;
+    int u, ue;  // stream-K: next unit, end of the range
+    int tile;   // data-parallel: next tile
+    __device__ WorkIter(int nkb_, int num_tiles_, int G, int c)
+        : nkb(nkb_), num_tiles(num_tiles_), stride(G), u(0), ue(0), tile(c) {
+        if (SK) {
+            const long long U = (long long)num_tiles * nkb;
+            u = (int)(U * c / G);
+            ue = (int)(U * (c + 1) / G);
+        }
+    }
+    __device__ bool next(int& t, int& kb0, int& kb1) {
+        if (SK) {
+            if (u >= ue) return false;
+            t = u / nkb;
+            kb0 = u - t * nkb;
+            kb1 = min(nkb, kb0 + (ue - u));
+            u += kb1 - kb0;
+            return true;
+        }
+        if (tile >= num_tiles) return false;
+        t = tile;
+        kb0 = 0;
+        kb1 = nkb;
+        tile += stride;
+        return true;
+    }
+};
 
 // Dequantise and store 32 consecutive outputs of one row (one TMEM load).
 __device__ __forceinline__ void store_row_chunk(const uint32_t (&v)[32], int xs, float deq, int nb,
@@ -132,12 +174,12 @@ __device__ __forceinline__ void store_row_chunk(const uint32_t (&v)[32], int xs,
 
 // Persistent CTAs walk the (m-tile, n-tile) grid with n fastest, so the CTAs in
 // flight share activation tiles and the whole packed weight stays in L2.
-template <int BN>
+template <int BN, bool SK>
 __global__ void __launch_bounds__(THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    int M, int N, int K, const float* __restrict__ gamma_p,
                    const float* __restrict__ scale, const int32_t* __restrict__ xsum, GemvOut out,
-                   unsigned* err) {
+                   unsigned* err, uint32_t* __restrict__ partials) {
     constexpr int P_BYTES = TileCfg<BN>::P_BYTES;
     constexpr int U_BYTES = TileCfg<BN>::U_BYTES;
     constexpr int UNPACK_VEC = TileCfg<BN>::UNPACK_VEC;
@@ -196,9 +238,11 @@ __global__ void __launch_bounds__(THREADS, 1)
             tc::prefetch_tmap(&tmA);
             tc::prefetch_tmap(&tmB);
             uint32_t g = 0;
-            for (int tile = blockIdx.x; tile < num_tiles && !aborted(&abort_sh); tile += gridDim.x) {
+            WorkIter<SK> it(nkb, num_tiles, gridDim.x, blockIdx.x);
+            int tile, kb0, kb1;
+            while (!aborted(&abort_sh) && it.next(tile, kb0, kb1)) {
                 const int m0 = (tile / n_tiles) * BM, n0 = (tile % n_tiles) * BN;
-                for (int kb = 0; kb < nkb; ++kb, ++g) {
+                for (int kb = kb0; kb < kb1; ++kb, ++g) {
                     const int s = g % TSTAGES;
                     if (g >= TSTAGES &&
                         !tc::mbar_wait(tempty(s), ((g / TSTAGES) - 1) & 1, WAIT_LIMIT_NS)) {
@@ -222,8 +266,9 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (lane == 0) {
             constexpr uint32_t idesc = tc::idesc_i8_s8u8(BM, BN);
             uint32_t g = 0, t = 0;
-            for (int tile = blockIdx.x; tile < num_tiles && !aborted(&abort_sh);
-                 tile += gridDim.x, ++t) {
+            WorkIter<SK> it(nkb, num_tiles, gridDim.x, blockIdx.x);
+            int tile, kb0, kb1;
+            for (; !aborted(&abort_sh) && it.next(tile, kb0, kb1); ++t) {
                 const int a = t & 1;
                 if (t >= 2 && !tc::mbar_wait(aempty(a), ((t >> 1) - 1) & 1, WAIT_LIMIT_NS)) {
                     report_timeout(err, &abort_sh);
@@ -232,7 +277,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                 tc::fence_after_sync();
                 const uint32_t d = tmem + a * BN;
                 bool ok = true;
-                for (int kb = 0; kb < nkb; ++kb, ++g) {
+                for (int kb = kb0; kb < kb1; ++kb, ++g) {
                     const int s = g % TSTAGES, u = g % USTAGES;
                     if (!tc::mbar_wait(ufull(u), (g / USTAGES) & 1, WAIT_LIMIT_NS) ||
                         !tc::mbar_wait(tfull(s), (g / TSTAGES) & 1, WAIT_LIMIT_NS)) {
@@ -245,7 +290,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                     const uint64_t bd = tc::desc_kmajor_sw128(tc::smem_u32(sU + u * U_BYTES));
 #pragma unroll
                     for (int kk = 0; kk < BK / 32; ++kk)  // 32 bytes of K per MMA: +2 in 16-byte units
-                        tc::mma_i8(d, ad + 2 * kk, bd + 2 * kk, idesc, (kb | kk) != 0);
+                        tc::mma_i8(d, ad + 2 * kk, bd + 2 * kk, idesc, kb != kb0 || kk != 0);
                     tc::mma_commit(tempty(s));
                     tc::mma_commit(uempty(u));
                 }
@@ -257,9 +302,11 @@ __global__ void __launch_bounds__(THREADS, 1)
         // ------------------------------------------------------------ unpack
         const int ut = threadIdx.x - 64;
         uint32_t g = 0;
-        for (int tile = blockIdx.x; tile < num_tiles && !aborted(&abort_sh); tile += gridDim.x) {
+        WorkIter<SK> it(nkb, num_tiles, gridDim.x, blockIdx.x);
+        int tile, kb0, kb1;
+        while (!aborted(&abort_sh) && it.next(tile, kb0, kb1)) {
             bool ok = true;
-            for (int kb = 0; kb < nkb; ++kb, ++g) {
+            for (int kb = kb0; kb < kb1; ++kb, ++g) {
                 const int s = g % TSTAGES, u = g % USTAGES;
                 if (!tc::mbar_wait(tfull(s), (g / TSTAGES) & 1, WAIT_LIMIT_NS) ||
                     (g >= USTAGES &&
@@ -307,7 +354,9 @@ __global__ void __launch_bounds__(THREADS, 1)
         const bool vec = (N % 8 == 0) && aligned16(out.y) && aligned16(out.y32) &&
                          aligned16(out.residual) && aligned16(out.acc);
         uint32_t t = 0;
-        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++t) {
+        WorkIter<SK> it(nkb, num_tiles, gridDim.x, blockIdx.x);
+        int tile, kb0, kb1;
+        for (; it.next(tile, kb0, kb1); ++t) {
             const int a = t & 1;
             bool ok = !aborted(&abort_sh) && tc::mbar_wait(afull(a), (t >> 1) & 1, WAIT_LIMIT_NS);
             if (!__all_sync(0xffffffffu, ok)) {  // tcgen05.ld below is warp-collective
@@ -318,15 +367,26 @@ __global__ void __launch_bounds__(THREADS, 1)
             const int m0 = (tile / n_tiles) * BM, n0 = (tile % n_tiles) * BN;
             const int m = m0 + q * 32 + lane;
             const bool mv = m < M;
-            const float deq = mv ? __fdiv_rn(gamma, scale[m]) : 0.0f;
-            const int xs = mv ? xsum[m] : 0;
+            const bool whole = !SK || (kb0 == 0 && kb1 == nkb);
+            // a piece of a split tile goes to slot 2c (the CTA's first piece) or 2c + 1,
+            // column-major, so that the 32 rows of a warp store one 128-byte line
+            uint32_t* slot = whole ? nullptr
+                                   : partials + (size_t)(2 * blockIdx.x + (t == 0 ? 0 : 1)) * BM * BN +
+                                         (q * 32 + lane);
+            const float deq = mv && whole ? __fdiv_rn(gamma, scale[m]) : 0.0f;
+            const int xs = mv && whole ? xsum[m] : 0;
 #pragma unroll 1
             for (int c = 0; c < BN / 32; ++c) {
                 uint32_t v[32];
                 tc::tmem_ld_32x32(tmem + (static_cast<uint32_t>(q * 32) << 16) + a * BN + c * 32, v);
                 tc::tmem_ld_wait();
                 const int nb = n0 + c * 32;
-                if (mv && nb < N) store_row_chunk(v, xs, deq, nb, N, static_cast<size_t>(m) * N + nb, out, vec);
+                if (SK && !whole) {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) slot[(size_t)(c * 32 + j) * BM] = v[j];
+                } else if (mv && nb < N) {
+                    store_row_chunk(v, xs, deq, nb, N, static_cast<size_t>(m) * N + nb, out, vec);
+                }
             }
             tc::fence_before_sync();
             tc::mbar_arrive(aempty(a));
@@ -346,6 +406,99 @@ __global__ void __launch_bounds__(THREADS, 1)
         tc::fence_after_sync();
         tc::tmem_dealloc(tmem, TMEM_COLS);
     }
+}
+
+// Dequantise and store 8 consecutive outputs of one row (stream-K fix-up).
+__device__ __forceinline__ void store_row8(const uint32_t (&v)[8], int xs, float deq, int nb, int N, size_t o,
+                                           const GemvOut& out, bool vec) {
+    int a[8];
+    float f[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        a[j] = static_cast<int>(v[j]) - xs;
+        f[j] = dequant(a[j], deq);
+    }
+    if (vec && nb + 8 <= N) {
+        if (out.y32) {
+            *reinterpret_cast<float4*>(out.y32 + o) = make_float4(f[0], f[1], f[2], f[3]);
+            *reinterpret_cast<float4*>(out.y32 + o + 4) = make_float4(f[4], f[5], f[6], f[7]);
+        } else {
+            uint4 r = make_uint4(0, 0, 0, 0);
+            if (out.residual) r = *reinterpret_cast<const uint4*>(out.residual + o);
+            const uint32_t rr[4] = {r.x, r.y, r.z, r.w};
+            uint32_t pk[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                float lo = f[2 * e], hi = f[2 * e + 1];
+                if (out.residual) {
+                    lo = __fadd_rn(bf16_bits_to_f32(rr[e] & 0xffffu), lo);
+                    hi = __fadd_rn(bf16_bits_to_f32(rr[e] >> 16), hi);
+                }
+                pk[e] = f32_to_bf16_bits(lo) | (static_cast<uint32_t>(f32_to_bf16_bits(hi)) << 16);
+            }
+            *reinterpret_cast<uint4*>(out.y + o) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        }
+        if (out.acc) {
+            *reinterpret_cast<int4*>(out.acc + o) = make_int4(a[0], a[1], a[2], a[3]);
+            *reinterpret_cast<int4*>(out.acc + o + 4) = make_int4(a[4], a[5], a[6], a[7]);
+        }
+        return;
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        if (nb + j >= N) break;
+        float v2 = f[j];
+        if (out.y32) {
+            out.y32[o + j] = v2;
+        } else {
+            if (out.residual) v2 = __fadd_rn(bf16_bits_to_f32(out.residual[o + j]), v2);
+            out.y[o + j] = f32_to_bf16_bits(v2);
+        }
+        if (out.acc) out.acc[o + j] = a[j];
+    }
+}
+
+// Stream-K fix-up: CTA (tile, 32-column chunk); a tile that one CTA finished
+// returns at once, a split tile sums its pieces (slots of the CTAs whose ranges
+// cover it) and runs the epilogue. Thread (quarter qd = tid / 128, row r = tid %
+// 128) owns 8 columns of one row; the pieces are column-major, so each warp load
+// reads one 128-byte line, and every piece's loads are in flight together.
+template <int BN>
+__global__ void __launch_bounds__(512) gemm_sk_fixup_kernel(int M, int N, int K, int G,
+                                                           const uint32_t* __restrict__ partials,
+                                                           const float* __restrict__ gamma_p,
+                                                           const float* __restrict__ scale,
+                                                           const int32_t* __restrict__ xsum, GemvOut out) {
+    grid_dependency_wait();
+    const int n_tiles = (N + BN - 1) / BN;
+    const int nkb = (K + BK - 1) / BK;
+    const long long U = (long long)n_tiles * ((M + BM - 1) / BM) * nkb;
+    const int tile = blockIdx.x;
+    const long long t0 = (long long)tile * nkb, t1 = t0 + nkb;  // units of this tile
+    // the CTA whose range [U c / G, U (c + 1) / G) holds unit u
+    auto owner = [&](long long u) { return (int)(((u + 1) * G + U - 1) / U) - 1; };
+    const int c_first = owner(t0), c_last = owner(t1 - 1);
+    if (c_first == c_last) return;
+    const int m0 = (tile / n_tiles) * BM, n0 = (tile % n_tiles) * BN;
+    const int r = threadIdx.x & (BM - 1), qd = threadIdx.x / BM;
+    const int m = m0 + r;
+    const int col = blockIdx.y * 32 + qd * 8;  // first column of this thread inside the tile
+    if (m >= M || n0 + col >= N) return;
+    uint32_t v[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) v[j] = 0;
+#pragma unroll 2
+    for (int cta = c_first; cta <= c_last; ++cta) {
+        const bool first_piece = (long long)(U * cta / G) >= t0;  // the range starts inside this tile
+        const uint32_t* src =
+            partials + (size_t)(2 * cta + (first_piece ? 0 : 1)) * BM * BN + (size_t)col * BM + r;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) v[j] += src[(size_t)j * BM];
+    }
+    const bool vec = (N % 8 == 0) && aligned16(out.y) && aligned16(out.y32) && aligned16(out.residual) &&
+                     aligned16(out.acc);
+    store_row8(v, xsum[m], __fdiv_rn(*gamma_p, scale[m]), n0 + col, N, static_cast<size_t>(m) * N + n0 + col,
+               out, vec);
 }
 
 // ---------------------------------------------------------------- host side
@@ -395,7 +548,7 @@ namespace {
 template <int BN>
 cudaError_t launch_bn(const uint8_t* Wp, const float* gamma, int64_t N, int64_t K, const int8_t* xq_g16t,
                       const float* scale, const int32_t* xsum, int64_t M, const GemvOut& out,
-                      cudaStream_t s, int dev, int sms) {
+                      cudaStream_t s, int dev, int sms, uint32_t* partials) {
     constexpr size_t smem = TileCfg<BN>::SMEM_BYTES;
     CUtensorMap mapA, mapB;
     if (!make_map(&mapA, xq_g16t, (uint64_t)M, (uint64_t)K, BM, BK, true) ||
@@ -404,17 +557,23 @@ cudaError_t launch_bn(const uint8_t* Wp, const float* gamma, int64_t N, int64_t 
     unsigned* err = nullptr;
     cudaError_t e = device_error_word(&err);
     if (e != cudaSuccess) return e;
-    static bool attr_set[64];
-    if (dev >= 64 || !attr_set[dev]) {
-        e = cudaFuncSetAttribute(gemm_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    const bool sk = partials != nullptr;
+    auto kern = sk ? gemm_tc_kernel<BN, true> : gemm_tc_kernel<BN, false>;
+    static bool attr_set[64][2];
+    if (dev >= 64 || !attr_set[dev][sk]) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        if (dev < 64) attr_set[dev] = true;
+        if (dev < 64) attr_set[dev][sk] = true;
     }
     const int64_t tiles = ((N + BN - 1) / BN) * ((M + BM - 1) / BM);
-    const unsigned grid = (unsigned)(tiles < sms ? tiles : sms);
-    gemm_tc_kernel<BN><<<grid, THREADS, smem, s>>>(mapA, mapB, (int)M, (int)N, (int)K, gamma, scale, xsum,
-                                                   out, err);
-    return cudaGetLastError();
+    const int64_t units = tiles * ((K + BK - 1) / BK);
+    const int64_t work = sk ? units : tiles;
+    const unsigned grid = (unsigned)(work < sms ? work : sms);
+    kern<<<grid, THREADS, smem, s>>>(mapA, mapB, (int)M, (int)N, (int)K, gamma, scale, xsum, out, err, partials);
+    e = cudaGetLastError();
+    if (e != cudaSuccess || !sk) return e;
+    return launch_pdl(gemm_sk_fixup_kernel<BN>, dim3((unsigned)tiles, BN / 32), dim3(512), 0, s, (int)M, (int)N,
+                      (int)K, (int)grid, (const uint32_t*)partials, gamma, scale, xsum, out);
 }
 }  // namespace
 
@@ -439,9 +598,35 @@ int gemm_tc_tile_width(int64_t M, int64_t N, int sms) {
     return best;
 }
 
+size_t gemm_sk_workspace_bytes(int sms) { return (size_t)2 * sms * BM * 256 * sizeof(uint32_t); }
+
+int device_sm_count() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+        cudaGetLastError();
+        return 148;
+    }
+    return n;
+}
+
+// Stream-K only where the data-parallel plan leaves much of its last wave idle
+// (under 70% of its CTA-slots busy) and the tiles are long in K (at least 32
+// k-blocks), so the pieces are large: each split tile costs a 128 KB write and
+// read of int32 pieces plus the fix-up launch, which ate the gain on the other
+// shapes measured (2560 -> 6912 at M = 512, 6912 -> 2560 at M = 4096).
+bool gemm_use_stream_k(int64_t M, int64_t N, int64_t K, int sms) {
+    const int64_t mt = (M + BM - 1) / BM;
+    const int bn = gemm_tc_tile_width(M, N, sms);
+    const int64_t dp_tiles = mt * ((N + bn - 1) / bn);
+    const int64_t waves = (dp_tiles + sms - 1) / sms;
+    const double busy = (double)dp_tiles / (double)(waves * sms);
+    return busy < 0.7 && (K + BK - 1) / BK >= 32;
+}
+
 cudaError_t launch_gemm_tc(const uint8_t* Wp, const float* gamma, int64_t N, int64_t K,
                            const int8_t* xq_g16t, const float* scale, const int32_t* xsum, int64_t M,
-                           const GemvOut& out, cudaStream_t s) {
+                           const GemvOut& out, cudaStream_t s, void* sk_ws, size_t sk_ws_bytes) {
     if (M == 0 || N == 0) return cudaSuccess;
     int dev = 0;
     cudaGetDevice(&dev);
@@ -451,10 +636,13 @@ cudaError_t launch_gemm_tc(const uint8_t* Wp, const float* gamma, int64_t N, int
         if (e != cudaSuccess) return e;
     }
     const int sms = dev < 64 ? num_sms[dev] : 148;
+    if (sk_ws && sk_ws_bytes >= gemm_sk_workspace_bytes(sms) && gemm_use_stream_k(M, N, K, sms))
+        return launch_bn<256>(Wp, gamma, N, K, xq_g16t, scale, xsum, M, out, s, dev, sms,
+                              static_cast<uint32_t*>(sk_ws));
     switch (gemm_tc_tile_width(M, N, sms)) {
-        case 64: return launch_bn<64>(Wp, gamma, N, K, xq_g16t, scale, xsum, M, out, s, dev, sms);
-        case 128: return launch_bn<128>(Wp, gamma, N, K, xq_g16t, scale, xsum, M, out, s, dev, sms);
-        default: return launch_bn<256>(Wp, gamma, N, K, xq_g16t, scale, xsum, M, out, s, dev, sms);
+        case 64: return launch_bn<64>(Wp, gamma, N, K, xq_g16t, scale, xsum, M, out, s, dev, sms, nullptr);
+        case 128: return launch_bn<128>(Wp, gamma, N, K, xq_g16t, scale, xsum, M, out, s, dev, sms, nullptr);
+        default: return launch_bn<256>(Wp, gamma, N, K, xq_g16t, scale, xsum, M, out, s, dev, sms, nullptr);
     }
 }
 

@@ -58,9 +58,13 @@ cudaError_t launch_gemv_generic(const uint8_t* Wp, const float* gamma, int64_t N
 // aligned Wp and xq_g16t (TMA); any M, N (tails are zero-filled by the TMA).
 bool gemm_tc_ok(int64_t N, int64_t K, const void* Wp, const void* xq);
 int gemm_tc_tile_width(int64_t M, int64_t N, int sms);
+// sk_ws / sk_ws_bytes: scratch for stream-K pieces (gemm_sk_workspace_bytes of the
+// device's SM count); null or too small means the data-parallel split only.
 cudaError_t launch_gemm_tc(const uint8_t* Wp, const float* gamma, int64_t N, int64_t K,
                            const int8_t* xq_g16t, const float* scale, const int32_t* xsum, int64_t M,
-                           const GemvOut& out, cudaStream_t s);
+                           const GemvOut& out, cudaStream_t s, void* sk_ws = nullptr, size_t sk_ws_bytes = 0);
+size_t gemm_sk_workspace_bytes(int sms);
+int device_sm_count();  // SMs of the current device (148 when it cannot be read)
 
 // ---- FFN glue (ffn.cu)
 // h = relu(g)^2 * u; hn = subln(h); q2, s2, xsum2 = quant(hn) in `layout`.

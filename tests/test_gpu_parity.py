@@ -169,6 +169,19 @@ def test_forward_tensor_core_tails(cuda_device, M, N, K):
     check_forward_full(Wp, gamma, Wp_ref, g_ref, x, cuda_device, residual=res)
 
 
+@pytest.mark.parametrize("M,N,K", [(200, 600, 4096), (300, 2560, 4160)])
+def test_forward_stream_k_split_tiles(cuda_device, M, N, K):
+    """Few tiles and at least 32 k-blocks: the GEMM splits tiles across CTAs
+    (stream-K) and a second kernel sums the int32 pieces. Ragged tokens, rows and
+    last k-block; with and without the residual."""
+    W = make_weights(N, K, 0.02, seed=M + N + 7 * K)
+    Wp, gamma, Wp_ref, g_ref = pack_both(W, cuda_device)
+    x = synth.activations(M, K, seed=M + 1, outliers=True)
+    res = synth.activations(M, N, seed=N + 1, outliers=False)
+    check_forward_full(Wp, gamma, Wp_ref, g_ref, x, cuda_device)
+    check_forward_full(Wp, gamma, Wp_ref, g_ref, x, cuda_device, residual=res)
+
+
 def test_forward_misaligned_input_takes_generic_path(cuda_device):
     K, N, M = 256, 64, 20
     W = make_weights(N, K, 0.02, seed=21)
@@ -294,6 +307,19 @@ def test_ffn_small_batches(cuda_device, M):
         assert_bf16_close(bits(y_dev), ref["y"], f"M={M} layer {layer}")
         assert_bf16_exact(bits(y_dev), ref["y"], f"M={M} layer {layer}")
         h_dev = y_dev
+
+
+def test_ffn_stream_k_fp32_projections(cuda_device):
+    """M = 40 at d = 4096, f = 1024: gate and up run on the tensor cores with
+    split tiles and fp32 outputs (the fix-up's fp32 store), down unsplit."""
+    d, f, M = 4096, 1024, 40
+    Wg, Wu, Wd = (make_weights(f, d, 0.02, 41), make_weights(f, d, 0.02, 42), make_weights(d, f, 0.02, 43))
+    P = [pack_both(W, cuda_device) for W in (Wg, Wu, Wd)]
+    x = synth.activations(M, d, seed=44, outliers=True)
+    y = bl.ffn(P[0][0], P[0][1], P[1][0], P[1][1], P[2][0], P[2][1], x.to(cuda_device), residual=x.to(cuda_device))
+    ref = oracle.ffn_layer(P[0][2], P[0][3], P[1][2], P[1][3], P[2][2], P[2][3], bits(x), residual=bits(x))
+    assert_bf16_close(bits(y), ref["y"])
+    assert_bf16_exact(bits(y), ref["y"])
 
 
 def test_ffn_small_ragged(cuda_device):
