@@ -130,9 +130,12 @@ bl_status bitlinear_quant_act(const uint16_t* x, int64_t M, int64_t K,
  *   acc       [M, N] device int32 output of the exact accumulator; may be NULL
  *   ws        device workspace of bitlinear_workspace_bytes(BL_OP_FORWARD, M, N, K) bytes
  * Kernel choice: M <= 16 streams the packed weights once through a
- * bandwidth-bound GEMV (K % 256 == 0, Wp and x 16-byte aligned); larger M runs
- * the tensor-core GEMM (K % 64 == 0, same alignment, any N); other shapes take a
- * generic kernel. Every path gives the same bits.
+ * bandwidth-bound GEMV (K % 256 == 0, Wp and x 16-byte aligned), quantising x
+ * inside the same kernel for M <= 4 when the codes of all M tokens fit in 48 KiB
+ * (M * (K + 64) bytes); larger M runs the tensor-core GEMM (K % 64 == 0, same
+ * alignment, any N), which for M > 16 also uses the workspace for split-tile
+ * partial sums; other shapes take a generic kernel. Every path gives the same
+ * bits.
  */
 bl_status bitlinear_forward(const uint8_t* Wp, const float* gamma, int64_t N, int64_t K,
                             const uint16_t* x, int64_t M, const uint16_t* residual,
