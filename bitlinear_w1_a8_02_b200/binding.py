@@ -36,6 +36,8 @@ SIGNATURES = {
     "bitlinear_pack_weights": (_ST, [_P, ctypes.c_int, _I, _I, _P, _P, _P, _S, _P]),
     "bitlinear_quant_act": (_ST, [_P, _I, _I, _P, _P, _P, _P]),
     "bitlinear_forward": (_ST, [_P, _P, _I, _I, _P, _I, _P, _P, _P, _P, _S, _P]),
+    "bitlinear_forward_ex": (_ST, [_P, _P, _P, ctypes.c_int32, _I, _P, _I, ctypes.c_int32, _P, _P, _P, _P, _S,
+                                   _P]),
     "bitlinear_ffn": (_ST, [_P, _P, _P, _P, _P, _P, _I, _I, _P, _I, _P, _P, _P, _S, _P]),
     "bitlinear_forward_noalloc": (_ST, [_P, _P, _I, _I, _P, _I, _P, _P, _P, _P]),
     "bitlinear_validate_packed": (_ST, [_P, _I, _I, _P, _P, _S, _P]),
@@ -167,6 +169,34 @@ def forward(Wp: torch.Tensor, gamma: torch.Tensor, x: torch.Tensor,
     st = lib().bitlinear_forward(_ptr(Wp), _ptr(gamma), N, K, _ptr(x), M, _ptr(residual), _ptr(y),
                                  _ptr(acc), _ptr(ws), ws.numel(), _stream(x.device))
     _check(st, "bitlinear_forward")
+    return (y, acc) if want_acc else y
+
+
+def forward_ex(Wp: torch.Tensor, gammas: torch.Tensor, seg_rows, x: torch.Tensor, rmsnorm: bool = False,
+               residual: Optional[torch.Tensor] = None, want_acc: bool = False,
+               out: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None):
+    """Projections of x against row-stacked packed weights (segment i has
+    seg_rows[i] rows and gamma gammas[i]), optionally after a unit-weight RMSNorm
+    of x: bf16 [M, sum(seg_rows)] (and the int32 accumulator with want_acc)."""
+    _cuda(Wp, "Wp", torch.uint8)
+    _cuda(x, "x", torch.bfloat16)
+    _cuda(gammas, "gammas", torch.float32)
+    N, KB = Wp.shape
+    M, K = x.shape
+    rows = (ctypes.c_int64 * len(seg_rows))(*[int(r) for r in seg_rows])
+    if sum(int(r) for r in seg_rows) != N:
+        raise ValueError(f"segments cover {sum(seg_rows)} rows, packed weights have {N}")
+    if K != 4 * KB:
+        raise ValueError(f"x has K={K}, packed weights have K={4 * KB}")
+    if residual is not None:
+        _cuda(residual, "residual", torch.bfloat16)
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device) if out is None else out
+    acc = torch.empty((M, N), dtype=torch.int32, device=x.device) if want_acc else None
+    need = workspace_bytes(BL_OP_FORWARD, M, N, K)
+    ws = _WS.get(x.device, need) if ws is None else ws
+    st = lib().bitlinear_forward_ex(_ptr(Wp), _ptr(gammas), rows, len(seg_rows), K, _ptr(x), M, int(bool(rmsnorm)),
+                                    _ptr(residual), _ptr(y), _ptr(acc), _ptr(ws), ws.numel(), _stream(x.device))
+    _check(st, "bitlinear_forward_ex")
     return (y, acc) if want_acc else y
 
 

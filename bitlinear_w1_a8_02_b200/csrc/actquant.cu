@@ -10,6 +10,14 @@
 // One CTA per token. Pass 1 reduces the absmax (order-free, so exact); pass 2
 // re-reads the row (an L1/L2 hit) and writes 16 codes per thread in the layout
 // the consumer wants (see XqLayout).
+//
+// Optional unit-weight RMSNorm in front (the transformer block's pre-norm and
+// the subln before the attention output projection; paper card "Method
+// Adaptation": subln): pass 1 also sums x^2 in fp64 (the squares of bf16 values
+// are exact in fp64 and so, for any realistic range, is their sum, whatever the
+// order), r = 1 / sqrtf(float(sum / K) + 1e-5), and the codes are those of
+// fl(x * r) with s = 127 / max(fl(max |x| * r), 1e-5) (rounding is monotonic,
+// so max |fl(x r)| = fl(max |x| r)).
 #include "common.cuh"
 #include "kernels.h"
 
@@ -43,13 +51,29 @@ __device__ __forceinline__ void unpack8(uint4 v, float* f) {
 }
 
 // Vector path: K % 16 == 0, x and xq 16-byte aligned.
+__device__ __forceinline__ double sumsq8(uint4 v) {
+    float f[8];
+    unpack8(v, f);
+    double ss = 0.0;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) ss = __fma_rn((double)f[e], (double)f[e], ss);
+    return ss;
+}
+
+// r of the optional RMSNorm from the row's sum of squares (in fp64).
+__device__ __forceinline__ float rms_factor(double ss, int K) {
+    const float ms = __double2float_rn(__ddiv_rn(ss, (double)K));
+    return __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, kRmsEps)));
+}
+
 template <int LAYOUT>
 __global__ void __launch_bounds__(kThreads) act_quant_vec_kernel(const uint16_t* __restrict__ x,
                                                                   int K, int8_t* __restrict__ xq,
                                                                   float* __restrict__ scale,
-                                                                  int32_t* __restrict__ xsum) {
+                                                                  int32_t* __restrict__ xsum, int norm) {
     __shared__ float fscratch[kWarps];
     __shared__ int iscratch[kWarps];
+    __shared__ double dscratch[kWarps];
     grid_dependency_wait();
     grid_dependents_launch();
     const int m = blockIdx.x;
@@ -57,8 +81,18 @@ __global__ void __launch_bounds__(kThreads) act_quant_vec_kernel(const uint16_t*
     const int nvec = K / 8;
 
     float amax = 0.0f;
-    for (int i = threadIdx.x; i < nvec; i += kThreads) amax = fmaxf(amax, absmax8(xr[i]));
+    double ss = 0.0;
+    for (int i = threadIdx.x; i < nvec; i += kThreads) {
+        const uint4 v = xr[i];
+        amax = fmaxf(amax, absmax8(v));
+        if (norm) ss += sumsq8(v);
+    }
     amax = block_max<kWarps>(amax, fscratch);
+    float r = 1.0f;
+    if (norm) {
+        r = rms_factor(block_sum<kWarps>(ss, dscratch), K);
+        amax = __fmul_rn(amax, r);
+    }
     const float s = __fdiv_rn(kActRange, fmaxf(amax, kActEps));
 
     const int KB = K / 4;
@@ -67,6 +101,10 @@ __global__ void __launch_bounds__(kThreads) act_quant_vec_kernel(const uint16_t*
         float f[16];
         unpack8(xr[2 * c], f);
         unpack8(xr[2 * c + 1], f + 8);
+        if (norm) {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) f[e] = __fmul_rn(f[e], r);
+        }
         int q[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
@@ -107,20 +145,32 @@ __global__ void __launch_bounds__(kThreads) act_quant_vec_kernel(const uint16_t*
 __global__ void __launch_bounds__(kThreads) act_quant_scalar_kernel(const uint16_t* __restrict__ x,
                                                                      int K, int8_t* __restrict__ xq,
                                                                      float* __restrict__ scale,
-                                                                     int32_t* __restrict__ xsum) {
+                                                                     int32_t* __restrict__ xsum, int norm) {
     __shared__ float fscratch[kWarps];
     __shared__ int iscratch[kWarps];
+    __shared__ double dscratch[kWarps];
     grid_dependency_wait();
     grid_dependents_launch();
     const int m = blockIdx.x;
     const uint16_t* xr = x + (size_t)m * K;
     float amax = 0.0f;
-    for (int k = threadIdx.x; k < K; k += kThreads) amax = fmaxf(amax, fabsf(bf16_bits_to_f32(xr[k])));
+    double ss = 0.0;
+    for (int k = threadIdx.x; k < K; k += kThreads) {
+        const float f = bf16_bits_to_f32(xr[k]);
+        amax = fmaxf(amax, fabsf(f));
+        if (norm) ss = __fma_rn((double)f, (double)f, ss);
+    }
     amax = block_max<kWarps>(amax, fscratch);
+    float r = 1.0f;
+    if (norm) {
+        r = rms_factor(block_sum<kWarps>(ss, dscratch), K);
+        amax = __fmul_rn(amax, r);
+    }
     const float s = __fdiv_rn(kActRange, fmaxf(amax, kActEps));
     int sum = 0;
     for (int k = threadIdx.x; k < K; k += kThreads) {
-        const int q = quant_code(bf16_bits_to_f32(xr[k]), s);
+        const float f = bf16_bits_to_f32(xr[k]);
+        const int q = quant_code(norm ? __fmul_rn(f, r) : f, s);
         xq[(size_t)m * K + k] = (int8_t)q;
         sum += q;
     }
@@ -134,22 +184,23 @@ __global__ void __launch_bounds__(kThreads) act_quant_scalar_kernel(const uint16
 }  // namespace
 
 cudaError_t launch_act_quant(const uint16_t* x, int64_t M, int64_t K, int layout, int8_t* xq,
-                             float* scale, int32_t* xsum, cudaStream_t s) {
+                             float* scale, int32_t* xsum, cudaStream_t s, bool rmsnorm) {
+    const int norm = rmsnorm ? 1 : 0;
     if (M == 0) return cudaSuccess;
     const bool vec = (K % 16 == 0) && ((uintptr_t)x % 16 == 0) && ((uintptr_t)xq % 16 == 0);
     if (!vec) {
         if (layout != XQ_NATURAL) return cudaErrorInvalidValue;
         return launch_pdl(act_quant_scalar_kernel, dim3((unsigned)M), dim3(kThreads), 0, s, x, (int)K,
-                          xq, scale, xsum);
+                          xq, scale, xsum, norm);
     }
     if (layout == XQ_NATURAL)
         return launch_pdl(act_quant_vec_kernel<XQ_NATURAL>, dim3((unsigned)M), dim3(kThreads), 0, s, x,
-                          (int)K, xq, scale, xsum);
+                          (int)K, xq, scale, xsum, norm);
     if (layout == XQ_PLANES)
         return launch_pdl(act_quant_vec_kernel<XQ_PLANES>, dim3((unsigned)M), dim3(kThreads), 0, s, x,
-                          (int)K, xq, scale, xsum);
+                          (int)K, xq, scale, xsum, norm);
     return launch_pdl(act_quant_vec_kernel<XQ_G16T>, dim3((unsigned)M), dim3(kThreads), 0, s, x, (int)K,
-                      xq, scale, xsum);
+                      xq, scale, xsum, norm);
 }
 
 }  // namespace bl

@@ -191,35 +191,80 @@ BL_API bl_status bitlinear_quant_act(const uint16_t* x, int64_t M, int64_t K, in
         bl::launch_act_quant(x, M, K, bl::XQ_NATURAL, xq, scale, xsum, (cudaStream_t)stream));
 }
 
-BL_API bl_status bitlinear_forward(const uint8_t* Wp, const float* gamma, int64_t N, int64_t K,
-                                   const uint16_t* x, int64_t M, const uint16_t* residual,
-                                   uint16_t* y, int32_t* acc, void* ws, size_t ws_bytes,
-                                   bl_stream_t stream) {
-    if (M < 0 || M > kMaxM || N < 0 || N > kMaxN || K < 4 || K % 4 != 0 || K > kMaxK)
-        return BL_ERR_SHAPE;
-    if (M == 0 || N == 0) return BL_OK;
-    if (!Wp || !gamma || !x || !y) return BL_ERR_NULL;
-    if (!aligned(gamma, 4) || !aligned(x, 2) || !aligned(y, 2) || (residual && !aligned(residual, 2)) ||
-        (acc && !aligned(acc, 4)))
-        return BL_ERR_ALIGN;
+namespace {
+
+// The forward behind bitlinear_forward and bitlinear_forward_ex: `out` carries
+// the row segments (gamma holds one value per segment), `rmsnorm` quantises the
+// unit-weight RMSNorm of x instead of x.
+bl_status forward_impl(const uint8_t* Wp, const float* gamma, int64_t N, int64_t K, const uint16_t* x,
+                       int64_t M, bool rmsnorm, bl::GemvOut out, void* ws, size_t ws_bytes,
+                       cudaStream_t s) {
     const ForwardWs w = forward_ws(M, K);
     if (bl_status st = check_ws(ws, ws_bytes, w.total)) return st;
     if (bl_status st = check_device()) return st;
-    cudaStream_t s = (cudaStream_t)stream;
     char* base = (char*)ws;
     int8_t* xq = (int8_t*)(base + w.xq);
     float* scale = (float*)(base + w.scale);
     int32_t* xsum = (int32_t*)(base + w.xsum);
 
-    const Path path = choose_path(Wp, N, K, M, xq, x);
+    Path path = choose_path(Wp, N, K, M, xq, x);
+    // segment ends that do not fall on the fast paths' tiles take the generic kernel
+    if ((path == Path::GemmTc && !bl::gemm_segments_ok(out, N)) ||
+        (path == Path::GemvFast && !bl::gemv_segments_ok(out, N)))
+        path = Path::GemvGeneric;
+    if (path == Path::GemvFast && bl::gemv_fused_ok(M, K))  // one kernel: quantise + GEMV
+        return cuda_status(bl::launch_gemv(Wp, gamma, N, K, nullptr, nullptr, nullptr, M, out, s, x, rmsnorm));
+    BL_TRY(bl::launch_act_quant(x, M, K, layout_of(path), xq, scale, xsum, s, rmsnorm));
+    return project(path, Wp, gamma, N, K, xq, scale, xsum, M, out, s, base + w.sk, w.sk_bytes);
+}
+
+bool forward_args_ok(int64_t N, int64_t K, int64_t M) {
+    return M >= 0 && M <= kMaxM && N >= 0 && N <= kMaxN && K >= 4 && K % 4 == 0 && K <= kMaxK;
+}
+
+}  // namespace
+
+BL_API bl_status bitlinear_forward(const uint8_t* Wp, const float* gamma, int64_t N, int64_t K,
+                                   const uint16_t* x, int64_t M, const uint16_t* residual,
+                                   uint16_t* y, int32_t* acc, void* ws, size_t ws_bytes,
+                                   bl_stream_t stream) {
+    if (!forward_args_ok(N, K, M)) return BL_ERR_SHAPE;
+    if (M == 0 || N == 0) return BL_OK;
+    if (!Wp || !gamma || !x || !y) return BL_ERR_NULL;
+    if (!aligned(gamma, 4) || !aligned(x, 2) || !aligned(y, 2) || (residual && !aligned(residual, 2)) ||
+        (acc && !aligned(acc, 4)))
+        return BL_ERR_ALIGN;
     bl::GemvOut out;
     out.y = y;
     out.residual = residual;
     out.acc = acc;
-    if (path == Path::GemvFast && bl::gemv_fused_ok(M, K))  // one kernel: quantise + GEMV
-        return cuda_status(bl::launch_gemv(Wp, gamma, N, K, nullptr, nullptr, nullptr, M, out, s, x));
-    BL_TRY(bl::launch_act_quant(x, M, K, layout_of(path), xq, scale, xsum, s));
-    return project(path, Wp, gamma, N, K, xq, scale, xsum, M, out, s, base + w.sk, w.sk_bytes);
+    return forward_impl(Wp, gamma, N, K, x, M, false, out, ws, ws_bytes, (cudaStream_t)stream);
+}
+
+BL_API bl_status bitlinear_forward_ex(const uint8_t* Wp, const float* gammas, const int64_t* seg_rows,
+                                      int32_t nseg, int64_t K, const uint16_t* x, int64_t M, int32_t rmsnorm,
+                                      const uint16_t* residual, uint16_t* y, int32_t* acc, void* ws,
+                                      size_t ws_bytes, bl_stream_t stream) {
+    if (nseg < 1 || nseg > 4 || (rmsnorm != 0 && rmsnorm != 1)) return BL_ERR_SHAPE;
+    if (!seg_rows) return BL_ERR_NULL;
+    bl::GemvOut out;
+    int64_t N = 0;
+    for (int i = 0; i < nseg; ++i) {
+        if (seg_rows[i] < 1) return BL_ERR_SHAPE;
+        N += seg_rows[i];
+        if (N > kMaxN) return BL_ERR_SHAPE;
+        if (i < nseg - 1) out.seg_end[i] = (int)N;
+    }
+    if (!forward_args_ok(N, K, M)) return BL_ERR_SHAPE;
+    if (M == 0) return BL_OK;
+    if (!Wp || !gammas || !x || !y) return BL_ERR_NULL;
+    if (!aligned(gammas, 4) || !aligned(x, 2) || !aligned(y, 2) || (residual && !aligned(residual, 2)) ||
+        (acc && !aligned(acc, 4)))
+        return BL_ERR_ALIGN;
+    out.y = y;
+    out.residual = residual;
+    out.acc = acc;
+    return forward_impl(Wp, gammas, N, K, x, M, rmsnorm != 0, out, ws, ws_bytes, (cudaStream_t)stream);
 }
 
 BL_API bl_status bitlinear_ffn(const uint8_t* Wg, const float* gg, const uint8_t* Wu,

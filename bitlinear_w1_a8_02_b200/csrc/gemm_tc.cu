@@ -385,7 +385,10 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
                     for (int j = 0; j < 32; ++j) slot[(size_t)(c * 32 + j) * BM] = v[j];
                 } else if (mv && nb < N) {
-                    store_row_chunk(v, xs, deq, nb, N, static_cast<size_t>(m) * N + nb, out, vec);
+                    // row segments with their own gamma end on 32-column chunks
+                    const int sgi = seg_of(out, nb);
+                    const float dq = sgi == 0 ? deq : __fdiv_rn(gamma_p[sgi], scale[m]);
+                    store_row_chunk(v, xs, dq, nb, N, static_cast<size_t>(m) * N + nb, out, vec);
                 }
             }
             tc::fence_before_sync();
@@ -497,8 +500,8 @@ __global__ void __launch_bounds__(512) gemm_sk_fixup_kernel(int M, int N, int K,
     }
     const bool vec = (N % 8 == 0) && aligned16(out.y) && aligned16(out.y32) && aligned16(out.residual) &&
                      aligned16(out.acc);
-    store_row8(v, xsum[m], __fdiv_rn(*gamma_p, scale[m]), n0 + col, N, static_cast<size_t>(m) * N + n0 + col,
-               out, vec);
+    store_row8(v, xsum[m], __fdiv_rn(gamma_p[seg_of(out, n0 + col)], scale[m]), n0 + col, N,
+               static_cast<size_t>(m) * N + n0 + col, out, vec);
 }
 
 // ---------------------------------------------------------------- host side
@@ -538,6 +541,12 @@ bool make_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, 
 }
 
 }  // namespace
+
+bool gemm_segments_ok(const GemvOut& out, int64_t N) {
+    for (int i = 0; i < 3; ++i)
+        if (out.seg_end[i] < N && out.seg_end[i] % 32 != 0) return false;
+    return true;
+}
 
 bool gemm_tc_ok(int64_t N, int64_t K, const void* Wp, const void* xq) {
     return N >= 1 && K % 64 == 0 && reinterpret_cast<uintptr_t>(Wp) % 16 == 0 &&

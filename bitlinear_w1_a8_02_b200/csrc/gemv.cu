@@ -106,6 +106,7 @@ struct GemvArgs {
     const int32_t* xsum;   // [M] (not fused)
     GemvOut out;
     unsigned* err;         // device error word (bounded waits that give up)
+    int norm;              // fused quantisation: unit-weight RMSNorm of x first
     int seg_chunks;        // 64-byte chunks per K segment of a streamed unit
     int pitch;             // shared-memory row pitch of a stage
     int codes_bytes;       // fused codes area at the start of dynamic shared memory
@@ -156,6 +157,19 @@ __device__ __forceinline__ uint32_t absmax16(uint4 v0, uint4 v1) {
     return max(c & 0xffffu, c >> 16);
 }
 
+// sum of the squares of 16 bf16 values in fp64 (each square is exact there)
+__device__ __forceinline__ double sumsq16(uint4 v0, uint4 v1) {
+    const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+    double ss = 0.0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const double lo = (double)__uint_as_float(w[j] << 16), hi = (double)__uint_as_float(w[j] & 0xffff0000u);
+        ss = __fma_rn(lo, lo, ss);
+        ss = __fma_rn(hi, hi, ss);
+    }
+    return ss;
+}
+
 // PLANES codes of 16 consecutive elements k = 16 g + e with fp32 values f[e]:
 // code rint(f s), taken from the low byte of fl(f s) + 1.5 * 2^23. The per-token
 // scale keeps |f s| <= 127 (1 + 2^-23) for finite inputs, so the clip to
@@ -190,14 +204,20 @@ __device__ __forceinline__ uint8_t* group_codes(uint8_t* codes, int m, int c, in
     return IL ? codes + 16 * c : codes + smem_plane_off(m, 0, KB) + 4 * c;
 }
 
-template <bool IL>
-__device__ __forceinline__ int quant_bf16x16(uint4 v0, uint4 v1, float s, uint8_t* plane0, int KB) {
+// XT and norm: the codes of fl(x * r) (RMSNorm factor r)
+template <bool IL, bool XT>
+__device__ __forceinline__ int quant_bf16x16(uint4 v0, uint4 v1, float s, uint8_t* plane0, int KB, bool norm,
+                                             float r) {
     const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
     float f[16];
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
         f[2 * j] = __uint_as_float(w[j] << 16);
         f[2 * j + 1] = __uint_as_float(w[j] & 0xffff0000u);
+    }
+    if (XT && norm) {
+#pragma unroll
+        for (int e = 0; e < 16; ++e) f[e] = __fmul_rn(f[e], r);
     }
     return quant_pack16<IL>(f, s, plane0, KB);
 }
@@ -207,9 +227,12 @@ __device__ __forceinline__ int quant_bf16x16(uint4 v0, uint4 v1, float s, uint8_
 // codes, and the code sum. Thread 0 records s and the dequantisation factors
 // gamma / s. The first 16-element group of the next token is loaded while the
 // current one is reduced.
-template <bool DUAL, bool IL>
+// XT: the call may ask for the RMSNorm (a.norm); without it the norm code is
+// compiled out (this prologue's size is its latency).
+template <bool DUAL, bool IL, bool XT>
 __device__ void fused_quantise(const GemvArgs& a, int KB, uint8_t* codes, uint32_t (*am_sh)[kWarps],
-                               float* s_sh, int* xs_sh, float* deq_sh, float* deq2_sh) {
+                               double (*ss_sh)[kWarps], float* s_sh, int* xs_sh, float* deq_sh,
+                               float* deq2_sh) {
     const int M = a.M, groups = KB / 4;  // 16-element groups per token
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int c0 = threadIdx.x;
@@ -233,20 +256,40 @@ __device__ void fused_quantise(const GemvArgs& a, int KB, uint8_t* codes, uint32
             n1 = xr[2 * groups + 2 * c0 + 1];
         }
         uint32_t mx = absmax16(v0, v1);  // 0 when this thread has no group
+        const bool norm = XT && a.norm;
+        double ss = norm ? sumsq16(v0, v1) : 0.0;
 #pragma unroll 1
-        for (int c = c0 + kThreads; c < groups; c += kThreads) mx = max(mx, absmax16(xr[2 * c], xr[2 * c + 1]));
+        for (int c = c0 + kThreads; c < groups; c += kThreads) {
+            const uint4 w0 = xr[2 * c], w1 = xr[2 * c + 1];
+            mx = max(mx, absmax16(w0, w1));
+            if (norm) ss += sumsq16(w0, w1);
+        }
         mx = __reduce_max_sync(0xffffffffu, mx);
-        if (lane == 0) am_sh[m][warp] = mx;
+        if (norm) ss = warp_sum(ss);
+        if (lane == 0) {
+            am_sh[m][warp] = mx;
+            if (XT) ss_sh[m][warp] = ss;
+        }
         consumer_sync();
         uint32_t amb = am_sh[m][0];
 #pragma unroll
         for (int w = 1; w < kWarps; ++w) amb = max(amb, am_sh[m][w]);
-        const float s = __fdiv_rn(kActRange, fmaxf(__uint_as_float(amb << 16), kActEps));
+        float amax = __uint_as_float(amb << 16), r = 1.0f;
+        if (norm) {  // unit-weight RMSNorm: max |fl(x r)| = fl(max |x| r)
+            double tot = ss_sh[m][0];
+#pragma unroll
+            for (int w = 1; w < kWarps; ++w) tot += ss_sh[m][w];
+            const float ms = __double2float_rn(__ddiv_rn(tot, (double)(4 * KB)));
+            r = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, kRmsEps)));
+            amax = __fmul_rn(amax, r);
+        }
+        const float s = __fdiv_rn(kActRange, fmaxf(amax, kActEps));
         int sum = 0;
-        if (c0 < groups) sum = quant_bf16x16<IL>(v0, v1, s, group_codes<IL>(codes, m, c0, KB), KB);
+        if (c0 < groups) sum = quant_bf16x16<IL, XT>(v0, v1, s, group_codes<IL>(codes, m, c0, KB), KB, norm, r);
 #pragma unroll 1
         for (int c = c0 + kThreads; c < groups; c += kThreads)
-            sum += quant_bf16x16<IL>(xr[2 * c], xr[2 * c + 1], s, group_codes<IL>(codes, m, c, KB), KB);
+            sum += quant_bf16x16<IL, XT>(xr[2 * c], xr[2 * c + 1], s, group_codes<IL>(codes, m, c, KB), KB, norm,
+                                         r);
         sum = __reduce_add_sync(0xffffffffu, sum);
         if (lane == 0) atomicAdd(&xs_sh[m], sum);
         if (threadIdx.x == 0) {
@@ -342,7 +385,9 @@ __device__ __forceinline__ void bulk_copy(uint32_t dst, const void* src, uint32_
 // segments into a ring of kStages shared-memory stages; the row pitch is
 // congruent to 64 mod 128 bytes so rows g and g + 1 of a quarter-warp fall on
 // different banks.
-template <int NT, int SRC, bool DUAL, bool DP>
+// XT: extended calls (row segments with their own gamma, RMSNorm of x); the
+// plain forward runs the instantiation without that code.
+template <int NT, int SRC, bool DUAL, bool DP, bool XT>
 __global__ void __launch_bounds__(kThreads + 32, NT == 1 ? 3 : 2) gemv_mma_kernel(const GemvArgs a) {
     constexpr int TOK = 8 * NT;
     constexpr bool FUSED = SRC != SRC_CODES;
@@ -354,6 +399,7 @@ __global__ void __launch_bounds__(kThreads + 32, NT == 1 ? 3 : 2) gemv_mma_kerne
     __shared__ float s_sh[TOK];
     __shared__ int xs_sh[TOK];
     __shared__ uint32_t am_sh[TOK][kWarps];
+    __shared__ double ss_sh[SRC == SRC_X && XT ? TOK : 1][kWarps];
     __shared__ float r_sh[TOK];
     __shared__ float deq_sh[TOK], deq2_sh[TOK];
     __shared__ int abort_sh;
@@ -478,7 +524,7 @@ __global__ void __launch_bounds__(kThreads + 32, NT == 1 ? 3 : 2) gemv_mma_kerne
 
     grid_dependency_wait();
     if (SRC == SRC_X) {
-        fused_quantise<DUAL, DP>(a, KB, codes, am_sh, s_sh, xs_sh, deq_sh, deq2_sh);
+        fused_quantise<DUAL, DP, XT>(a, KB, codes, am_sh, ss_sh, s_sh, xs_sh, deq_sh, deq2_sh);
     } else if (SRC == SRC_H) {
         finalise_quantise<DP>(a, KB, codes, s_sh, xs_sh, r_sh, deq_sh);
     } else if (threadIdx.x < TOK && tok0 + (int)threadIdx.x < a.M) {
@@ -653,7 +699,8 @@ __global__ void __launch_bounds__(kThreads + 32, NT == 1 ? 3 : 2) gemv_mma_kerne
 #pragma unroll
                 for (int w = 0; w < kWarps; ++w) sum += red[w][r][cl];
                 const int accv = sum - xs_sh[cl];
-                float v = dequant(accv, deq_sh[cl]);
+                const int sgi = XT ? seg_of(a.out, n) : 0;  // row segments with their own gamma
+                float v = dequant(accv, sgi == 0 ? deq_sh[cl] : __fdiv_rn(a.gamma[sgi], s_sh[cl]));
                 if (!store) continue;
                 const size_t o = (size_t)m * N + n;
                 if (a.out.y32) {
@@ -689,7 +736,7 @@ __global__ void __launch_bounds__(kThreads) gemv_generic_kernel(
     }
     acc = warp_sum(acc);
     if (lane == 0) {
-        const float deq = __fdiv_rn(*gamma_p, scale[m]);
+        const float deq = __fdiv_rn(gamma_p[seg_of(out, n)], scale[m]);
         float v = dequant(acc, deq);
         const size_t o = (size_t)m * N + n;
         if (out.y32) {
@@ -713,9 +760,9 @@ int sm_count() {
     return n;
 }
 
-template <int NT, int SRC, bool DUAL, bool DP = false>
+template <int NT, int SRC, bool DUAL, bool DP = false, bool XT = false>
 cudaError_t launch_variant(const GemvArgs& a, dim3 grid, size_t smem, cudaStream_t s) {
-    auto kern = gemv_mma_kernel<NT, SRC, DUAL, DP>;
+    auto kern = gemv_mma_kernel<NT, SRC, DUAL, DP, XT>;
     static bool done[64];
     int dev = 0;
     cudaGetDevice(&dev);
@@ -729,10 +776,10 @@ cudaError_t launch_variant(const GemvArgs& a, dim3 grid, size_t smem, cudaStream
 
 // Codes in shared memory: a single token takes the dp4a path (the MMA path would
 // spend 7 of its 8 token columns on padding).
-template <int SRC, bool DUAL>
+template <int SRC, bool DUAL, bool XT = false>
 cudaError_t launch_fused(const GemvArgs& a, dim3 grid, size_t smem, cudaStream_t s) {
-    if (a.M == 1) return launch_variant<1, SRC, DUAL, true>(a, grid, smem, s);
-    return launch_variant<1, SRC, DUAL, false>(a, grid, smem, s);
+    if (a.M == 1) return launch_variant<1, SRC, DUAL, true, XT>(a, grid, smem, s);
+    return launch_variant<1, SRC, DUAL, false, XT>(a, grid, smem, s);
 }
 
 // Segment plan, shared-memory size and grid of one streamed GEMV launch.
@@ -778,26 +825,41 @@ GemvArgs base_args(const uint8_t* Wp, const float* gamma, int64_t N, int64_t K, 
 
 bool gemv_fast_ok(int64_t N, int64_t K) { return N >= 1 && K % 256 == 0; }
 
+bool gemv_segments_ok(const GemvOut& out, int64_t N) {
+    for (int i = 0; i < 3; ++i)
+        if (out.seg_end[i] < N && out.seg_end[i] % 16 != 0) return false;
+    return true;
+}
+
 bool gemv_fused_ok(int64_t M, int64_t K) {
     return M >= 1 && M <= kFusedMaxTokens && (size_t)M * (K + 64) <= (size_t)kFusedSmemLimit;
 }
 
 cudaError_t launch_gemv(const uint8_t* Wp, const float* gamma, int64_t N, int64_t K,
                         const int8_t* Xp, const float* scale, const int32_t* xsum, int64_t M,
-                        const GemvOut& out, cudaStream_t s, const uint16_t* x_fused) {
+                        const GemvOut& out, cudaStream_t s, const uint16_t* x_fused, bool rmsnorm) {
     if (M == 0 || N == 0) return cudaSuccess;
     if (x_fused && !gemv_fused_ok(M, K)) return cudaErrorInvalidValue;
+    if (!gemv_segments_ok(out, N)) return cudaErrorInvalidValue;
     GemvArgs a = base_args(Wp, gamma, N, K, M, out);
     a.x = x_fused;
+    a.norm = (x_fused && rmsnorm) ? 1 : 0;
     a.Xp = Xp;
     a.scale = scale;
     a.xsum = xsum;
     StreamPlan p;
     cudaError_t e = plan_stream(a, N, K, M, 1, x_fused != nullptr, p);
     if (e != cudaSuccess) return e;
-    if (x_fused) return launch_fused<SRC_X, false>(a, dim3(p.grid_x, 1), p.smem, s);
-    if (M <= 8) return launch_variant<1, SRC_CODES, false>(a, dim3(p.grid_x, 1), p.smem, s);
-    return launch_variant<2, SRC_CODES, false>(a, dim3(p.grid_x, (unsigned)((M + 15) / 16)), p.smem, s);
+    const dim3 g1(p.grid_x, 1), g2(p.grid_x, (unsigned)((M + 15) / 16));
+    const bool xt = a.norm || out.seg_end[0] < N;
+    if (xt) {
+        if (x_fused) return launch_fused<SRC_X, false, true>(a, g1, p.smem, s);
+        if (M <= 8) return launch_variant<1, SRC_CODES, false, false, true>(a, g1, p.smem, s);
+        return launch_variant<2, SRC_CODES, false, false, true>(a, g2, p.smem, s);
+    }
+    if (x_fused) return launch_fused<SRC_X, false>(a, g1, p.smem, s);
+    if (M <= 8) return launch_variant<1, SRC_CODES, false>(a, g1, p.smem, s);
+    return launch_variant<2, SRC_CODES, false>(a, g2, p.smem, s);
 }
 
 cudaError_t launch_ffn_up_fused(const uint8_t* Wg, const float* gg, const uint8_t* Wu, const float* gu,

@@ -18,8 +18,10 @@ cudaError_t launch_count_bad_codes(const uint8_t* Wp, int64_t nbytes, unsigned l
                                    cudaStream_t s);
 
 // ---- activation quantisation (actquant.cu); layout is an XqLayout
+// rmsnorm: quantise fl(x * r), r = 1 / sqrtf(float(sum_k x^2 / K) + 1e-5) per token
+// (unit-weight RMSNorm, sum in fp64), instead of x.
 cudaError_t launch_act_quant(const uint16_t* x, int64_t M, int64_t K, int layout, int8_t* xq,
-                             float* scale, int32_t* xsum, cudaStream_t s);
+                             float* scale, int32_t* xsum, cudaStream_t s, bool rmsnorm = false);
 
 // ---- decode GEMV (gemv.cu)
 // Output modes: bf16 y (+ residual, + int32 acc dump) or fp32 dequantised y32.
@@ -28,15 +30,25 @@ struct GemvOut {
     const uint16_t* residual = nullptr; // [M, N] bf16 bits or null
     int32_t* acc = nullptr;             // [M, N] or null
     float* y32 = nullptr;               // [M, N] fp32 (used instead of y when set)
+    // Row segments with their own gamma (weights stacked row-wise): output row n
+    // uses gamma[seg_of(n)]; rows >= seg_end[i] lie past segment i. One segment by
+    // default. The GEMV needs the ends on 16-row tiles, the GEMM on 32 columns.
+    int seg_end[3] = {0x7fffffff, 0x7fffffff, 0x7fffffff};
 };
+
+__host__ __device__ __forceinline__ int seg_of(const GemvOut& o, int n) {
+    return (n >= o.seg_end[0]) + (n >= o.seg_end[1]) + (n >= o.seg_end[2]);
+}
 // Requires K % 256 == 0 and 16-byte aligned Wp. Codes either come as PLANES
 // layout Xp (+ scale, xsum) from the act-quant kernel, or, when x_fused is given
 // (16-byte aligned bf16 x, gemv_fused_ok(M, K)), are computed inside the kernel.
 bool gemv_fast_ok(int64_t N, int64_t K);
 bool gemv_fused_ok(int64_t M, int64_t K);
+bool gemv_segments_ok(const GemvOut& out, int64_t N);  // segment ends on 16-row tiles
 cudaError_t launch_gemv(const uint8_t* Wp, const float* gamma, int64_t N, int64_t K,
                         const int8_t* Xp, const float* scale, const int32_t* xsum, int64_t M,
-                        const GemvOut& out, cudaStream_t s, const uint16_t* x_fused = nullptr);
+                        const GemvOut& out, cudaStream_t s, const uint16_t* x_fused = nullptr,
+                        bool rmsnorm = false);  // fused quantisation of a unit-weight RMSNorm of x
 // FFN sub-layer for M <= 4 tokens in two streamed kernels (K = d for the up
 // projections, f for the down one; both multiples of 256, f + 64 codes per token
 // in shared memory). up: h = relu(g)^2 * u [M, f] fp32 plus per (token, 16-row
@@ -57,6 +69,7 @@ cudaError_t launch_gemv_generic(const uint8_t* Wp, const float* gamma, int64_t N
 // xq_g16t: G16T layout codes for M tokens. Requires K % 64 == 0 and 16-byte
 // aligned Wp and xq_g16t (TMA); any M, N (tails are zero-filled by the TMA).
 bool gemm_tc_ok(int64_t N, int64_t K, const void* Wp, const void* xq);
+bool gemm_segments_ok(const GemvOut& out, int64_t N);  // segment ends on 32-column chunks
 int gemm_tc_tile_width(int64_t M, int64_t N, int sms);
 // sk_ws / sk_ws_bytes: scratch for stream-K pieces (gemm_sk_workspace_bytes of the
 // device's SM count); null or too small means the data-parallel split only.

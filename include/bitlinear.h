@@ -143,6 +143,39 @@ bl_status bitlinear_forward(const uint8_t* Wp, const float* gamma, int64_t N, in
                             void* ws, size_t ws_bytes, bl_stream_t stream);
 
 /*
+ * Several BitLinear projections of one input in one call, optionally after a
+ * unit-weight RMSNorm of the input: the attention side of a BitNet b1.58 block
+ * (paper card "BitNet b1.58 2B4T Technical Report", "Method Adaptation":
+ * BitLinear replaces the linear layers, subln sub-layer normalisation; fishai
+ * digest, BitLinear list). The query, key and value projections read the same
+ * normalised x; the output projection reads the subln-normalised attention
+ * output and adds the residual.
+ *   y[m, n] = [residual[m, n] +] bf16(acc[m, n] * gammas[seg(n)] / s_m)
+ *   xq, s   = quant(rmsnorm ? x * r : x),  r = 1 / sqrtf(float(sum_k x^2 / K) + 1e-5)
+ *             per token (sum in fp64; x * r kept in fp32 and quantised as in
+ *             bitlinear_forward)
+ * Arguments:
+ *   Wp        [N, K/4] device: the packed rows of nseg weight matrices stacked
+ *             row-wise (each packed by bitlinear_pack_weights; packed rows are
+ *             independent, so stacking is a byte copy); N = sum of seg_rows
+ *   gammas    [nseg] device fp32: gamma of each matrix, in the same order
+ *   seg_rows  [nseg] host: rows of each matrix, each >= 1; 1 <= nseg <= 4
+ *   K, x, M   as bitlinear_forward
+ *   rmsnorm   0: quantise x; 1: quantise the unit-weight RMSNorm of x
+ *   residual, y, acc   [M, N], as bitlinear_forward
+ *   ws        device workspace of bitlinear_workspace_bytes(BL_OP_FORWARD, M, N, K)
+ * Kernel choice as bitlinear_forward. Segment boundaries on multiples of 16 rows
+ * keep the streamed GEMV (M <= 16) and on multiples of 32 the tensor-core GEMM;
+ * other boundaries run the generic kernel. Errors: BL_ERR_SHAPE for nseg outside
+ * 1..4, rmsnorm not 0 or 1, a segment without rows, or the bitlinear_forward
+ * shape rules on N = sum of seg_rows; otherwise as bitlinear_forward.
+ */
+bl_status bitlinear_forward_ex(const uint8_t* Wp, const float* gammas, const int64_t* seg_rows,
+                               int32_t nseg, int64_t K, const uint16_t* x, int64_t M,
+                               int32_t rmsnorm, const uint16_t* residual, uint16_t* y,
+                               int32_t* acc, void* ws, size_t ws_bytes, bl_stream_t stream);
+
+/*
  * One FFN sub-layer of BitNet b1.58 (fishai digest: ReLU^2 in the FFN, subln;
  * paper card, "Method Adaptation": subln, ReLU^2 feed-forward, no bias):
  *   xq, s   = quant(x)                       x [M, d]

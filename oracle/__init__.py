@@ -62,6 +62,7 @@ def _l():
             "orc_subln_rms": (F, [P, I, P]),
             "orc_relu2_gate": (F, [F, F]),
             "orc_ffn_layer": (ctypes.c_int, [P, F, P, F, P, F, I, I, P, I, P, P, P, P, P, P, P]),
+            "orc_forward_ex": (ctypes.c_int, [P, P, P, I, I, P, I, I, P, P, P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(lib, name)
@@ -216,6 +217,27 @@ def forward(Wp: np.ndarray, gamma, x_bf16: np.ndarray, residual=None):
     if rc != 0:
         raise MemoryError("oracle forward failed")
     return dict(y=y, acc=acc, xq=xq, s=s, xsum=xs)
+
+
+def forward_ex(Wp: np.ndarray, gammas, seg_rows, x_bf16: np.ndarray, rmsnorm=False, residual=None):
+    """Projections of one input against row-stacked weight matrices (segment i:
+    seg_rows[i] rows, gamma gammas[i]), optionally after a unit-weight RMSNorm of
+    the input. Returns dict(y, acc); y as bf16 bits [M, N]."""
+    Wp = _c(Wp, np.uint8)
+    x = _c(x_bf16, np.uint16)
+    g = _c(np.asarray(gammas, np.float32), np.float32)
+    rows = _c(np.asarray(seg_rows, np.int64), np.int64)
+    N = int(rows.sum())
+    M, K = x.shape
+    assert Wp.shape == (N, K // 4) and g.size == rows.size
+    res = None if residual is None else _c(residual, np.uint16)
+    y = np.empty((M, N), np.uint16)
+    acc = np.empty((M, N), np.int32)
+    rc = _l().orc_forward_ex(_p(Wp), _p(g), _p(rows), rows.size, K, _p(x), M, int(bool(rmsnorm)), _p(res),
+                             _p(y), _p(acc))
+    if rc != 0:
+        raise MemoryError("oracle forward_ex failed")
+    return dict(y=y, acc=acc)
 
 
 def subln_rms(h: np.ndarray):

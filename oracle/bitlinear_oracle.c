@@ -321,3 +321,56 @@ done:
     free(xf); free(xq); free(s); free(accg); free(accu); free(h); free(hn); free(q2); free(s2); free(accd);
     return rc;
 }
+
+/* ------------------------------------------------------------------------- */
+/* Several BitLinear projections of one input: the weight matrices are stacked
+ * row-wise (for example the attention's query, key and value projections, which
+ * read the same x), each keeps its own absmean gamma ([card] "Method
+ * Adaptation": absmean per weight tensor), and the input may first pass through
+ * a unit-weight RMSNorm (the block's pre-norm, and the subln in front of the
+ * attention output projection; [news] BitLinear list, [card] "Method
+ * Adaptation": subln). Reading: the same RMSNorm as the FFN's subln (sum of
+ * squares in fp64, r = 1 / sqrtf(float(sum / K) + 1e-5f), xn = x * r in fp32,
+ * not rounded to bf16 before the quantisation).
+ *   Wp [N, K/4], N = sum of seg_rows[0..nseg-1]; rows of segment i use gammas[i].
+ *   x, residual, y: [M, K], [M, N], [M, N] bf16 bits; acc_out [M, N] or NULL.   */
+int orc_forward_ex(const uint8_t* Wp, const float* gammas, const int64_t* seg_rows, int64_t nseg,
+                   int64_t K, const uint16_t* x, int64_t M, int64_t rmsnorm,
+                   const uint16_t* residual, uint16_t* y, int32_t* acc_out) {
+    int64_t N = 0;
+    for (int64_t i = 0; i < nseg; ++i) N += seg_rows[i];
+    float* xf = (float*)malloc(sizeof(float) * (size_t)(M * K));
+    float* xn = (float*)malloc(sizeof(float) * (size_t)(M * K));
+    int8_t* xq = (int8_t*)malloc((size_t)(M * K));
+    float* s = (float*)malloc(sizeof(float) * (size_t)M);
+    int32_t* acc = (int32_t*)malloc(sizeof(int32_t) * (size_t)(M * N));
+    int rc = 0;
+    if (!xf || !xn || !xq || !s || !acc) {
+        rc = -1;
+        goto done;
+    }
+    orc_bf16_to_f32_array(x, M * K, xf);
+    for (int64_t m = 0; m < M; ++m) {
+        if (rmsnorm)
+            orc_subln_rms(xf + m * K, K, xn + m * K);
+        else
+            memcpy(xn + m * K, xf + m * K, sizeof(float) * (size_t)K);
+    }
+    orc_quant_act(xn, M, K, xq, s, NULL);
+    orc_int_gemm_packed(Wp, xq, M, N, K, acc);
+    for (int64_t m = 0; m < M; ++m) {
+        int64_t n = 0;
+        for (int64_t i = 0; i < nseg; ++i) {
+            float deq = gammas[i] / s[m];
+            for (int64_t e = 0; e < seg_rows[i]; ++e, ++n) {
+                float v = (float)acc[m * N + n] * deq;
+                if (residual) v = orc_bf16_to_f32(residual[m * N + n]) + v;
+                y[m * N + n] = orc_f32_to_bf16(v);
+            }
+        }
+    }
+    if (acc_out) memcpy(acc_out, acc, sizeof(int32_t) * (size_t)(M * N));
+done:
+    free(xf); free(xn); free(xq); free(s); free(acc);
+    return rc;
+}

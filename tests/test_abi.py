@@ -130,6 +130,28 @@ def test_host_validation_pack_quant_ffn_validate():
     assert v(None, 4, 16, None, P(A), 256, None) == NULL
 
 
+def test_host_validation_forward_ex():
+    L = bl.lib()
+    F = L.bitlinear_forward_ex
+    need = L.bitlinear_workspace_bytes(bl.BL_OP_FORWARD, 1, 96, 256)
+
+    def call(rows, nseg=None, K=256, M=1, norm=0, g=A, ws=A, wsb=need):
+        arr = None if rows is None else (ctypes.c_int64 * max(1, len(rows)))(*rows)
+        n = len(rows) if nseg is None else nseg
+        return F(P(A), P(g), arr, n, K, P(A), M, norm, None, P(A), None, P(ws), wsb, None)
+
+    assert call([48, 16, 32], nseg=0) == SHAPE
+    assert call([48, 16, 32, 8, 8], nseg=5) == SHAPE
+    assert call([48, 0, 32]) == SHAPE
+    assert call([48, 16, 32], norm=2) == SHAPE
+    assert call([48, 16, 32], K=258) == SHAPE
+    assert call(None, nseg=3) == NULL
+    assert call([48, 16, 32], M=0) == OK
+    assert call([48, 16, 32], g=None) == NULL
+    assert call([48, 16, 32], g=A + 2) == ALIGN
+    assert call([48, 16, 32], wsb=need - 1) == WS
+
+
 def test_host_validation_selftest():
     L = bl.lib()
     assert L.bitlinear_selftest_timeout(0, None) == SHAPE

@@ -182,6 +182,56 @@ def test_forward_stream_k_split_tiles(cuda_device, M, N, K):
     check_forward_full(Wp, gamma, Wp_ref, g_ref, x, cuda_device, residual=res)
 
 
+def stacked(shapes_rows, K, seed, dev):
+    """Pack each matrix on the GPU and in the oracle; stack rows and gammas."""
+    parts = [pack_both(make_weights(n, K, synth.SIGMA_2B, seed + i), dev) for i, n in enumerate(shapes_rows)]
+    Wp = torch.cat([p[0] for p in parts])
+    gam = torch.cat([p[1].reshape(1) for p in parts])
+    Wp_ref = np.concatenate([p[2] for p in parts])
+    g_ref = [p[3] for p in parts]
+    return Wp, gam, Wp_ref, g_ref
+
+
+@pytest.mark.parametrize("M", [1, 3, 9, 40, 300])
+@pytest.mark.parametrize("norm", [False, True])
+def test_forward_ex_qkv(cuda_device, M, norm):
+    """The attention's query/key/value projections (2560 -> 2560 / 640 / 640) of
+    one input in one call, with and without the block's pre-norm: single-token
+    dp4a GEMV, fused multi-token GEMV, act-quant + GEMV, and the tensor-core GEMM."""
+    K, rows = 2560, [2560, 640, 640]
+    Wp, gam, Wp_ref, g_ref = stacked(rows, K, 80, cuda_device)
+    x = synth.activations(M, K, seed=81 + M, outliers=True)
+    y, acc = bl.forward_ex(Wp, gam, rows, x.to(cuda_device), rmsnorm=norm, want_acc=True)
+    ref = oracle.forward_ex(Wp_ref, g_ref, rows, bits(x), rmsnorm=norm)
+    assert np.array_equal(np_(acc), ref["acc"]), "int32 accumulators"
+    assert_bf16_close(bits(y), ref["y"])
+    assert_bf16_exact(bits(y), ref["y"])
+
+
+@pytest.mark.parametrize("M", [1, 4, 17])
+def test_forward_ex_output_projection_with_subln(cuda_device, M):
+    """The attention output projection (2560 -> 2560): subln RMSNorm of the
+    attention output, quantisation, projection, residual add."""
+    K, rows = 2560, [2560]
+    Wp, gam, Wp_ref, g_ref = stacked(rows, K, 90, cuda_device)
+    x = synth.activations(M, K, seed=91 + M, outliers=False)
+    res = synth.activations(M, K, seed=92 + M, outliers=False)
+    y = bl.forward_ex(Wp, gam, rows, x.to(cuda_device), rmsnorm=True, residual=res.to(cuda_device))
+    ref = oracle.forward_ex(Wp_ref, g_ref, rows, bits(x), rmsnorm=True, residual=bits(res))
+    assert_bf16_exact(bits(y), ref["y"])
+
+
+@pytest.mark.parametrize("M", [1, 20])
+def test_forward_ex_unaligned_segments_take_the_generic_kernel(cuda_device, M):
+    K, rows = 256, [40, 24, 8]
+    Wp, gam, Wp_ref, g_ref = stacked(rows, K, 95, cuda_device)
+    x = synth.activations(M, K, seed=96, outliers=True)
+    y, acc = bl.forward_ex(Wp, gam, rows, x.to(cuda_device), rmsnorm=True, want_acc=True)
+    ref = oracle.forward_ex(Wp_ref, g_ref, rows, bits(x), rmsnorm=True)
+    assert np.array_equal(np_(acc), ref["acc"])
+    assert_bf16_exact(bits(y), ref["y"])
+
+
 def test_forward_misaligned_input_takes_generic_path(cuda_device):
     K, N, M = 256, 64, 20
     W = make_weights(N, K, 0.02, seed=21)

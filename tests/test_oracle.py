@@ -305,3 +305,63 @@ def test_ffn_requant_tracks_unnormalised_codes():
     mismatch = np.mean(q_direct != out["q2"])
     assert mismatch < 1e-3
     assert np.all(np.abs(q_direct.astype(int) - out["q2"].astype(int)) <= 1)
+
+
+# ----------------------------------------------------------------------------- stacked projections
+
+def test_forward_ex_structured_closed_form():
+    """Two stacked matrices with their own gamma, constant input.
+
+    Segment 0 row j has j+1 leading +1 codes, segment 1 rows are all -1; a constant
+    token c quantises to 127 everywhere, so acc = 127 (j+1) and -127 K, and
+    y = acc * gamma_i * a / 127 with a = c, or a = c r after the unit-weight
+    RMSNorm (r = 1 / sqrt(c^2 + eps)). A swapped gamma, a missing norm or a sum in
+    place of the mean moves y far outside bf16 rounding.
+    """
+    K, n0, n1 = 16, 6, 3
+    g = np.array([0.5, 0.25], np.float32)
+    W0 = _packed_rows([[1] * (j + 1) + [0] * (K - j - 1) for j in range(n0)])
+    W1 = _packed_rows([[-1] * K for _ in range(n1)])
+    Wp = np.concatenate([W0, W1])
+    for c, res_val, norm in ((0.0625, 0.0, False), (0.0625, 1.5, True), (3.0, -2.0, True)):
+        x = bf16_bits(torch.full((1, K), c).to(torch.bfloat16))
+        res = bf16_bits(torch.full((1, n0 + n1), res_val).to(torch.bfloat16))
+        out = oracle.forward_ex(Wp, g, [n0, n1], x, rmsnorm=norm, residual=res)
+        cb = float(torch.tensor(c).to(torch.bfloat16))
+        a = cb / math.sqrt(cb * cb + 1e-5) if norm else cb
+        acc = [127 * (j + 1) for j in range(n0)] + [-127 * K] * n1
+        gam = [float(g[0])] * n0 + [float(g[1])] * n1
+        assert out["acc"][0].tolist() == acc
+        term = np.array([acc[n] * gam[n] * a / 127 for n in range(n0 + n1)])
+        y = res_val + term
+        got = oracle.bf16_to_f32(out["y"])[0].astype(np.float64)
+        # one bf16 rounding of the sum, plus fp32 roundings far below it
+        assert np.all(np.abs(got - y) <= 2.0 ** -8 * (np.abs(res_val) + np.abs(term))), (norm, got, y)
+
+
+def test_forward_ex_segments_are_the_separate_projections():
+    K, M = 256, 5
+    Ws = [synth.weights(n, K, 0.02, 70 + i) for i, n in enumerate((48, 16, 32))]
+    packed = [oracle.pack_weights(bf16_bits(w)) for w in Ws]
+    x = bf16_bits(synth.activations(M, K, seed=71, outliers=True))
+    res = bf16_bits(synth.activations(M, 96, seed=72, outliers=False))
+    out = oracle.forward_ex(np.concatenate([p[0] for p in packed]), [p[1] for p in packed], [48, 16, 32], x,
+                            residual=res)
+    col = 0
+    for (Wp, gamma), n in zip(packed, (48, 16, 32)):
+        ref = oracle.forward(Wp, gamma, x, residual=np.ascontiguousarray(res[:, col:col + n]))
+        assert np.array_equal(out["acc"][:, col:col + n], ref["acc"])
+        assert np.array_equal(out["y"][:, col:col + n], ref["y"])
+        col += n
+
+
+def test_forward_ex_rmsnorm_only_rescales_the_codes():
+    # The RMSNorm is a positive per-token rescale: the codes (so acc) are those of
+    # x itself except at rare rounding ties.
+    K, N, M = 512, 64, 16
+    Wp, gamma = oracle.pack_weights(bf16_bits(synth.weights(N, K, 0.02, 73)))
+    x = bf16_bits(synth.activations(M, K, seed=74, outliers=True))
+    plain = oracle.forward_ex(Wp, [gamma], [N], x, rmsnorm=False)
+    normed = oracle.forward_ex(Wp, [gamma], [N], x, rmsnorm=True)
+    diff = np.abs(plain["acc"].astype(np.int64) - normed["acc"].astype(np.int64))
+    assert np.mean(diff != 0) < 0.05 and np.all(diff <= 3 * 2)
