@@ -12,7 +12,8 @@ and replayed.
 
 Extras on the same line: batched decode (M = 4, 8, 16), prefill int8 TOPS
 (M = 512, 2048, 4096), the 100B-class bandwidth case, the 30-layer FFN chain,
-the roofline of the dominant kernel, the end-to-end number through the public
+every BitLinear of 30 decoder layers at one token (Q/K/V with the pre-norm, the
+output projection with its subln, the FFN), the roofline of the dominant kernel, the end-to-end number through the public
 API with host buffers, the CPU oracle baseline and the SM clocks.
 
 Multi-GPU: one process per GPU (torchrun); every rank runs the same independent
@@ -378,7 +379,47 @@ def run_extras(args, bl, synth, dev, hbm_peak, int8_peak):
             ent["frac_int8_peak"] = round(tops / int8_peak, 4)
         ffn[f"M{M}"] = ent
     out["ffn_2b_30_layers"] = ffn
-    del layers
+
+    # Every BitLinear of a 2B-shaped decoder layer, 30 layers, one token per step:
+    # Q/K/V in one call with the block's pre-norm, the output projection with its
+    # subln and the residual, then the FFN. The attention itself (RoPE, softmax,
+    # the KV cache) is not part of this library: the output projection reads a
+    # fixed synthetic attention output.
+    qkv_rows = [2560, 640, 640]
+    dec = []
+    for layer in range(LAYERS):
+        qkv = [bl.pack_weights(synth.weights(n, d, synth.SIGMA_2B, 5000 + 10 * layer + i, device=dev))
+               for i, n in enumerate(qkv_rows)]
+        o_w = bl.pack_weights(synth.weights(d, d, synth.SIGMA_2B, 5000 + 10 * layer + 3, device=dev))
+        dec.append((torch.cat([w for w, _ in qkv]), torch.cat([g_.reshape(1) for _, g_ in qkv]),
+                    o_w[0], o_w[1].reshape(1)))
+    linears = {}
+    for M in (1,):
+        h0 = synth.activations(M, d, seed=3, outliers=False, device=dev)
+        attn = synth.activations(M, d, seed=4, outliers=False, device=dev)
+        yqkv = torch.empty((M, sum(qkv_rows)), dtype=torch.bfloat16, device=dev)
+        hbuf = [torch.empty_like(h0) for _ in range(3)]
+        ws_f = torch.empty(bl.workspace_bytes(bl.BL_OP_FFN, M, f, d), dtype=torch.uint8, device=dev)
+        ws_q = torch.empty(bl.workspace_bytes(bl.BL_OP_FORWARD, M, sum(qkv_rows), d), dtype=torch.uint8,
+                           device=dev)
+
+        def fn():
+            h = h0
+            for li in range(LAYERS):
+                wq, gq, wo, go = dec[li]
+                g_, u_, d_ = layers[li]
+                bl.forward_ex(wq, gq, qkv_rows, h, rmsnorm=True, out=yqkv, ws=ws_q)
+                h1 = hbuf[(2 * li) % 3]
+                bl.forward_ex(wo, go, [d], attn, rmsnorm=True, residual=h, out=h1, ws=ws_q)
+                h2 = hbuf[(2 * li + 1) % 3]
+                bl.ffn(g_[0], g_[1], u_[0], u_[1], d_[0], d_[1], h1, residual=h1, out=h2, ws=ws_f)
+                h = h2
+        ms = time_graph(torch, fn, reps=5)
+        wbytes = LAYERS * (sum(qkv_rows) * d + d * d + 3 * d * f) / 4
+        linears[f"M{M}"] = {"ms_30_layers": round(ms, 4), "us_per_layer": round(ms * 1e3 / LAYERS, 2),
+                            "launches_per_layer": 4, "packed_gbs": round(wbytes / (ms * 1e-3) / 1e9, 1)}
+    out["decoder_linears_2b_30_layers"] = linears
+    del layers, dec
     torch.cuda.empty_cache()
     return out
 
