@@ -36,6 +36,8 @@ SIGNATURES = {
     "bitlinear_pack_weights": (_ST, [_P, ctypes.c_int, _I, _I, _P, _P, _P, _S, _P]),
     "bitlinear_quant_act": (_ST, [_P, _I, _I, _P, _P, _P, _P]),
     "bitlinear_forward": (_ST, [_P, _P, _I, _I, _P, _I, _P, _P, _P, _P, _S, _P]),
+    "bitlinear_pack_weights_rowwise": (_ST, [_P, ctypes.c_int32, _I, _I, _P, _P, _P]),
+    "bitlinear_forward_rowwise": (_ST, [_P, _P, _I, _I, _P, _I, _P, _P, _P, _P, _S, _P]),
     "bitlinear_forward_ex": (_ST, [_P, _P, _P, ctypes.c_int32, _I, _P, _I, ctypes.c_int32, _P, _P, _P, _P, _S,
                                    _P]),
     "bitlinear_ffn": (_ST, [_P, _P, _P, _P, _P, _P, _I, _I, _P, _I, _P, _P, _P, _S, _P]),
@@ -169,6 +171,43 @@ def forward(Wp: torch.Tensor, gamma: torch.Tensor, x: torch.Tensor,
     st = lib().bitlinear_forward(_ptr(Wp), _ptr(gamma), N, K, _ptr(x), M, _ptr(residual), _ptr(y),
                                  _ptr(acc), _ptr(ws), ws.numel(), _stream(x.device))
     _check(st, "bitlinear_forward")
+    return (y, acc) if want_acc else y
+
+
+def pack_weights_rowwise(W: torch.Tensor):
+    """Per-row absmean variant: W [N, K] (bf16 or fp32, CUDA) -> (Wp uint8 [N, K/4], gammas fp32 [N])."""
+    if W.dtype not in (torch.bfloat16, torch.float32):
+        raise TypeError("W must be bf16 or fp32")
+    _cuda(W, "W", W.dtype)
+    N, K = W.shape
+    Wp = torch.empty((N, K // 4), dtype=torch.uint8, device=W.device)
+    gammas = torch.empty(N, dtype=torch.float32, device=W.device)
+    st = lib().bitlinear_pack_weights_rowwise(_ptr(W), BL_FP32 if W.dtype == torch.float32 else BL_BF16, N, K,
+                                              _ptr(Wp), _ptr(gammas), _stream(W.device))
+    _check(st, "bitlinear_pack_weights_rowwise")
+    return Wp, gammas
+
+
+def forward_rowwise(Wp: torch.Tensor, gammas: torch.Tensor, x: torch.Tensor,
+                    residual: Optional[torch.Tensor] = None, want_acc: bool = False,
+                    out: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None):
+    """bitlinear_forward with one gamma per output row."""
+    _cuda(Wp, "Wp", torch.uint8)
+    _cuda(x, "x", torch.bfloat16)
+    _cuda(gammas, "gammas", torch.float32)
+    N, KB = Wp.shape
+    M, K = x.shape
+    if K != 4 * KB or gammas.numel() != N:
+        raise ValueError("shapes of Wp, gammas and x do not match")
+    if residual is not None:
+        _cuda(residual, "residual", torch.bfloat16)
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device) if out is None else out
+    acc = torch.empty((M, N), dtype=torch.int32, device=x.device) if want_acc else None
+    need = workspace_bytes(BL_OP_FORWARD, M, N, K)
+    ws = _WS.get(x.device, need) if ws is None else ws
+    st = lib().bitlinear_forward_rowwise(_ptr(Wp), _ptr(gammas), N, K, _ptr(x), M, _ptr(residual), _ptr(y),
+                                         _ptr(acc), _ptr(ws), ws.numel(), _stream(x.device))
+    _check(st, "bitlinear_forward_rowwise")
     return (y, acc) if want_acc else y
 
 

@@ -180,6 +180,20 @@ BL_API bl_status bitlinear_pack_weights(const void* W, int wdt, int64_t N, int64
     return BL_OK;
 }
 
+BL_API bl_status bitlinear_pack_weights_rowwise(const void* W, int wdt, int64_t N, int64_t K, uint8_t* Wp,
+                                                float* gammas, bl_stream_t stream) {
+    if (wdt != BL_BF16 && wdt != BL_FP32) return BL_ERR_DTYPE;
+    if (N < 1 || K < 4 || K % 4 != 0 || N > kMaxN || K > kMaxK) return BL_ERR_SHAPE;
+    if (!W || !Wp || !gammas) return BL_ERR_NULL;
+    if (!aligned(W, 16) || !aligned(gammas, 4)) return BL_ERR_ALIGN;
+    if (bl_status st = check_device()) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    const bool fp32 = wdt == BL_FP32;
+    BL_TRY(bl::launch_absmean_rows(W, fp32, N, K, gammas, s));
+    BL_TRY(bl::launch_ternary_pack(W, fp32, N, K, gammas, Wp, s, true));
+    return BL_OK;
+}
+
 BL_API bl_status bitlinear_quant_act(const uint16_t* x, int64_t M, int64_t K, int8_t* xq,
                                      float* scale, int32_t* xsum, bl_stream_t stream) {
     if (M < 0 || M > kMaxM || K < 4 || K % 4 != 0 || K > kMaxK) return BL_ERR_SHAPE;
@@ -265,6 +279,23 @@ BL_API bl_status bitlinear_forward_ex(const uint8_t* Wp, const float* gammas, co
     out.residual = residual;
     out.acc = acc;
     return forward_impl(Wp, gammas, N, K, x, M, rmsnorm != 0, out, ws, ws_bytes, (cudaStream_t)stream);
+}
+
+BL_API bl_status bitlinear_forward_rowwise(const uint8_t* Wp, const float* gammas, int64_t N, int64_t K,
+                                           const uint16_t* x, int64_t M, const uint16_t* residual, uint16_t* y,
+                                           int32_t* acc, void* ws, size_t ws_bytes, bl_stream_t stream) {
+    if (!forward_args_ok(N, K, M)) return BL_ERR_SHAPE;
+    if (M == 0 || N == 0) return BL_OK;
+    if (!Wp || !gammas || !x || !y) return BL_ERR_NULL;
+    if (!aligned(gammas, 4) || !aligned(x, 2) || !aligned(y, 2) || (residual && !aligned(residual, 2)) ||
+        (acc && !aligned(acc, 4)))
+        return BL_ERR_ALIGN;
+    bl::GemvOut out;
+    out.y = y;
+    out.residual = residual;
+    out.acc = acc;
+    out.per_row = 1;
+    return forward_impl(Wp, gammas, N, K, x, M, false, out, ws, ws_bytes, (cudaStream_t)stream);
 }
 
 BL_API bl_status bitlinear_ffn(const uint8_t* Wg, const float* gg, const uint8_t* Wu,

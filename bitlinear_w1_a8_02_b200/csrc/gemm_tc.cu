@@ -114,6 +114,26 @@ struct WorkIter {
     }
 };
 
+// Per-row gamma variant: outputs nb .. nb + cnt - 1 of one row, each with
+// deq = gamma[n] / s (one IEEE division per output, as the definition reads).
+template <int CNT>
+__device__ __forceinline__ void store_row_per_row_gamma(const uint32_t* v, int xs, float s, const float* gamma,
+                                                        int nb, int N, size_t o, const GemvOut& out) {
+#pragma unroll 4
+    for (int j = 0; j < CNT; ++j) {
+        if (nb + j >= N) break;
+        const int a = static_cast<int>(v[j]) - xs;
+        float f = dequant(a, __fdiv_rn(gamma[nb + j], s));
+        if (out.y32) {
+            out.y32[o + j] = f;
+        } else {
+            if (out.residual) f = __fadd_rn(bf16_bits_to_f32(out.residual[o + j]), f);
+            out.y[o + j] = f32_to_bf16_bits(f);
+        }
+        if (out.acc) out.acc[o + j] = a;
+    }
+}
+
 // Dequantise and store 32 consecutive outputs of one row (one TMEM load).
 __device__ __forceinline__ void store_row_chunk(const uint32_t (&v)[32], int xs, float deq, int nb,
                                                 int N, size_t o, const GemvOut& out, bool vec) {
@@ -174,7 +194,9 @@ __device__ __forceinline__ void store_row_chunk(const uint32_t (&v)[32], int xs,
 
 // Persistent CTAs walk the (m-tile, n-tile) grid with n fastest, so the CTAs in
 // flight share activation tiles and the whole packed weight stays in L2.
-template <int BN, bool SK>
+// PR: one gamma per output row (the per-row variant); without it that code is
+// compiled out of the epilogue.
+template <int BN, bool SK, bool PR>
 __global__ void __launch_bounds__(THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    int M, int N, int K, const float* __restrict__ gamma_p,
@@ -384,6 +406,8 @@ __global__ void __launch_bounds__(THREADS, 1)
                 if (SK && !whole) {
 #pragma unroll
                     for (int j = 0; j < 32; ++j) slot[(size_t)(c * 32 + j) * BM] = v[j];
+                } else if (PR && mv && nb < N) {
+                    store_row_per_row_gamma<32>(v, xs, scale[m], gamma_p, nb, N, static_cast<size_t>(m) * N + nb, out);
                 } else if (mv && nb < N) {
                     // row segments with their own gamma end on 32-column chunks
                     const int sgi = seg_of(out, nb);
@@ -466,7 +490,7 @@ __device__ __forceinline__ void store_row8(const uint32_t (&v)[8], int xs, float
 // cover it) and runs the epilogue. Thread (quarter qd = tid / 128, row r = tid %
 // 128) owns 8 columns of one row; the pieces are column-major, so each warp load
 // reads one 128-byte line, and every piece's loads are in flight together.
-template <int BN>
+template <int BN, bool PR>
 __global__ void __launch_bounds__(512) gemm_sk_fixup_kernel(int M, int N, int K, int G,
                                                            const uint32_t* __restrict__ partials,
                                                            const float* __restrict__ gamma_p,
@@ -500,6 +524,11 @@ __global__ void __launch_bounds__(512) gemm_sk_fixup_kernel(int M, int N, int K,
     }
     const bool vec = (N % 8 == 0) && aligned16(out.y) && aligned16(out.y32) && aligned16(out.residual) &&
                      aligned16(out.acc);
+    if (PR) {
+        store_row_per_row_gamma<8>(v, xsum[m], scale[m], gamma_p, n0 + col, N, static_cast<size_t>(m) * N + n0 + col,
+                                   out);
+        return;
+    }
     store_row8(v, xsum[m], __fdiv_rn(gamma_p[seg_of(out, n0 + col)], scale[m]), n0 + col, N,
                static_cast<size_t>(m) * N + n0 + col, out, vec);
 }
@@ -554,7 +583,7 @@ bool gemm_tc_ok(int64_t N, int64_t K, const void* Wp, const void* xq) {
 }
 
 namespace {
-template <int BN>
+template <int BN, bool PR = false>
 cudaError_t launch_bn(const uint8_t* Wp, const float* gamma, int64_t N, int64_t K, const int8_t* xq_g16t,
                       const float* scale, const int32_t* xsum, int64_t M, const GemvOut& out,
                       cudaStream_t s, int dev, int sms, uint32_t* partials) {
@@ -567,7 +596,7 @@ cudaError_t launch_bn(const uint8_t* Wp, const float* gamma, int64_t N, int64_t 
     cudaError_t e = device_error_word(&err);
     if (e != cudaSuccess) return e;
     const bool sk = partials != nullptr;
-    auto kern = sk ? gemm_tc_kernel<BN, true> : gemm_tc_kernel<BN, false>;
+    auto kern = sk ? gemm_tc_kernel<BN, true, PR> : gemm_tc_kernel<BN, false, PR>;
     static bool attr_set[64][2];
     if (dev >= 64 || !attr_set[dev][sk]) {
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -581,7 +610,7 @@ cudaError_t launch_bn(const uint8_t* Wp, const float* gamma, int64_t N, int64_t 
     kern<<<grid, THREADS, smem, s>>>(mapA, mapB, (int)M, (int)N, (int)K, gamma, scale, xsum, out, err, partials);
     e = cudaGetLastError();
     if (e != cudaSuccess || !sk) return e;
-    return launch_pdl(gemm_sk_fixup_kernel<BN>, dim3((unsigned)tiles, BN / 32), dim3(512), 0, s, (int)M, (int)N,
+    return launch_pdl(gemm_sk_fixup_kernel<BN, PR>, dim3((unsigned)tiles, BN / 32), dim3(512), 0, s, (int)M, (int)N,
                       (int)K, (int)grid, (const uint32_t*)partials, gamma, scale, xsum, out);
 }
 }  // namespace
@@ -645,7 +674,11 @@ cudaError_t launch_gemm_tc(const uint8_t* Wp, const float* gamma, int64_t N, int
         if (e != cudaSuccess) return e;
     }
     const int sms = dev < 64 ? num_sms[dev] : 148;
-    if (sk_ws && sk_ws_bytes >= gemm_sk_workspace_bytes(sms) && gemm_use_stream_k(M, N, K, sms))
+    const bool sk_ok = sk_ws && sk_ws_bytes >= gemm_sk_workspace_bytes(sms) && gemm_use_stream_k(M, N, K, sms);
+    if (out.per_row)  // the per-row gamma variant runs 256-row tiles only
+        return launch_bn<256, true>(Wp, gamma, N, K, xq_g16t, scale, xsum, M, out, s, dev, sms,
+                                    sk_ok ? static_cast<uint32_t*>(sk_ws) : nullptr);
+    if (sk_ok)
         return launch_bn<256>(Wp, gamma, N, K, xq_g16t, scale, xsum, M, out, s, dev, sms,
                               static_cast<uint32_t*>(sk_ws));
     switch (gemm_tc_tile_width(M, N, sms)) {

@@ -699,7 +699,7 @@ __global__ void __launch_bounds__(kThreads + 32, NT == 1 ? 3 : 2) gemv_mma_kerne
 #pragma unroll
                 for (int w = 0; w < kWarps; ++w) sum += red[w][r][cl];
                 const int accv = sum - xs_sh[cl];
-                const int sgi = XT ? seg_of(a.out, n) : 0;  // row segments with their own gamma
+                const int sgi = XT ? gamma_index(a.out, n) : 0;  // segments / rows with their own gamma
                 float v = dequant(accv, sgi == 0 ? deq_sh[cl] : __fdiv_rn(a.gamma[sgi], s_sh[cl]));
                 if (!store) continue;
                 const size_t o = (size_t)m * N + n;
@@ -736,7 +736,7 @@ __global__ void __launch_bounds__(kThreads) gemv_generic_kernel(
     }
     acc = warp_sum(acc);
     if (lane == 0) {
-        const float deq = __fdiv_rn(gamma_p[seg_of(out, n)], scale[m]);
+        const float deq = __fdiv_rn(gamma_p[gamma_index(out, n)], scale[m]);
         float v = dequant(acc, deq);
         const size_t o = (size_t)m * N + n;
         if (out.y32) {
@@ -851,7 +851,7 @@ cudaError_t launch_gemv(const uint8_t* Wp, const float* gamma, int64_t N, int64_
     cudaError_t e = plan_stream(a, N, K, M, 1, x_fused != nullptr, p);
     if (e != cudaSuccess) return e;
     const dim3 g1(p.grid_x, 1), g2(p.grid_x, (unsigned)((M + 15) / 16));
-    const bool xt = a.norm || out.seg_end[0] < N;
+    const bool xt = a.norm || out.seg_end[0] < N || out.per_row;
     if (xt) {
         if (x_fused) return launch_fused<SRC_X, false, true>(a, g1, p.smem, s);
         if (M <= 8) return launch_variant<1, SRC_CODES, false, false, true>(a, g1, p.smem, s);

@@ -13,7 +13,9 @@ int absmean_blocks(int64_t n);
 cudaError_t launch_absmean(const void* W, bool fp32, int64_t n, double* partial, float* gamma,
                            cudaStream_t s);
 cudaError_t launch_ternary_pack(const void* W, bool fp32, int64_t N, int64_t K, const float* gamma,
-                                uint8_t* Wp, cudaStream_t s);
+                                uint8_t* Wp, cudaStream_t s, bool per_row = false);
+// gammas[n] = fp32(sum_k |W[n, k]| / K) (per-row absmean variant)
+cudaError_t launch_absmean_rows(const void* W, bool fp32, int64_t N, int64_t K, float* gammas, cudaStream_t s);
 cudaError_t launch_count_bad_codes(const uint8_t* Wp, int64_t nbytes, unsigned long long* count,
                                    cudaStream_t s);
 
@@ -34,10 +36,16 @@ struct GemvOut {
     // uses gamma[seg_of(n)]; rows >= seg_end[i] lie past segment i. One segment by
     // default. The GEMV needs the ends on 16-row tiles, the GEMM on 32 columns.
     int seg_end[3] = {0x7fffffff, 0x7fffffff, 0x7fffffff};
+    int per_row = 0;  // one gamma per output row (gamma[n]) instead of segments
 };
 
 __host__ __device__ __forceinline__ int seg_of(const GemvOut& o, int n) {
     return (n >= o.seg_end[0]) + (n >= o.seg_end[1]) + (n >= o.seg_end[2]);
+}
+
+// index into gamma of output row n
+__host__ __device__ __forceinline__ int gamma_index(const GemvOut& o, int n) {
+    return o.per_row ? n : seg_of(o, n);
 }
 // Requires K % 256 == 0 and 16-byte aligned Wp. Codes either come as PLANES
 // layout Xp (+ scale, xsum) from the act-quant kernel, or, when x_fused is given

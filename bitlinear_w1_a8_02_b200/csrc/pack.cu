@@ -7,6 +7,8 @@
 //   gamma = fp32( sum |W| / (N*K) ), the sum and the division in fp64
 //   q     = clip(rint(W / (gamma + 1e-5)), -1, 1), one IEEE fp32 division
 //   byte j of row n = sum_i (q[n][4j+i] + 1) << 2i
+// Per-row variant: gamma_n = fp32( sum_k |W[n, k]| / K ) (fp64 sum and division),
+// and row n is ternarised with its own gamma_n.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -45,15 +47,31 @@ __global__ void absmean_final_kernel(const double* __restrict__ partial, int nbl
     if (threadIdx.x == 0) *gamma = __double2float_rn(__ddiv_rn(acc, (double)n));
 }
 
-// One packed byte (four weights) per thread.
+// Per-row absmean: one CTA per row, fp64 sum in a fixed order (thread strides,
+// warp butterfly, warps in index order).
 template <bool FP32>
+__global__ void __launch_bounds__(kPackThreads) absmean_rows_kernel(const void* __restrict__ W, int64_t K,
+                                                                    float* __restrict__ gammas) {
+    __shared__ double scratch[kPackThreads / 32];
+    const int64_t row = blockIdx.x;
+    double acc = 0.0;
+    for (int64_t k = threadIdx.x; k < K; k += kPackThreads)
+        acc = __dadd_rn(acc, fabs((double)load_w<FP32>(W, row * K + k)));
+    acc = block_sum<kPackThreads / 32>(acc, scratch);
+    if (threadIdx.x == 0) gammas[row] = __double2float_rn(__ddiv_rn(acc, (double)K));
+}
+
+// One packed byte (four weights) per thread. gamma: one value, or one per row
+// (ROWS) for row-major bytes of KB per row.
+template <bool FP32, bool ROWS>
 __global__ void __launch_bounds__(kPackThreads) ternary_pack_kernel(const void* __restrict__ W,
-                                                                    int64_t nbytes,
+                                                                    int64_t nbytes, int64_t KB,
                                                                     const float* __restrict__ gamma,
                                                                     uint8_t* __restrict__ Wp) {
-    const float d = __fadd_rn(*gamma, kWeightEps);
+    const float d0 = ROWS ? 0.0f : __fadd_rn(*gamma, kWeightEps);
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     for (int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; j < nbytes; j += stride) {
+        const float d = ROWS ? __fadd_rn(gamma[j / KB], kWeightEps) : d0;
         float w[4];
         if (FP32) {
             const float4 v = reinterpret_cast<const float4*>(W)[j];
@@ -114,13 +132,27 @@ cudaError_t launch_absmean(const void* W, bool fp32, int64_t n, double* partial,
 }
 
 cudaError_t launch_ternary_pack(const void* W, bool fp32, int64_t N, int64_t K, const float* gamma,
-                                uint8_t* Wp, cudaStream_t s) {
-    const int64_t nbytes = N * (K / 4);
+                                uint8_t* Wp, cudaStream_t s, bool per_row) {
+    const int64_t nbytes = N * (K / 4), KB = K / 4;
     const int g = grid_for(nbytes, 148 * 64);
+    if (per_row) {
+        if (fp32)
+            ternary_pack_kernel<true, true><<<g, kPackThreads, 0, s>>>(W, nbytes, KB, gamma, Wp);
+        else
+            ternary_pack_kernel<false, true><<<g, kPackThreads, 0, s>>>(W, nbytes, KB, gamma, Wp);
+    } else if (fp32) {
+        ternary_pack_kernel<true, false><<<g, kPackThreads, 0, s>>>(W, nbytes, KB, gamma, Wp);
+    } else {
+        ternary_pack_kernel<false, false><<<g, kPackThreads, 0, s>>>(W, nbytes, KB, gamma, Wp);
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_absmean_rows(const void* W, bool fp32, int64_t N, int64_t K, float* gammas, cudaStream_t s) {
     if (fp32)
-        ternary_pack_kernel<true><<<g, kPackThreads, 0, s>>>(W, nbytes, gamma, Wp);
+        absmean_rows_kernel<true><<<(unsigned)N, kPackThreads, 0, s>>>(W, K, gammas);
     else
-        ternary_pack_kernel<false><<<g, kPackThreads, 0, s>>>(W, nbytes, gamma, Wp);
+        absmean_rows_kernel<false><<<(unsigned)N, kPackThreads, 0, s>>>(W, K, gammas);
     return cudaGetLastError();
 }
 

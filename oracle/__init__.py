@@ -63,6 +63,8 @@ def _l():
             "orc_relu2_gate": (F, [F, F]),
             "orc_ffn_layer": (ctypes.c_int, [P, F, P, F, P, F, I, I, P, I, P, P, P, P, P, P, P]),
             "orc_forward_ex": (ctypes.c_int, [P, P, P, I, I, P, I, I, P, P, P]),
+            "orc_pack_weights_rowwise": (ctypes.c_int, [P, I, I, P, P]),
+            "orc_forward_rowwise": (ctypes.c_int, [P, P, I, I, P, I, P, P, P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(lib, name)
@@ -237,6 +239,35 @@ def forward_ex(Wp: np.ndarray, gammas, seg_rows, x_bf16: np.ndarray, rmsnorm=Fal
                              _p(y), _p(acc))
     if rc != 0:
         raise MemoryError("oracle forward_ex failed")
+    return dict(y=y, acc=acc)
+
+
+def pack_weights_rowwise(W: np.ndarray):
+    """Per-row absmean variant: W [N, K] (fp32, or bf16 bits) -> (Wp uint8 [N, K/4], gammas fp32 [N])."""
+    if W.dtype == np.uint16:
+        W = bf16_to_f32(W)
+    W = _c(W, np.float32)
+    N, K = W.shape
+    Wp = np.empty((N, K // 4), np.uint8)
+    g = np.empty(N, np.float32)
+    if _l().orc_pack_weights_rowwise(_p(W), N, K, _p(Wp), _p(g)) != 0:
+        raise MemoryError("oracle pack_weights_rowwise failed")
+    return Wp, g
+
+
+def forward_rowwise(Wp: np.ndarray, gammas: np.ndarray, x_bf16: np.ndarray, residual=None):
+    """Forward with one gamma per output row. Returns dict(y, acc); y as bf16 bits."""
+    Wp = _c(Wp, np.uint8)
+    x = _c(x_bf16, np.uint16)
+    g = _c(np.asarray(gammas, np.float32), np.float32)
+    N = Wp.shape[0]
+    M, K = x.shape
+    assert Wp.shape[1] * 4 == K and g.size == N
+    res = None if residual is None else _c(residual, np.uint16)
+    y = np.empty((M, N), np.uint16)
+    acc = np.empty((M, N), np.int32)
+    if _l().orc_forward_rowwise(_p(Wp), _p(g), N, K, _p(x), M, _p(res), _p(y), _p(acc)) != 0:
+        raise MemoryError("oracle forward_rowwise failed")
     return dict(y=y, acc=acc)
 
 

@@ -374,3 +374,51 @@ done:
     free(xf); free(xn); free(xq); free(s); free(acc);
     return rc;
 }
+
+/* ------------------------------------------------------------------------- */
+/* Per-row absmean variant of the weight path (one gamma per output row instead
+ * of one per tensor; the pages give absmean per weight tensor, [card] "Method
+ * Adaptation", so this is a variant of that reading): gamma_n = mean_k |W[n,k]|
+ * (fp64 sum in k order, fp64 division by K, one rounding to fp32), row n
+ * ternarised with its own gamma_n, then packed as usual.                      */
+int orc_pack_weights_rowwise(const float* W, int64_t N, int64_t K, uint8_t* Wp, float* gammas) {
+    int8_t* q = (int8_t*)malloc((size_t)(N * K));
+    if (!q) return -1;
+    for (int64_t n = 0; n < N; ++n) {
+        gammas[n] = orc_absmean(W + n * K, K);
+        orc_ternarize(W + n * K, K, gammas[n], q + n * K);
+    }
+    orc_pack(q, N, K, Wp);
+    free(q);
+    return 0;
+}
+
+/* Forward with per-row gammas: y[m, n] = bf16([res +] float(acc) * (gamma_n / s_m)). */
+int orc_forward_rowwise(const uint8_t* Wp, const float* gammas, int64_t N, int64_t K,
+                        const uint16_t* x, int64_t M, const uint16_t* residual,
+                        uint16_t* y, int32_t* acc_out) {
+    float* xf = (float*)malloc(sizeof(float) * (size_t)(M * K));
+    int8_t* xq = (int8_t*)malloc((size_t)(M * K));
+    float* s = (float*)malloc(sizeof(float) * (size_t)M);
+    int32_t* acc = (int32_t*)malloc(sizeof(int32_t) * (size_t)(M * N));
+    int rc = 0;
+    if (!xf || !xq || !s || !acc) {
+        rc = -1;
+        goto done;
+    }
+    orc_bf16_to_f32_array(x, M * K, xf);
+    orc_quant_act(xf, M, K, xq, s, NULL);
+    orc_int_gemm_packed(Wp, xq, M, N, K, acc);
+    for (int64_t m = 0; m < M; ++m) {
+        for (int64_t n = 0; n < N; ++n) {
+            float deq = gammas[n] / s[m];
+            float v = (float)acc[m * N + n] * deq;
+            if (residual) v = orc_bf16_to_f32(residual[m * N + n]) + v;
+            y[m * N + n] = orc_f32_to_bf16(v);
+        }
+    }
+    if (acc_out) memcpy(acc_out, acc, sizeof(int32_t) * (size_t)(M * N));
+done:
+    free(xf); free(xq); free(s); free(acc);
+    return rc;
+}

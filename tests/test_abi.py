@@ -152,6 +152,23 @@ def test_host_validation_forward_ex():
     assert call([48, 16, 32], wsb=need - 1) == WS
 
 
+def test_host_validation_rowwise():
+    L = bl.lib()
+    pk = L.bitlinear_pack_weights_rowwise
+    assert pk(P(A), 7, 8, 16, P(A), P(A), None) == DTYPE
+    assert pk(P(A), bl.BL_BF16, 8, 18, P(A), P(A), None) == SHAPE
+    assert pk(P(A), bl.BL_BF16, 0, 16, P(A), P(A), None) == SHAPE
+    assert pk(P(A), bl.BL_BF16, 8, 16, P(A), None, None) == NULL
+    assert pk(P(A + 8), bl.BL_BF16, 8, 16, P(A), P(A), None) == ALIGN
+    F = L.bitlinear_forward_rowwise
+    need = L.bitlinear_workspace_bytes(bl.BL_OP_FORWARD, 1, 512, 256)
+    assert F(P(A), P(A), 512, 258, P(A), 1, None, P(A), None, P(A), need, None) == SHAPE
+    assert F(P(A), P(A), 512, 256, P(A), 0, None, P(A), None, P(A), need, None) == OK
+    assert F(P(A), None, 512, 256, P(A), 1, None, P(A), None, P(A), need, None) == NULL
+    assert F(P(A), P(A + 2), 512, 256, P(A), 1, None, P(A), None, P(A), need, None) == ALIGN
+    assert F(P(A), P(A), 512, 256, P(A), 1, None, P(A), None, P(A), need - 1, None) == WS
+
+
 def test_host_validation_selftest():
     L = bl.lib()
     assert L.bitlinear_selftest_timeout(0, None) == SHAPE

@@ -232,6 +232,32 @@ def test_forward_ex_unaligned_segments_take_the_generic_kernel(cuda_device, M):
     assert_bf16_exact(bits(y), ref["y"])
 
 
+@pytest.mark.parametrize("N,K,dtype", [(2560, 2560, "bf16"), (640, 2560, "bf16"), (512, 256, "fp32"),
+                                       (3, 12, "bf16"), (136, 196, "fp32")])
+def test_pack_rowwise_parity(cuda_device, N, K, dtype):
+    W = make_weights(N, K, 0.02, seed=N + K, dtype=dtype)
+    Wp, g = bl.pack_weights_rowwise(W.to(cuda_device))
+    Wp_ref, g_ref = oracle.pack_weights_rowwise(bits(W) if dtype == "bf16" else np_(W))
+    assert np.array_equal(np_(g).view(np.uint32), g_ref.view(np.uint32)), "per-row gamma bits"
+    assert np.array_equal(np_(Wp), Wp_ref), "packed bytes"
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 6912, 2560), (1, 2560, 6912), (4, 640, 2560), (9, 2560, 2560),
+                                   (64, 2400, 2560), (300, 640, 4096), (20, 100, 1024), (5, 33, 260)])
+def test_forward_rowwise_parity(cuda_device, M, N, K):
+    """One gamma per output row: the single-token dp4a GEMV, the fused and unfused
+    multi-token GEMV, the tensor-core GEMM (also with split tiles) and the generic kernel."""
+    W = make_weights(N, K, 0.02, seed=3 * N + K)
+    Wp, g = bl.pack_weights_rowwise(W.to(cuda_device))
+    Wp_ref, g_ref = oracle.pack_weights_rowwise(bits(W))
+    x = synth.activations(M, K, seed=M + 5, outliers=True)
+    res = synth.activations(M, N, seed=M + 6, outliers=False)
+    y, acc = bl.forward_rowwise(Wp, g, x.to(cuda_device), residual=res.to(cuda_device), want_acc=True)
+    ref = oracle.forward_rowwise(Wp_ref, g_ref, bits(x), residual=bits(res))
+    assert np.array_equal(np_(acc), ref["acc"]), "int32 accumulators"
+    assert_bf16_exact(bits(y), ref["y"])
+
+
 def test_forward_misaligned_input_takes_generic_path(cuda_device):
     K, N, M = 256, 64, 20
     W = make_weights(N, K, 0.02, seed=21)

@@ -365,3 +365,47 @@ def test_forward_ex_rmsnorm_only_rescales_the_codes():
     normed = oracle.forward_ex(Wp, [gamma], [N], x, rmsnorm=True)
     diff = np.abs(plain["acc"].astype(np.int64) - normed["acc"].astype(np.int64))
     assert np.mean(diff != 0) < 0.05 and np.all(diff <= 3 * 2)
+
+
+# ----------------------------------------------------------------------------- per-row gamma variant
+
+def test_rowwise_worked_2x4():
+    g = json.load(open(os.path.join(GOLDEN, "rowwise_2x4.json")))
+    W = np.array(g["W"], np.float32)
+    Wp, gam = oracle.pack_weights_rowwise(W)
+    assert gam.tolist() == g["gammas"]
+    q, bad = oracle.unpack(Wp, 4)
+    assert bad == 0 and q.tolist() == g["q"]
+    assert Wp.tolist() == g["packed"]
+    Wp_t, gam_t = oracle.pack_weights(W)
+    assert float(gam_t) == g["per_tensor_gamma"]
+    assert oracle.unpack(Wp_t, 4)[0][1].tolist() == g["per_tensor_q_row1"]
+
+
+def test_rowwise_single_row_is_per_tensor():
+    W = bf16_bits(synth.weights(1, 2560, 0.02, 61))
+    Wp_r, g_r = oracle.pack_weights_rowwise(W)
+    Wp_t, g_t = oracle.pack_weights(W)
+    assert np.array_equal(Wp_r, Wp_t) and g_r[0] == g_t
+
+
+def test_rowwise_power_of_two_row_scales():
+    # row n = 2^(n-3) * base: every row's gamma scales exactly and its codes equal the base row's
+    base = synth.weights(1, 512, 0.02, 62).float().numpy()[0]
+    W = np.stack([base * np.float32(2.0 ** (n - 3)) for n in range(8)]).astype(np.float32)
+    Wp, g = oracle.pack_weights_rowwise(W)
+    for n in range(8):
+        assert g[n] == np.float32(g[3] * np.float32(2.0 ** (n - 3)))
+    q, _ = oracle.unpack(Wp, 512)
+    # eps = 1e-5 in d = gamma + eps shifts the boundaries by ~1e-5 / gamma: allow rare flips
+    assert np.mean(q != q[3]) < 1e-3
+
+
+def test_forward_rowwise_with_equal_gammas_is_forward():
+    K, N, M = 256, 48, 3
+    Wp, gamma = oracle.pack_weights(bf16_bits(synth.weights(N, K, 0.02, 63)))
+    x = bf16_bits(synth.activations(M, K, seed=64, outliers=True))
+    res = bf16_bits(synth.activations(M, N, seed=65, outliers=False))
+    a = oracle.forward_rowwise(Wp, np.full(N, gamma, np.float32), x, residual=res)
+    b = oracle.forward(Wp, gamma, x, residual=res)
+    assert np.array_equal(a["acc"], b["acc"]) and np.array_equal(a["y"], b["y"])
