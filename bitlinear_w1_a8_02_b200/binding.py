@@ -36,7 +36,7 @@ SIGNATURES = {
     "bitlinear_pack_weights": (_ST, [_P, ctypes.c_int, _I, _I, _P, _P, _P, _S, _P]),
     "bitlinear_quant_act": (_ST, [_P, _I, _I, _P, _P, _P, _P]),
     "bitlinear_forward": (_ST, [_P, _P, _I, _I, _P, _I, _P, _P, _P, _P, _S, _P]),
-    "bitlinear_pack_weights_rowwise": (_ST, [_P, ctypes.c_int32, _I, _I, _P, _P, _P]),
+    "bitlinear_pack_weights_rowwise": (_ST, [_P, ctypes.c_int, _I, _I, _P, _P, _P]),
     "bitlinear_forward_rowwise": (_ST, [_P, _P, _I, _I, _P, _I, _P, _P, _P, _P, _S, _P]),
     "bitlinear_forward_ex": (_ST, [_P, _P, _P, ctypes.c_int32, _I, _P, _I, ctypes.c_int32, _P, _P, _P, _P, _S,
                                    _P]),

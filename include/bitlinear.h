@@ -143,6 +143,30 @@ bl_status bitlinear_forward(const uint8_t* Wp, const float* gamma, int64_t N, in
                             void* ws, size_t ws_bytes, bl_stream_t stream);
 
 /*
+ * Per-row absmean variant of bitlinear_pack_weights: one gamma per output row
+ * instead of one per tensor (the pages give absmean per weight tensor, paper
+ * card "BitNet b1.58 2B4T Technical Report", "Method Adaptation"; this is the
+ * finer-grained variant of that reading):
+ *   gammas[n] = fp32( sum_k |W[n, k]| / K )     sum and division in fp64
+ *   q[n, k]   = clip(rint(W[n, k] / (gammas[n] + 1e-5)), -1, 1)
+ * and the same packed layout. Arguments as bitlinear_pack_weights, with
+ * gammas [N] device fp32 (4-byte aligned) in place of gamma; no workspace.
+ */
+bl_status bitlinear_pack_weights_rowwise(const void* W, int wdt, int64_t N, int64_t K,
+                                         uint8_t* Wp, float* gammas, bl_stream_t stream);
+
+/*
+ * bitlinear_forward with the per-row gammas of bitlinear_pack_weights_rowwise:
+ *   y[m, n] = bf16([residual[m, n] +] float(acc[m, n]) * (gammas[n] / s_m))
+ * Arguments, kernel choice and errors as bitlinear_forward, with gammas [N]
+ * device fp32 in place of gamma; the same workspace.
+ */
+bl_status bitlinear_forward_rowwise(const uint8_t* Wp, const float* gammas, int64_t N, int64_t K,
+                                    const uint16_t* x, int64_t M, const uint16_t* residual,
+                                    uint16_t* y, int32_t* acc,
+                                    void* ws, size_t ws_bytes, bl_stream_t stream);
+
+/*
  * Several BitLinear projections of one input in one call, optionally after a
  * unit-weight RMSNorm of the input: the attention side of a BitNet b1.58 block
  * (paper card "BitNet b1.58 2B4T Technical Report", "Method Adaptation":
@@ -170,30 +194,6 @@ bl_status bitlinear_forward(const uint8_t* Wp, const float* gamma, int64_t N, in
  * 1..4, rmsnorm not 0 or 1, a segment without rows, or the bitlinear_forward
  * shape rules on N = sum of seg_rows; otherwise as bitlinear_forward.
  */
-/*
- * Per-row absmean variant of bitlinear_pack_weights: one gamma per output row
- * instead of one per tensor (the pages give absmean per weight tensor, paper
- * card "BitNet b1.58 2B4T Technical Report", "Method Adaptation"; this is the
- * finer-grained variant of that reading):
- *   gammas[n] = fp32( sum_k |W[n, k]| / K )     sum and division in fp64
- *   q[n, k]   = clip(rint(W[n, k] / (gammas[n] + 1e-5)), -1, 1)
- * and the same packed layout. Arguments as bitlinear_pack_weights, with
- * gammas [N] device fp32 (4-byte aligned) in place of gamma; no workspace.
- */
-bl_status bitlinear_pack_weights_rowwise(const void* W, int32_t wdt, int64_t N, int64_t K,
-                                         uint8_t* Wp, float* gammas, bl_stream_t stream);
-
-/*
- * bitlinear_forward with the per-row gammas of bitlinear_pack_weights_rowwise:
- *   y[m, n] = bf16([residual[m, n] +] float(acc[m, n]) * (gammas[n] / s_m))
- * Arguments, kernel choice and errors as bitlinear_forward, with gammas [N]
- * device fp32 in place of gamma; the same workspace.
- */
-bl_status bitlinear_forward_rowwise(const uint8_t* Wp, const float* gammas, int64_t N, int64_t K,
-                                    const uint16_t* x, int64_t M, const uint16_t* residual,
-                                    uint16_t* y, int32_t* acc,
-                                    void* ws, size_t ws_bytes, bl_stream_t stream);
-
 bl_status bitlinear_forward_ex(const uint8_t* Wp, const float* gammas, const int64_t* seg_rows,
                                int32_t nseg, int64_t K, const uint16_t* x, int64_t M,
                                int32_t rmsnorm, const uint16_t* residual, uint16_t* y,
