@@ -64,6 +64,28 @@ def dist_env():
             int(os.environ.get("LOCAL_RANK", 0)))
 
 
+def rank_ops(torch, dist, world: int, device):
+    """Barrier and max-over-ranks of a float, the two collectives the timing
+    uses (NCCL on the GPUs; the same code runs under gloo on the CPU in tests)."""
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(v: float) -> float:
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+    return barrier, max_over_ranks
+
+
+def whole_job_gbs(world: int, step_bytes: int, steps: int, ms_total: float) -> float:
+    """Aggregate throughput: every rank streams step_bytes per step (weak
+    scaling); the time is the slowest rank's."""
+    return world * step_bytes * steps / (ms_total * 1e-3) / 1e9
+
+
 # ----------------------------------------------------------------------------- clocks
 
 class ClockSampler:
@@ -139,16 +161,7 @@ def run_ours(args):
     int8_peak = float(peaks["bf16_tflops"]) * INT8_PER_BF16
     int8_peak_sust = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])) * INT8_PER_BF16
 
-    def barrier():
-        if world > 1:
-            dist.barrier()
-
-    def max_over_ranks(v: float) -> float:
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    barrier, max_over_ranks = rank_ops(torch, dist, world, dev)
 
     # ---- decode weights: 30 copies of each of the four shapes, packed on device
     weights = []  # weights[layer][shape] = (Wp, gamma)
@@ -204,7 +217,7 @@ def run_ours(args):
     clk = clocks.stop()
     ms_total = max_over_ranks(ev0.elapsed_time(ev1))
     ms_step = ms_total / args.steps
-    value = world * step_bytes * args.steps / (ms_total * 1e-3) / 1e9
+    value = whole_job_gbs(world, step_bytes, args.steps, ms_total)
 
     # ---- dominant kernel: the decode GEMV. At M = 1 each forward call is one
     # kernel (quantisation fused); consecutive calls overlap through programmatic
