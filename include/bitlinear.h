@@ -26,9 +26,10 @@
  *   - No C++ exception crosses this boundary. A failed launch returns BL_ERR_CUDA.
  *   - Calls on different streams may overlap only if their workspaces differ.
  *
- * Packed weight format (this library's reading; the pages only say "four ternary
- * weights in one 8-bit value"): Wp is [N, K/4] uint8, row-major. Byte j of row n
- * holds weights k = 4j .. 4j+3; weight 4j+i is stored in bits 2i..2i+1 as the
+ * Packed weight format (this library's reading; the paper card, "Method
+ * Adaptation", only fixes four ternary weights per 8-bit value): Wp is [N, K/4]
+ * uint8, row-major. Byte j of row n holds weights k = 4j .. 4j+3; weight 4j+i
+ * is stored in bits 2i..2i+1 as the
  * code q+1 in {0, 1, 2} (q in {-1, 0, +1}). Code 3 is invalid.
  *
  * Arithmetic (every step is one IEEE fp32 operation, round to nearest even, with
@@ -144,8 +145,8 @@ bl_status bitlinear_forward(const uint8_t* Wp, const float* gamma, int64_t N, in
 
 /*
  * Per-row absmean variant of bitlinear_pack_weights: one gamma per output row
- * instead of one per tensor (the pages give absmean per weight tensor, paper
- * card "BitNet b1.58 2B4T Technical Report", "Method Adaptation"; this is the
+ * instead of one per tensor (the paper card "BitNet b1.58 2B4T Technical
+ * Report", "Method Adaptation", gives one absmean per weight tensor; this is the
  * finer-grained variant of that reading):
  *   gammas[n] = fp32( sum_k |W[n, k]| / K )     sum and division in fp64
  *   q[n, k]   = clip(rint(W[n, k] / (gammas[n] + 1e-5)), -1, 1)
@@ -264,7 +265,7 @@ bl_status bitlinear_validate_packed(const uint8_t* Wp, int64_t N, int64_t K, int
 bl_status bitlinear_get_device_error(bl_stream_t stream);
 
 /*
- * Self-test of the failure path (the pages have no counterpart; it exists to
+ * Self-test of the failure path (no counterpart in the method; it exists to
  * test this library's error reporting). Launches, on `stream`, one thread that
  * waits with the library's bounded mbarrier wait on a barrier nothing arrives
  * on; after limit_us microseconds (1 .. 2,000,000) the wait gives up, records a

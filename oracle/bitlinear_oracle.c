@@ -18,7 +18,7 @@
  *           "core innovations of the architecture".
  *   [wiki]  wikiprompt "1.58-bit large language model", introduction.
  *
- * Readings where the pages are silent (every one is listed with its reason in the
+ * Readings where the sources above are silent (every one is listed with its reason in the
  * design notes of the repository):
  *   - gamma is one scalar per weight tensor: gamma = mean |W|, summed in fp64 in
  *     row-major order, divided in fp64 by N*K and rounded once to fp32.
@@ -377,8 +377,8 @@ done:
 
 /* ------------------------------------------------------------------------- */
 /* Per-row absmean variant of the weight path (one gamma per output row instead
- * of one per tensor; the pages give absmean per weight tensor, [card] "Method
- * Adaptation", so this is a variant of that reading): gamma_n = mean_k |W[n,k]|
+ * of one per tensor; [card] "Method Adaptation" gives one absmean per weight
+ * tensor, so this is a variant of that reading): gamma_n = mean_k |W[n,k]|
  * (fp64 sum in k order, fp64 division by K, one rounding to fp32), row n
  * ternarised with its own gamma_n, then packed as usual.                      */
 int orc_pack_weights_rowwise(const float* W, int64_t N, int64_t K, uint8_t* Wp, float* gammas) {
