@@ -29,8 +29,8 @@
  * Packed weight format (this library's reading; the paper card, "Method
  * Adaptation", only fixes four ternary weights per 8-bit value): Wp is [N, K/4]
  * uint8, row-major. Byte j of row n holds weights k = 4j .. 4j+3; weight 4j+i
- * is stored in bits 2i..2i+1 as the
- * code q+1 in {0, 1, 2} (q in {-1, 0, +1}). Code 3 is invalid.
+ * is stored in bits 2i..2i+1 as the code q+1 in {0, 1, 2} (q in {-1, 0, +1}).
+ * Code 3 is invalid.
  *
  * Arithmetic (every step is one IEEE fp32 operation, round to nearest even, with
  * no fused multiply-add, unless noted):
