@@ -258,6 +258,30 @@ def test_forward_rowwise_parity(cuda_device, M, N, K):
     assert_bf16_exact(bits(y), ref["y"])
 
 
+def test_forward_largest_k_extreme_codes(cuda_device):
+    """K at its documented maximum (262144) with every weight +1 and every code
+    127: the field-scaled int32 accumulators of the streamed GEMV reach their
+    largest values (128 * 127 * K / 4 < 2^31) and acc = 127 K exactly."""
+    K, N, M = 262144, 17, 1
+    W = torch.ones((N, K), dtype=torch.bfloat16)
+    Wp, gamma, Wp_ref, g_ref = pack_both(W, cuda_device)
+    x = torch.ones((M, K), dtype=torch.bfloat16)
+    y, acc = bl.forward(Wp, gamma, x.to(cuda_device), want_acc=True)
+    assert np.all(np_(acc) == 127 * K)
+    ref = oracle.forward(Wp_ref, g_ref, bits(x))
+    assert np.array_equal(np_(acc), ref["acc"])
+    assert_bf16_exact(bits(y), ref["y"])
+
+
+def test_forward_largest_m(cuda_device):
+    """M at its documented maximum (65535 tokens) on the tensor-core path."""
+    M, N, K = 65535, 16, 64
+    W = make_weights(N, K, 0.02, seed=97)
+    Wp, gamma, Wp_ref, g_ref = pack_both(W, cuda_device)
+    x = synth.activations(M, K, seed=98, outliers=True)
+    check_forward_full(Wp, gamma, Wp_ref, g_ref, x, cuda_device)
+
+
 def test_forward_misaligned_input_takes_generic_path(cuda_device):
     K, N, M = 256, 64, 20
     W = make_weights(N, K, 0.02, seed=21)
