@@ -26,8 +26,11 @@ inline bool aligned(const void* p, size_t a) { return (uintptr_t)p % a == 0; }
 
 // Workspace carving -----------------------------------------------------------
 // Tensor-core projections (M > 16) may split tiles across CTAs (stream-K) and
-// need scratch for the pieces; the smaller paths do not.
-inline size_t sk_bytes(int64_t M) { return M > 16 ? align_up(bl::gemm_sk_workspace_bytes(bl::device_sm_count())) : 0; }
+// need scratch for the pieces; the smaller paths do not. Sized for 148 SMs
+// without asking the device (workspace sizes are host-only arithmetic); a device
+// with more SMs finds the scratch too small and keeps the data-parallel split.
+constexpr int kStreamKSms = 148;
+inline size_t sk_bytes(int64_t M) { return M > 16 ? align_up(bl::gemm_sk_workspace_bytes(kStreamKSms)) : 0; }
 
 struct ForwardWs {
     size_t xq, scale, xsum, sk, sk_bytes, total;

@@ -638,15 +638,6 @@ int gemm_tc_tile_width(int64_t M, int64_t N, int sms) {
 
 size_t gemm_sk_workspace_bytes(int sms) { return (size_t)2 * sms * BM * 256 * sizeof(uint32_t); }
 
-int device_sm_count() {
-    int dev = 0, n = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
-        cudaGetLastError();
-        return 148;
-    }
-    return n;
-}
 
 // Stream-K only where the data-parallel plan leaves much of its last wave idle
 // (under 70% of its CTA-slots busy) and the tiles are long in K (at least 32

@@ -85,7 +85,6 @@ cudaError_t launch_gemm_tc(const uint8_t* Wp, const float* gamma, int64_t N, int
                            const int8_t* xq_g16t, const float* scale, const int32_t* xsum, int64_t M,
                            const GemvOut& out, cudaStream_t s, void* sk_ws = nullptr, size_t sk_ws_bytes = 0);
 size_t gemm_sk_workspace_bytes(int sms);
-int device_sm_count();  // SMs of the current device (148 when it cannot be read)
 
 // ---- FFN glue (ffn.cu)
 // h = relu(g)^2 * u; hn = subln(h); q2, s2, xsum2 = quant(hn) in `layout`.
