@@ -23,10 +23,20 @@
 // fused. Before the dependency wait each CTA asks for its first tiles to be
 // prefetched into L2, so DRAM already streams while the previous kernel ends.
 //
-// Fused activation quantisation: when the codes of all M tokens fit in shared
-// memory, each CTA quantises x itself (absmax per token, then PLANES codes into
-// shared memory), so a forward call is one kernel. Otherwise the codes come from
-// the act-quant kernel through the workspace.
+// Single token (DP): an 8-column MMA would spend 7 columns on padding, so each
+// thread instead owns 4 rows of the unit and every 64th packed word, and runs one
+// dp4a per 2-bit field against the token's plane words, which the quantiser
+// stores interleaved (the four plane words of a 16-code group side by side).
+//
+// Fused activation quantisation: when the codes of all M (<= 4) tokens fit in
+// shared memory, each CTA quantises x itself (absmax per token, then PLANES codes
+// into shared memory), so a forward call is one kernel. Otherwise the codes come
+// from the act-quant kernel through the workspace.
+//
+// Extended calls (XT): row segments with their own gamma (stacked projections),
+// one gamma per row, and a unit-weight RMSNorm of x before the quantisation are
+// compiled into separate instantiations; the plain forward's code stays as small
+// as before (its prologue runs once per launch from a cold instruction cache).
 //
 // Programmatic dependent launch: before waiting for the previous kernel in the
 // stream (griddepcontrol.wait) a CTA only issues L2 prefetches of its weights,
