@@ -59,6 +59,12 @@ def test_workspace_sizes():
     assert f(bl.BL_OP_FORWARD, -1, 1, 4) == 0
     for op in (bl.BL_OP_FORWARD, bl.BL_OP_FFN):
         assert f(op, 1, 2560, 2560) % 256 == 0
+    # tensor-core calls (M > 16) carry the stream-K scratch: two 128 x 256 int32
+    # slots per SM, sized for 148 SMs without asking a device
+    sk = 2 * 148 * 128 * 256 * 4
+    assert f(bl.BL_OP_FORWARD, 17, 2560, 2560) >= 17 * 2560 + sk
+    assert f(bl.BL_OP_FFN, 17, 6912, 2560) >= sk
+    assert f(bl.BL_OP_FORWARD, 16, 2560, 2560) < sk
 
 
 # Fake, never-dereferenced addresses: every call below must fail host-side
