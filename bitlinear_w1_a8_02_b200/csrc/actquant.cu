@@ -13,9 +13,11 @@
 //
 // Optional unit-weight RMSNorm in front (the transformer block's pre-norm and
 // the subln before the attention output projection; paper card "Method
-// Adaptation": subln): pass 1 also sums x^2 in fp64 (the squares of bf16 values
-// are exact in fp64 and so, for any realistic range, is their sum, whatever the
-// order), r = 1 / sqrtf(float(sum / K) + 1e-5), and the codes are those of
+// Adaptation": subln): pass 1 also sums x^2 in fp64 (each square of a bf16 value
+// is exact in fp64, but with outlier channels the squares span more than 53 bits,
+// so the sum depends on the order in its last bits; the fp32 r below differs from
+// a sequential sum's only if the two fp64 sums straddle an fp32 rounding
+// boundary), r = 1 / sqrtf(float(sum / K) + 1e-5), and the codes are those of
 // fl(x * r) with s = 127 / max(fl(max |x| * r), 1e-5) (rounding is monotonic,
 // so max |fl(x r)| = fl(max |x| r)).
 #include "common.cuh"

@@ -409,3 +409,33 @@ def test_forward_rowwise_with_equal_gammas_is_forward():
     a = oracle.forward_rowwise(Wp, np.full(N, gamma, np.float32), x, residual=res)
     b = oracle.forward(Wp, gamma, x, residual=res)
     assert np.array_equal(a["acc"], b["acc"]) and np.array_equal(a["y"], b["y"])
+
+
+def test_forward_rowwise_worked_2x4():
+    # Hand-derived two-token forward over the per-row golden weights: the two rows
+    # have different gammas and the two tokens different scales, so taking the
+    # token's index for the row's gamma, or one gamma for every row, fails here.
+    g = json.load(open(os.path.join(GOLDEN, "rowwise_2x4.json")))
+    fw = g["forward"]
+    Wp = np.array(g["packed"], np.uint8)
+    gammas = np.array(g["gammas"], np.float32)
+    x = bf16_bits(torch.tensor(fw["x"], dtype=torch.float32).to(torch.bfloat16))
+    xq, s, xs = oracle.quant_act(x)
+    assert xq.tolist() == fw["xq"] and s.tolist() == fw["s"] and xs.tolist() == fw["xsum"]
+    # the dequantisation the variant defines, per output element
+    y32 = np.array(fw["y32"], np.float32)
+    for m in range(2):
+        for n in range(2):
+            assert np.float32(fw["acc"][m][n]) * (gammas[n] / s[m]) == y32[m, n]
+    out = oracle.forward_rowwise(Wp, gammas, x)
+    assert out["acc"].tolist() == fw["acc"]
+    want = bf16_bits(torch.tensor(fw["y"], dtype=torch.float32).to(torch.bfloat16))
+    assert np.array_equal(out["y"], want)
+    assert np.array_equal(want, bf16_bits(torch.from_numpy(y32).to(torch.bfloat16)))
+    res = bf16_bits(torch.tensor(fw["residual"], dtype=torch.float32).to(torch.bfloat16))
+    out_r = oracle.forward_rowwise(Wp, gammas, x, residual=res)
+    want_r = bf16_bits(torch.tensor(fw["y_residual"], dtype=torch.float32).to(torch.bfloat16))
+    assert np.array_equal(out_r["y"], want_r)
+    # neither the per-tensor path nor a transposed gamma choice reproduces it
+    for wrong in (np.full(2, gammas[0], np.float32), gammas[::-1].copy()):
+        assert not np.array_equal(oracle.forward_rowwise(Wp, wrong, x)["y"], want)
