@@ -10,11 +10,15 @@ no L2 flush is needed). Each call quantises the token per absmax, runs the
 ternary GEMV and dequantises to bf16. The step is captured once in a CUDA graph
 and replayed.
 
-Extras on the same line: batched decode (M = 4, 8, 16), prefill int8 TOPS
-(M = 512, 2048, 4096), the 100B-class bandwidth case, the 30-layer FFN chain,
-every BitLinear of 30 decoder layers at one token (Q/K/V with the pre-norm, the
-output projection with its subln, the FFN), the roofline of the dominant kernel, the end-to-end number through the public
-API with host buffers, the CPU oracle baseline and the SM clocks.
+Extras on the same line: batched decode (M = 4, 8, 16) and the 100B-class
+shapes at M = 1 and 16, each rotating ceil(3 x L2 / matrix bytes) weight copies
+so every call reads its weights from DRAM; prefill int8 TOPS (M = 512, 2048,
+4096 at the 2B shapes, M = 2048 at the 100B-class shapes) against the int8 peak
+measured here with torch._int_mm; the 30-layer FFN chain; every BitLinear of 30
+decoder layers at one token (Q/K/V with the pre-norm, the output projection with
+its subln, the FFN) beside the pages' whole-model CPU figure; the roofline of the
+dominant kernel; the end-to-end number through the public API with host buffers;
+the CPU oracle on all host cores and on one thread; and the SM clocks.
 
 Multi-GPU: one process per GPU (torchrun); every rank runs the same independent
 decode step on its own weights (weak scaling, no data-path collective); the
@@ -47,8 +51,49 @@ LAYERS = 30
 # per launch on average (x 1.011). Set to None whenever the kernel changes until
 # a new capture is taken.
 GEMV_TRAFFIC_PER_LAUNCH = 2753472
+# The pages' only latency figure, quoted beside the whole-decoder-layer number as
+# context (not a target): whole-model CPU decode, ms per output token.
+PAGES_CPU_MS_PER_TOKEN = 29.0
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 INT8_PER_BF16 = 2.0  # nominal dense int8 (= fp8) rate over dense bf16 on B200
+
+
+def measure_int8_peak(torch, dev, sustained_s: float = 3.0):
+    """Dense int8 tensor throughput of this GPU as cuBLASLt gives it: torch._int_mm
+    at 8192^3 (2 N^3 ops), best of 10 single calls (burst) and back to back for
+    `sustained_s` seconds (sustained). None if the call is unavailable."""
+    n = 8192
+    try:
+        a = torch.randint(-127, 128, (n, n), dtype=torch.int8, device=dev)
+        b = torch.randint(-127, 128, (n, n), dtype=torch.int8, device=dev).t().contiguous().t()
+        torch._int_mm(a, b)
+        torch.cuda.synchronize()
+    except (RuntimeError, AttributeError) as e:
+        return {"available": False, "why": str(e).splitlines()[0][:200]}
+    ops = 2.0 * n ** 3
+    best = float("inf")
+    for _ in range(10):
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        torch._int_mm(a, b)
+        e1.record()
+        torch.cuda.synchronize()
+        best = min(best, e0.elapsed_time(e1))
+    reps = max(1, int(sustained_s / (best * 1e-3)))
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        torch._int_mm(a, b)
+    e1.record()
+    torch.cuda.synchronize()
+    sust_ms = e0.elapsed_time(e1) / reps
+    del a, b
+    torch.cuda.empty_cache()
+    return {"available": True, "burst_tops": round(ops / (best * 1e-3) / 1e12, 1),
+            "sustained_tops": round(ops / (sust_ms * 1e-3) / 1e12, 1), "n": n, "reps_sustained": reps,
+            "how": "torch._int_mm int8 x int8 -> int32, 8192^3: best of 10 (burst); back to back (sustained)"}
 
 
 def load_peaks():
@@ -158,8 +203,16 @@ def run_ours(args):
                                 device_id=dev)
     peaks, peak_kind = load_peaks()
     hbm_peak = float(peaks["hbm_gbs"])
-    int8_peak = float(peaks["bf16_tflops"]) * INT8_PER_BF16
-    int8_peak_sust = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])) * INT8_PER_BF16
+    int8_from_bf16 = float(peaks["bf16_tflops"]) * INT8_PER_BF16
+    int8_from_bf16_sust = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])) * INT8_PER_BF16
+    int8_meas = measure_int8_peak(torch, dev) if (rank == 0 and not args.no_extras) else {"available": False,
+                                                                                           "why": "not measured"}
+    if int8_meas.get("available"):
+        int8_peak, int8_peak_sust = int8_meas["burst_tops"], int8_meas["sustained_tops"]
+        int8_kind = "measured on this GPU (torch._int_mm, 8192^3)"
+    else:
+        int8_peak, int8_peak_sust = int8_from_bf16, int8_from_bf16_sust
+        int8_kind = peak_kind + " bf16 x 2 (the nominal dense int8 / bf16 ratio)"
 
     barrier, max_over_ranks = rank_ops(torch, dist, world, dev)
 
@@ -266,8 +319,10 @@ def run_ours(args):
         "e2e": e2e,
         "gpu_launches": args.steps * LAYERS * len(DECODE_SHAPES) * kernels_per_call,
         "clocks": clk,
-        "peaks": {"hbm_gbs": hbm_peak, "int8_tops_burst": int8_peak, "int8_tops_sustained": int8_peak_sust,
-                  "kind": peak_kind + " (int8 = bf16 x 2, the nominal dense ratio)"},
+        "peaks": {"hbm_gbs": hbm_peak, "hbm_kind": peak_kind, "int8_tops_burst": int8_peak,
+                  "int8_tops_sustained": int8_peak_sust, "int8_kind": int8_kind, "int8_measured": int8_meas,
+                  "int8_cross_check_bf16x2": {"burst": round(int8_from_bf16, 1),
+                                              "sustained": round(int8_from_bf16_sust, 1)}},
         "extras": extras,
     }
     print(json.dumps(line), flush=True)
@@ -297,34 +352,45 @@ def time_graph(torch, fn, reps: int, warm: int = 3):
     return ms
 
 
+def cold_copies(l2_bytes: int, matrix_bytes: int) -> int:
+    """Weight copies to rotate so that every call reads its weights from DRAM:
+    ceil(3 x L2 / bytes of one copy), at least 2."""
+    return max(2, -(-3 * l2_bytes // matrix_bytes))
+
+
 def run_extras(args, bl, synth, dev, hbm_peak, int8_peak):
     import torch
 
     out = {}
-    # batched decode and prefill at the 2B FFN shapes (3 rotating copies > L2 at M<=16)
+    l2 = int(torch.cuda.get_device_properties(dev).L2_cache_size)
+    out["l2_bytes"] = l2
+    # Batched decode at the 2B FFN shapes: ceil(3 L2 / 4.42 MB) rotating weight
+    # copies per shape (about 90 on a 126 MB L2), so every call streams its
+    # weights from DRAM; the codes of x and the outputs stay in L2.
     shapes = [(2560, 6912), (6912, 2560)]
-    packs = {}
-    for si, (K, N) in enumerate(shapes):
-        packs[(K, N)] = [bl.pack_weights(synth.weights(N, K, synth.SIGMA_2B, 50 + 10 * si + c, device=dev))
-                         for c in range(8)]
     batched = {}
-    for M in (4, 8, 16):
-        per = {}
-        for K, N in shapes:
+    for si, (K, N) in enumerate(shapes):
+        ncp = cold_copies(l2, K * N // 4)
+        cps = [bl.pack_weights(synth.weights(N, K, synth.SIGMA_2B, 50 + 1000 * si + c, device=dev))
+               for c in range(ncp)]
+        for M in (4, 8, 16):
             x = synth.activations(M, K, seed=M, device=dev)
             y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
             ws = torch.empty(bl.workspace_bytes(bl.BL_OP_FORWARD, M, N, K), dtype=torch.uint8, device=dev)
-            cp = packs[(K, N)]
 
             def fn():
-                for Wp, g in cp:
+                for Wp, g in cps:
                     bl.forward(Wp, g, x, out=y, ws=ws)
-            ms = time_graph(torch, fn, reps=20) / len(cp)
-            per[f"{K}x{N}"] = {"us_per_call": round(ms * 1e3, 2),
-                               "gbs": round(K * N / 4 / (ms * 1e-3) / 1e9, 1)}
-        batched[f"M{M}"] = per
+            ms = time_graph(torch, fn, reps=10) / len(cps)
+            gbs = K * N / 4 / (ms * 1e-3) / 1e9
+            batched.setdefault(f"M{M}", {})[f"{K}x{N}"] = {
+                "us_per_call": round(ms * 1e3, 2), "gbs": round(gbs, 1), "hbm_frac": round(gbs / hbm_peak, 4),
+                "copies": len(cps), "rotated_mb": round(len(cps) * K * N / 4 / 1e6, 1)}
+        del cps
     out["batched_decode_2b"] = batched
 
+    packs = {(K, N): bl.pack_weights(synth.weights(N, K, synth.SIGMA_2B, 50 + 1000 * si, device=dev))
+             for si, (K, N) in enumerate(shapes)}
     prefill = {}
     for M in (512, 2048, 4096):
         per = {}
@@ -332,7 +398,7 @@ def run_extras(args, bl, synth, dev, hbm_peak, int8_peak):
             x = synth.activations(M, K, seed=M, device=dev)
             y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
             ws = torch.empty(bl.workspace_bytes(bl.BL_OP_FORWARD, M, N, K), dtype=torch.uint8, device=dev)
-            Wp, g = packs[(K, N)][0]
+            Wp, g = packs[(K, N)]
 
             def fn():
                 bl.forward(Wp, g, x, out=y, ws=ws)
@@ -344,10 +410,13 @@ def run_extras(args, bl, synth, dev, hbm_peak, int8_peak):
     out["prefill_2b"] = prefill
     del packs
 
-    # 100B-class bandwidth stress: M = 1 and 16, two copies per shape (235 MB > L2)
+    # 100B-class shapes: M = 1 and 16 rotate ceil(3 L2 / 58.7 MB) copies (7 on a
+    # 126 MB L2: 411 MB per shape) so every call reads its weights from DRAM;
+    # M = 2048 is the tensor-core GEMM on one copy.
     big = {}
     for K, N in ((8192, 28672), (28672, 8192)):
-        cps = [bl.pack_weights(synth.weights(N, K, synth.SIGMA_100B, 90 + c, device=dev)) for c in range(2)]
+        ncp = cold_copies(l2, K * N // 4)
+        cps = [bl.pack_weights(synth.weights(N, K, synth.SIGMA_100B, 90 + c, device=dev)) for c in range(ncp)]
         torch.cuda.empty_cache()
         for M in (1, 16):
             x = synth.activations(M, K, seed=M, device=dev)
@@ -360,8 +429,22 @@ def run_extras(args, bl, synth, dev, hbm_peak, int8_peak):
             ms = time_graph(torch, fn, reps=10) / len(cps)
             gbs = K * N / 4 / (ms * 1e-3) / 1e9
             big[f"{K}x{N}_M{M}"] = {"us_per_call": round(ms * 1e3, 2), "gbs": round(gbs, 1),
-                                    "hbm_frac": round(gbs / hbm_peak, 4)}
-        del cps
+                                    "hbm_frac": round(gbs / hbm_peak, 4), "copies": len(cps),
+                                    "rotated_mb": round(len(cps) * K * N / 4 / 1e6, 1)}
+        M = 2048
+        x = synth.activations(M, K, seed=M, device=dev)
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(bl.workspace_bytes(bl.BL_OP_FORWARD, M, N, K), dtype=torch.uint8, device=dev)
+        Wp, g = cps[0]
+
+        def fn():
+            bl.forward(Wp, g, x, out=y, ws=ws)
+        ms = time_graph(torch, fn, reps=5)
+        tops = 2.0 * M * N * K / (ms * 1e-3) / 1e12
+        big[f"{K}x{N}_M{M}"] = {"ms": round(ms, 4), "tops": round(tops, 1),
+                                "frac_int8_peak": round(tops / int8_peak, 4)}
+        del cps, x, y, ws
+        torch.cuda.empty_cache()
     out["stress_100b"] = big
 
     # FFN chain: 30 layers, d=2560, f=6912, residual add
@@ -430,7 +513,13 @@ def run_extras(args, bl, synth, dev, hbm_peak, int8_peak):
         ms = time_graph(torch, fn, reps=5)
         wbytes = LAYERS * (sum(qkv_rows) * d + d * d + 3 * d * f) / 4
         linears[f"M{M}"] = {"ms_30_layers": round(ms, 4), "us_per_layer": round(ms * 1e3 / LAYERS, 2),
-                            "launches_per_layer": 4, "packed_gbs": round(wbytes / (ms * 1e-3) / 1e9, 1)}
+                            "launches_per_layer": 4, "packed_gbs": round(wbytes / (ms * 1e-3) / 1e9, 1),
+                            "pages_context": {
+                                "ms_per_token": PAGES_CPU_MS_PER_TOKEN,
+                                "what": "whole 2B model per output token on a laptop CPU (i7-13800H, 8 threads, "
+                                        "bitnet.cpp); includes attention, embeddings and the LM head, which "
+                                        "this number does not",
+                                "source": "paper card 'BitNet b1.58 2B4T Technical Report', Evidence, Table 1"}}
     out["decoder_linears_2b_30_layers"] = linears
     del layers, dec
     torch.cuda.empty_cache()
@@ -473,28 +562,52 @@ def run_e2e(args, bl, dev, graph, xs, ys, step_bytes, world, barrier, max_over_r
             "d2h_bytes_per_step": d2h, "ms_per_step": round(ms / args.steps, 5)}
 
 
+def cpu_model() -> str:
+    """The host CPU's model name (from /proc/cpuinfo)."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    return ln.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 def cpu_baseline(weights, xs, bl, budget_s: float):
     """The oracle (as it stands) on a bounded sample of the decode step: whole
-    layers of the four shapes, one after another, until the budget is spent."""
+    layers of the four shapes, one after another, until the budget is spent;
+    once on every host core (the reported value) and once on one thread."""
     import numpy as np
 
     import oracle
 
     bits = [x.cpu().view(__import__("torch").int16).numpy().view(np.uint16) for x in xs]
     host = [[(Wp.cpu().numpy(), float(g.cpu().item())) for Wp, g in row] for row in weights]
-    done_bytes, n_layers = 0, 0
-    t0 = time.perf_counter()
-    while time.perf_counter() - t0 < budget_s:
-        row = host[n_layers % LAYERS]
-        for (Wp, g), xb in zip(row, bits):
-            oracle.forward(Wp, g, xb)
-            done_bytes += Wp.size
-        n_layers += 1
-    dt = time.perf_counter() - t0
-    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
-    return {"value": round(done_bytes / dt / 1e9, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
-            "sample": f"{n_layers} layers of the decode step, cycling over its 30 layers "
-                      f"(4 shapes each, M=1): {done_bytes} packed bytes in {dt:.2f} s"}
+
+    def run(threads: int, seconds: float):
+        used = oracle.set_threads(threads)
+        done_bytes, n_layers = 0, 0
+        t0 = time.perf_counter()
+        while time.perf_counter() - t0 < seconds:
+            row = host[n_layers % LAYERS]
+            for (Wp, g), xb in zip(row, bits):
+                oracle.forward(Wp, g, xb)
+                done_bytes += Wp.size
+            n_layers += 1
+        dt = time.perf_counter() - t0
+        return used, done_bytes, n_layers, dt
+
+    all_cores = os.cpu_count() or 1
+    used, nbytes, nl, dt = run(all_cores, budget_s)
+    used1, nbytes1, nl1, dt1 = run(1, budget_s / 2)
+    oracle.set_threads(all_cores)
+    return {"value": round(nbytes / dt / 1e9, 4), "unit": "GB/s", "cores": used, "kind": "oracle",
+            "sample": f"{nl} layers of the decode step, cycling over its 30 layers "
+                      f"(4 shapes each, M=1): {nbytes} packed bytes in {dt:.2f} s",
+            "cpu_model": cpu_model(),
+            "single_thread": {"value": round(nbytes1 / dt1 / 1e9, 4), "unit": "GB/s", "cores": used1,
+                              "sample": f"{nl1} layers, {nbytes1} packed bytes in {dt1:.2f} s"}}
 
 
 # ----------------------------------------------------------------------------- reference arm
@@ -532,8 +645,8 @@ def run_reference(args):
         step()
     dt = time.perf_counter() - t0
     value = step_bytes * args.steps / dt / 1e9
-    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
-    sample = "one layer of the four decode shapes per step (M=1), of the 30-layer step"
+    cores = oracle.set_threads(0)
+    sample = f"one layer of the four decode shapes per step (M=1), of the 30-layer step; {cpu_model()}"
     line = {
         "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3),

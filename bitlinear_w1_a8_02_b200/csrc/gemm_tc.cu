@@ -619,38 +619,53 @@ cudaError_t launch_bn(const uint8_t* Wp, const float* gamma, int64_t N, int64_t 
 // estimate is waves x relative time of one tile; a narrower tile still loads the
 // whole activation tile and pays the same per-k-block overheads, so on B200 a
 // 128-row tile takes 0.68 and a 64-row tile 0.59 of a 256-row tile (measured).
-int gemm_tc_tile_width(int64_t M, int64_t N, int sms) {
+namespace {
+constexpr int kWidths[3] = {256, 128, 64};
+constexpr double kTileCost[3] = {1.0, 0.68, 0.59};
+
+// Estimated time (in 256-row tile times) and width of the best data-parallel plan.
+double best_data_parallel(int64_t M, int64_t N, int sms, int* width) {
     const int64_t mt = (M + BM - 1) / BM;
-    const int widths[3] = {256, 128, 64};
-    const double tile_cost[3] = {1.0, 0.68, 0.59};
     int best = 256;
     double best_time = 0.0;
     for (int i = 0; i < 3; ++i) {
-        const int64_t tiles = mt * ((N + widths[i] - 1) / widths[i]);
-        const double time = (double)((tiles + sms - 1) / sms) * tile_cost[i];
+        const int64_t tiles = mt * ((N + kWidths[i] - 1) / kWidths[i]);
+        const double time = (double)((tiles + sms - 1) / sms) * kTileCost[i];
         if (i == 0 || time < best_time - 1e-9) {
-            best = widths[i];
+            best = kWidths[i];
             best_time = time;
         }
     }
-    return best;
+    *width = best;
+    return best_time;
+}
+}  // namespace
+
+int gemm_tc_tile_width(int64_t M, int64_t N, int sms) {
+    int w = 256;
+    best_data_parallel(M, N, sms, &w);
+    return w;
 }
 
 size_t gemm_sk_workspace_bytes(int sms) { return (size_t)2 * sms * BM * 256 * sizeof(uint32_t); }
 
 
-// Stream-K only where the data-parallel plan leaves much of its last wave idle
-// (under 70% of its CTA-slots busy) and the tiles are long in K (at least 32
-// k-blocks), so the pieces are large: each split tile costs a 128 KB write and
+// Stream-K only where the best data-parallel plan leaves much of its last wave
+// idle (under 70% of its CTA-slots busy), the tiles are long in K (at least 32
+// k-blocks, so the pieces are large: each split tile costs a 128 KB write and
 // read of int32 pieces plus the fix-up launch, which ate the gain on the other
-// shapes measured (2560 -> 6912 at M = 512, 6912 -> 2560 at M = 4096).
+// shapes measured: 2560 -> 6912 at M = 512, 6912 -> 2560 at M = 4096), and the
+// plan stream-K actually runs (256-row tiles spread evenly over the SMs) is
+// estimated faster than that data-parallel plan.
 bool gemm_use_stream_k(int64_t M, int64_t N, int64_t K, int sms) {
     const int64_t mt = (M + BM - 1) / BM;
-    const int bn = gemm_tc_tile_width(M, N, sms);
+    int bn = 256;
+    const double dp_time = best_data_parallel(M, N, sms, &bn);
     const int64_t dp_tiles = mt * ((N + bn - 1) / bn);
     const int64_t waves = (dp_tiles + sms - 1) / sms;
     const double busy = (double)dp_tiles / (double)(waves * sms);
-    return busy < 0.7 && (K + BK - 1) / BK >= 32;
+    const double sk_time = (double)(mt * ((N + 255) / 256)) / (double)sms;
+    return busy < 0.7 && (K + BK - 1) / BK >= 32 && sk_time < dp_time;
 }
 
 cudaError_t launch_gemm_tc(const uint8_t* Wp, const float* gamma, int64_t N, int64_t K,

@@ -124,7 +124,7 @@ bl_status bitlinear_quant_act(const uint16_t* x, int64_t M, int64_t K,
  *   Wp        [N, K/4] device packed weights; 16-byte aligned
  *   gamma     [1] device fp32 (as written by bitlinear_pack_weights)
  *   N, K      N >= 0, K >= 4, K % 4 == 0
- *   x         [M, K] device bf16 bits; 16-byte aligned
+ *   x         [M, K] device bf16 bits; 2-byte aligned (16-byte for the fast kernels)
  *   M         M >= 0; M == 0 or N == 0 launches nothing
  *   residual  [M, N] device bf16 bits added before the final rounding; may be NULL
  *   y         [M, N] device bf16 bits output; 4-byte aligned
@@ -228,9 +228,13 @@ bl_status bitlinear_ffn(const uint8_t* Wg, const float* gg, const uint8_t* Wu, c
  * engine that reserved all device memory at start-up and allows no allocation
  * afterwards, or a latency-critical loop in which an allocation would implicitly
  * synchronise the device. They may also have no workspace buffer to pass. This
- * call computes exactly what bitlinear_forward computes (same kernels, same bits)
- * but keeps its scratch in a fixed 1 MiB array inside the library's own device
- * memory, which every GPU that loads the library holds until the process exits.
+ * call computes what bitlinear_forward computes, to the same integers and bf16
+ * bits, but keeps its scratch in a fixed 1 MiB array inside the library's own
+ * device memory, which every GPU that loads the library holds until the process
+ * exits. It always runs the separate act-quant kernel and then the GEMV (the
+ * streamed one when K % 256 == 0 and Wp and x are 16-byte aligned, else the
+ * generic one), also for M > 16, where bitlinear_forward uses the tensor cores:
+ * large M is correct but slow here.
  *
  *   Arguments as bitlinear_forward, minus ws / ws_bytes.
  *   Limit: the scratch must hold the activation codes plus two per-token words:
@@ -239,6 +243,8 @@ bl_status bitlinear_ffn(const uint8_t* Wg, const float* gg, const uint8_t* Wu, c
  *   No call allocates device memory or calls an allocating library routine.
  *   The first call on each device looks up the array's device address
  *   (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   After a cudaDeviceReset the next call on that device looks it up again
+ *   (the same rule applies to that call).
  *   Every call on a device shares the one array, which keeps the last call's
  *   contents (nothing in it needs to start at zero). Calls that can overlap on
  *   the GPU (other streams, unordered host threads) race on it: order them.

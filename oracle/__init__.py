@@ -45,6 +45,7 @@ def _l():
         I = ctypes.c_int64
         F = ctypes.c_float
         sig = {
+            "orc_set_threads": (ctypes.c_int, [ctypes.c_int]),
             "orc_bf16_to_f32": (F, [ctypes.c_uint16]),
             "orc_f32_to_bf16": (ctypes.c_uint16, [F]),
             "orc_bf16_to_f32_array": (None, [P, I, P]),
@@ -80,6 +81,14 @@ def _p(a):
 
 def _c(a, dtype):
     return np.ascontiguousarray(a, dtype=dtype)
+
+
+# --------------------------------------------------------------------------- threads
+
+def set_threads(n: int) -> int:
+    """Threads of the oracle's OpenMP loops (0 leaves it unchanged); returns the
+    count in effect. Results do not depend on it."""
+    return int(_l().orc_set_threads(int(n)))
 
 
 # --------------------------------------------------------------------------- bf16

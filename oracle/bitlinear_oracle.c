@@ -43,11 +43,26 @@
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
 
 #define ORC_W_EPS 1e-5f   /* eps in W / (gamma + eps) */
 #define ORC_X_EPS 1e-5f   /* floor on the per-token absmax */
 #define ORC_QB 127.0f     /* int8 activation range: codes in [-128, 127], scale to 127 */
 #define ORC_RMS_EPS 1e-5f /* subln RMSNorm eps */
+
+/* Threads of the OpenMP loops over independent output elements (timing only:
+ * results do not depend on it). Returns the count now in effect.             */
+int orc_set_threads(int n) {
+#ifdef _OPENMP
+    if (n > 0) omp_set_num_threads(n);
+    return omp_get_max_threads();
+#else
+    (void)n;
+    return 1;
+#endif
+}
 
 /* ------------------------------------------------------------------------- */
 /* bf16 <-> fp32. bf16 is the upper half of an fp32 word; widening is exact and

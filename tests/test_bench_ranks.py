@@ -50,3 +50,12 @@ def test_whole_job_value_is_weak_scaling_aggregate():
     # two ranks each streaming 1 GB per step for 10 steps in (slowest) 1 s -> 20 GB/s
     assert bench.whole_job_gbs(2, 10 ** 9, 10, 1000.0) == pytest.approx(20.0)
     assert bench.whole_job_gbs(1, 10 ** 9, 10, 1000.0) == pytest.approx(10.0)
+
+
+def test_cold_rotation_exceeds_three_l2():
+    l2 = 126 * 1024 * 1024
+    for nbytes in (2560 * 640 // 4, 2560 * 6912 // 4, 8192 * 28672 // 4):
+        n = bench.cold_copies(l2, nbytes)
+        assert n * nbytes >= 3 * l2 and (n - 1) * nbytes < 3 * l2 or n == 2
+    assert bench.cold_copies(l2, 2560 * 6912 // 4) == 90
+    assert bench.cold_copies(l2, 8192 * 28672 // 4) == 7

@@ -135,6 +135,17 @@ def test_forward_prefill_sampled(cuda_device, K, N, M):
     check_forward_sampled(Wp, gamma, Wp_ref, g_ref, x, cuda_device, rows, toks)
 
 
+@pytest.mark.parametrize("K,N", [(2560, 6912), (6912, 2560)])
+def test_forward_prefill_full_output(cuda_device, K, N):
+    """Every output of a 512-token prefill at the 2B FFN shapes (the tensor-core
+    GEMM, stream-K split for 6912 -> 2560) against the oracle."""
+    M = 512
+    W = make_weights(N, K, 0.02, seed=3100 + K + N)
+    Wp, gamma, Wp_ref, g_ref = pack_both(W, cuda_device)
+    x = synth.activations(M, K, seed=3200 + M, outliers=True)
+    check_forward_full(Wp, gamma, Wp_ref, g_ref, x, cuda_device)
+
+
 @pytest.mark.parametrize("M", [1, 16, 2048])
 @pytest.mark.parametrize("K,N", [(8192, 28672), (28672, 8192)])
 def test_forward_100b_sampled(cuda_device, K, N, M):
@@ -378,11 +389,14 @@ def test_ffn_chain_decode_teacher_forced(cuda_device):
 
 
 def test_ffn_prefill_sampled_tokens(cuda_device):
-    d, f, M = 2560, 6912, 512
+    """All 30 layers at d=2560, f=6912, M=512, teacher-forced: each layer's GPU
+    input rows of the sampled tokens go to the oracle, whose outputs are compared
+    bit for bit (tokens are independent, so a sampled row is an exact check)."""
+    d, f, M, L = 2560, 6912, 512, 30
     h = synth.activations(M, d, seed=2, outliers=False)
     h_dev = h.to(cuda_device)
-    toks = sample_indices(M, 6, seed=4)
-    for layer in range(3):
+    toks = sample_indices(M, 8, seed=4)
+    for layer in range(L):
         (Wg, gg, Wgr, ggr), (Wu, gu, Wur, gur), (Wd, gd, Wdr, gdr) = ffn_weights(layer, d, f, cuda_device)
         y_dev = bl.ffn(Wg, gg, Wu, gu, Wd, gd, h_dev, residual=h_dev)
         xin = bits(h_dev)[toks]
