@@ -669,13 +669,16 @@ PROFILE_CASES = {
     "gemv_2b_down": (6912, 2560, 1),
     "gemv_2b_m16": (2560, 6912, 16),
     "gemv_100b": (8192, 28672, 1),
+    "gemv_100b_m16": (8192, 28672, 16),
+    "gemv_100b_down_m16": (28672, 8192, 16),
     "gemm_2b": (2560, 6912, 4096),
     "gemm_2b_down": (6912, 2560, 4096),
 }
 
 
-def run_profile_case(name: str, reps: int):
-    """Run one forward call `reps` times (after packing); for ncu -k/-s/-c."""
+def run_profile_case(name: str, reps: int, gemv_kernel: int = 0):
+    """Run one forward call `reps` times (after packing); for ncu -k/-s/-c.
+    gemv_kernel selects the M <= 16 kernel (bitlinear_set_gemv_kernel)."""
     import torch
 
     import bitlinear_w1_a8_02_b200 as bl
@@ -689,10 +692,12 @@ def run_profile_case(name: str, reps: int):
     x = synth.activations(M, K, seed=2, device=dev)
     y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
     ws = torch.empty(bl.workspace_bytes(bl.BL_OP_FORWARD, M, N, K), dtype=torch.uint8, device=dev)
-    for _ in range(reps):
-        bl.forward(Wp, g, x, out=y, ws=ws)
+    with bl.gemv_kernel(gemv_kernel):
+        for _ in range(reps):
+            bl.forward(Wp, g, x, out=y, ws=ws)
     torch.cuda.synchronize()
-    print(f"profile case {name}: K={K} N={N} M={M}, {reps} calls", flush=True)
+    assert bl.get_device_error() == 0
+    print(f"profile case {name}: K={K} N={N} M={M}, {reps} calls, GEMV kernel {gemv_kernel}", flush=True)
 
 
 def main():
@@ -707,9 +712,11 @@ def main():
     ap.add_argument("--profile-case", choices=sorted(PROFILE_CASES),
                     help="run one forward call repeatedly for an ncu capture, then exit")
     ap.add_argument("--reps", type=int, default=5)
+    ap.add_argument("--gemv-kernel", type=int, default=0,
+                    help="M <= 16 kernel for --profile-case: 0 auto, 1 streamed, 2 tensor-core")
     args = ap.parse_args()
     if args.profile_case:
-        run_profile_case(args.profile_case, args.reps)
+        run_profile_case(args.profile_case, args.reps, args.gemv_kernel)
         return
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

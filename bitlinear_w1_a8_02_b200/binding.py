@@ -24,6 +24,7 @@ STATUS_NAMES = {
 }
 BL_BF16, BL_FP32 = 0, 1
 BL_OP_PACK, BL_OP_FORWARD, BL_OP_FFN, BL_OP_VALIDATE = 0, 1, 2, 3
+BL_GEMV_AUTO, BL_GEMV_STREAM, BL_GEMV_TENSOR = 0, 1, 2
 
 # Every symbol include/bitlinear.h declares, with (restype, argtypes).
 _P = ctypes.c_void_p
@@ -45,6 +46,7 @@ SIGNATURES = {
     "bitlinear_validate_packed": (_ST, [_P, _I, _I, _P, _P, _S, _P]),
     "bitlinear_get_device_error": (_ST, [_P]),
     "bitlinear_selftest_timeout": (_ST, [_I, _P]),
+    "bitlinear_set_gemv_kernel": (ctypes.c_int, [ctypes.c_int]),
 }
 
 
@@ -278,3 +280,27 @@ def get_device_error(device=None) -> int:
     """Synchronise and return the pending device status (0 when clean)."""
     device = torch.device("cuda", torch.cuda.current_device()) if device is None else device
     return int(lib().bitlinear_get_device_error(_stream(device)))
+
+
+def set_gemv_kernel(kind: int) -> int:
+    """Process-wide choice of the M <= 16 kernel (BL_GEMV_*); returns the previous one."""
+    prev = int(lib().bitlinear_set_gemv_kernel(int(kind)))
+    if prev < 0:
+        raise ValueError(f"unknown GEMV kernel {kind}")
+    return prev
+
+
+class gemv_kernel:
+    """Context manager: run the enclosed calls with one M <= 16 kernel."""
+
+    def __init__(self, kind: int):
+        self.kind = kind
+        self.prev = None
+
+    def __enter__(self):
+        self.prev = set_gemv_kernel(self.kind)
+        return self
+
+    def __exit__(self, *exc):
+        set_gemv_kernel(self.prev)
+        return False

@@ -6,6 +6,8 @@
 // exception escape.
 #include <bitlinear.h>
 
+#include <atomic>
+
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -106,7 +108,16 @@ bl_status check_ws(const void* ws, size_t ws_bytes, size_t need) {
 }
 
 // Which kernel runs a projection, and the activation-code layout it reads.
-enum class Path { GemvFast, GemvGeneric, GemmTc };
+enum class Path { GemvFast, GemvGeneric, GemmTc, GemvTc };
+
+// Process-wide choice of the M <= 16 kernel (bitlinear_set_gemv_kernel).
+std::atomic<int> g_gemv_kernel{BL_GEMV_AUTO};
+
+// Automatic choice for M <= 16: the streamed dp4a / mma.sync GEMV. Measured on
+// B200 with cold weights, the tensor-core GEMV is slower or equal at every
+// shape and token count (its weight stream stays near 2.3 TB/s: each 512-code
+// stage touches 128 rows), so it runs only when selected.
+inline bool prefer_gemv_tc(int64_t, int64_t, int64_t) { return false; }
 
 // `x` is the bf16 input the codes are made from (the fast quantiser reads it
 // 16 bytes at a time); null when the codes come from the FFN glue kernel.
@@ -114,12 +125,20 @@ inline Path choose_path(const uint8_t* Wp, int64_t N, int64_t K, int64_t M, cons
                         const void* x) {
     if (x && !aligned(x, 16)) return Path::GemvGeneric;
     if (M > 16 && bl::gemm_tc_ok(N, K, Wp, xq)) return Path::GemmTc;
-    if (bl::gemv_fast_ok(N, K) && aligned(Wp, 16)) return Path::GemvFast;
+    if (bl::gemv_fast_ok(N, K) && aligned(Wp, 16)) {
+        const int kind = g_gemv_kernel.load(std::memory_order_relaxed);
+        const bool tc_ok = bl::gemv_tc_ok(N, K, M, Wp, xq);
+        if (kind == BL_GEMV_TENSOR && tc_ok) return Path::GemvTc;
+        if (kind == BL_GEMV_AUTO && tc_ok && prefer_gemv_tc(N, K, M)) return Path::GemvTc;
+        return Path::GemvFast;
+    }
     return Path::GemvGeneric;
 }
 
 inline int layout_of(Path p) {
-    return p == Path::GemmTc ? bl::XQ_G16T : p == Path::GemvFast ? bl::XQ_PLANES : bl::XQ_NATURAL;
+    return (p == Path::GemmTc || p == Path::GemvTc) ? bl::XQ_G16T
+           : p == Path::GemvFast                     ? bl::XQ_PLANES
+                                                     : bl::XQ_NATURAL;
 }
 
 // One BitLinear projection of already-quantised codes `xq` (in layout_of(path)).
@@ -132,6 +151,8 @@ bl_status project(Path path, const uint8_t* Wp, const float* gamma, int64_t N, i
                 bl::launch_gemm_tc(Wp, gamma, N, K, xq, scale, xsum, M, out, s, sk_ws, sk_ws_bytes));
         case Path::GemvFast:
             return cuda_status(bl::launch_gemv(Wp, gamma, N, K, xq, scale, xsum, M, out, s));
+        case Path::GemvTc:
+            return cuda_status(bl::launch_gemv_tc(Wp, gamma, N, K, xq, scale, xsum, M, out, s));
         default:
             return cuda_status(bl::launch_gemv_generic(Wp, gamma, N, K, xq, scale, M, out, s));
     }
@@ -154,6 +175,11 @@ BL_API const char* bitlinear_status_string(bl_status st) {
         case BL_ERR_BAD_CODE: return "BL_ERR_BAD_CODE: packed weights hold the invalid code 3";
     }
     return "unknown bl_status";
+}
+
+BL_API int bitlinear_set_gemv_kernel(int kind) {
+    if (kind < BL_GEMV_AUTO || kind > BL_GEMV_TENSOR) return -1;
+    return g_gemv_kernel.exchange(kind);
 }
 
 BL_API size_t bitlinear_workspace_bytes(int op, int64_t M, int64_t N, int64_t K) {
@@ -227,7 +253,7 @@ bl_status forward_impl(const uint8_t* Wp, const float* gamma, int64_t N, int64_t
     Path path = choose_path(Wp, N, K, M, xq, x);
     // segment ends that do not fall on the fast paths' tiles take the generic kernel
     if ((path == Path::GemmTc && !bl::gemm_segments_ok(out, N)) ||
-        (path == Path::GemvFast && !bl::gemv_segments_ok(out, N)))
+        ((path == Path::GemvFast || path == Path::GemvTc) && !bl::gemv_segments_ok(out, N)))
         path = Path::GemvGeneric;
     if (path == Path::GemvFast && bl::gemv_fused_ok(M, K))  // one kernel: quantise + GEMV
         return cuda_status(bl::launch_gemv(Wp, gamma, N, K, nullptr, nullptr, nullptr, M, out, s, x, rmsnorm));

@@ -533,7 +533,10 @@ __global__ void __launch_bounds__(512) gemm_sk_fixup_kernel(int M, int N, int K,
                static_cast<size_t>(m) * N + n0 + col, out, vec);
 }
 
+}  // namespace
+
 // ---------------------------------------------------------------- host side
+namespace {
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
                                    const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
@@ -553,8 +556,8 @@ EncodeTiledFn encode_fn() {
     }
     return fn;
 }
+}  // namespace
 
-// 2-D uint8 tensor map over [rows, cols] (cols contiguous), box [box_rows, box_cols].
 bool make_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows,
               uint32_t box_cols, bool swizzle128) {
     EncodeTiledFn enc = encode_fn();
@@ -568,8 +571,6 @@ bool make_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, 
                swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
-
-}  // namespace
 
 bool gemm_segments_ok(const GemvOut& out, int64_t N) {
     for (int i = 0; i < 3; ++i)

@@ -2,6 +2,7 @@
 // interface is include/bitlinear.h). Each returns the cudaError_t of its launch.
 #pragma once
 
+#include <cuda.h>  // CUtensorMap (type only)
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -85,6 +86,21 @@ cudaError_t launch_gemm_tc(const uint8_t* Wp, const float* gamma, int64_t N, int
                            const int8_t* xq_g16t, const float* scale, const int32_t* xsum, int64_t M,
                            const GemvOut& out, cudaStream_t s, void* sk_ws = nullptr, size_t sk_ws_bytes = 0);
 size_t gemm_sk_workspace_bytes(int sms);
+
+// 2-D uint8 TMA tensor map over [rows, cols] (cols contiguous), box [box_rows,
+// box_cols], optionally 128-byte swizzled; false when the driver refuses it.
+bool make_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows,
+              uint32_t box_cols, bool swizzle128);
+
+// ---- tensor-core GEMV for up to 16 tokens (gemv_tc.cu)
+// xq_g16t: G16T layout codes of M <= 16 tokens. Requires K % 256 == 0 and
+// 16-byte aligned Wp and xq_g16t; any N.
+bool gemv_tc_ok(int64_t N, int64_t K, int64_t M, const void* Wp, const void* xq);
+cudaError_t launch_gemv_tc(const uint8_t* Wp, const float* gamma, int64_t N, int64_t K,
+                           const int8_t* xq_g16t, const float* scale, const int32_t* xsum, int64_t M,
+                           const GemvOut& out, cudaStream_t s);
+// K-split of the tensor-core GEMV (CTAs per cluster) for a shape, >= 1.
+int gemv_tc_split(int64_t N, int64_t K, int sms);
 
 // ---- FFN glue (ffn.cu)
 // h = relu(g)^2 * u; hn = subln(h); q2, s2, xsum2 = quant(hn) in `layout`.

@@ -1,7 +1,9 @@
-// Inline-PTX wrappers for the sm_100a pieces the tensor-core GEMM uses:
-// mbarriers (with bounded waits), TMA tile loads (no multicast), tcgen05 TMEM
-// allocation, MMA issue/commit and TMEM loads, and the shared-memory matrix
-// descriptor of the 128-byte-swizzled K-major operand layout.
+// Inline-PTX wrappers for the sm_100a pieces the tensor-core kernels use:
+// mbarriers (with bounded waits), TMA tile loads and L2 prefetches (no
+// multicast), tcgen05 TMEM allocation, MMA issue/commit (A from shared memory
+// or from TMEM), TMEM loads and stores, cluster barriers and asynchronous adds
+// into a peer CTA's shared memory, and the shared-memory matrix descriptor of
+// the 128-byte-swizzled K-major operand layout.
 #pragma once
 
 #include <cuda.h>  // CUtensorMap (type only)
@@ -142,6 +144,92 @@ __device__ __forceinline__ void tmem_ld_wait() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// D[tmem] (+)= A[tmem] x B[smem desc]: the A operand (M = 128 rows, K = 32
+// bytes = 8 columns per lane) is read from tensor memory at `a_tmem`.
+__device__ __forceinline__ void mma_i8_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                              uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// 32 lanes x 32 consecutive 32-bit columns: thread t writes lane (base lane + t).
+__device__ __forceinline__ void tmem_st_32x32(uint32_t taddr, const uint32_t (&v)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+        "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
+        "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]),
+        "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]),
+        "r"(v[29]), "r"(v[30]), "r"(v[31])
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_st_wait() {
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// 32 lanes x 8 / 16 consecutive 32-bit columns: thread t reads lane (base lane + t).
+__device__ __forceinline__ void tmem_ld_32x8(uint32_t taddr, uint32_t (&v)[8]) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+                   "=r"(v[7])
+                 : "r"(taddr)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld_32x16(uint32_t taddr, uint32_t (&v)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+          "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]),
+          "=r"(v[14]), "=r"(v[15])
+        : "r"(taddr)
+        : "memory");
+}
+
+// ---------------------------------------------------------------- clusters
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+// Every non-exited thread of every CTA in the cluster arrives, then waits.
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
+}
+
+// Shared-memory address of the same variable in CTA `rank` of this cluster.
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t saddr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+    return r;
+}
+
+// Asynchronous 32-bit add into another CTA's shared memory; the 4 bytes count as
+// transaction bytes on that CTA's mbarrier `remote_bar`.
+__device__ __forceinline__ void red_add_remote(uint32_t remote_addr, uint32_t v, uint32_t remote_bar) {
+    asm volatile(
+        "red.async.relaxed.cluster.shared::cluster.mbarrier::complete_tx::bytes.add.u32 [%0], %1, [%2];" ::"r"(
+            remote_addr),
+        "r"(v), "r"(remote_bar)
+        : "memory");
+}
+
+// L2 prefetch of one 2-D TMA tile (no shared memory written).
+__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap* m, int x, int y) {
+    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global [%0, {%1, %2}];" ::"l"(reinterpret_cast<uint64_t>(m)),
+                 "r"(x), "r"(y)
+                 : "memory");
+}
+
 // Shared-memory matrix descriptor: K-major operand in the canonical 128-byte
 // swizzle layout (8 rows x 128 bytes per 1024-byte atom, atoms 1024 bytes
 // apart). Start address and offsets are in 16-byte units; version 1 (sm100).
@@ -153,6 +241,16 @@ __device__ __forceinline__ uint64_t desc_kmajor_sw128(uint32_t saddr) {
     d |= static_cast<uint64_t>(1) << 46;                  // descriptor version [46,48)
     d |= static_cast<uint64_t>(2) << 61;                  // SWIZZLE_128B       [61,64)
     return d;
+}
+
+// Instruction descriptor of kind::i8 with A unsigned (weight codes 0..2) and B
+// signed (activation codes): int32 D, both K-major, M x N tile.
+__host__ __device__ constexpr uint32_t idesc_i8_u8s8(int m, int n) {
+    return (2u << 4)                          // D format: S32
+           | (0u << 7)                        // A format: unsigned 8-bit
+           | (1u << 10)                       // B format: signed 8-bit
+           | (static_cast<uint32_t>(n >> 3) << 17)
+           | (static_cast<uint32_t>(m >> 4) << 24);
 }
 
 // Instruction descriptor of kind::i8: int32 D, A signed, B unsigned, both

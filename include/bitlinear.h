@@ -77,6 +77,13 @@ typedef enum {
     BL_OP_VALIDATE = 3  /* sizes ignored */
 } bl_op;
 
+/* Kernels for M <= 16 tokens (bitlinear_set_gemv_kernel). */
+typedef enum {
+    BL_GEMV_AUTO = 0,   /* the library picks per call (default) */
+    BL_GEMV_STREAM = 1, /* streamed GEMV: dp4a (one token) / mma.sync (2..16 tokens) on registers */
+    BL_GEMV_TENSOR = 2  /* tcgen05 GEMV: weights unpacked into tensor memory, tokens as the MMA's N */
+} bl_gemv_kernel;
+
 /* Human-readable name of a status. Never NULL; host only. */
 const char* bitlinear_status_string(bl_status status);
 
@@ -252,6 +259,22 @@ bl_status bitlinear_ffn(const uint8_t* Wg, const float* gg, const uint8_t* Wu, c
 bl_status bitlinear_forward_noalloc(const uint8_t* Wp, const float* gamma, int64_t N, int64_t K,
                                     const uint16_t* x, int64_t M, const uint16_t* residual,
                                     uint16_t* y, int32_t* acc, bl_stream_t stream);
+
+/*
+ * Selects, for the whole process, which kernel the forward calls
+ * (bitlinear_forward, _ex, _rowwise and the projections inside bitlinear_ffn)
+ * use for M <= 16 tokens; the choice is read when a call launches its kernels.
+ * It exists to compare the kernels and to pin one in deployment; every kernel
+ * computes the same integers and bf16 bits. A kernel that cannot take a call's
+ * shape or alignment (both need K % 256 == 0 and 16-byte aligned Wp and x)
+ * leaves that call to the automatic choice. The paper card "BitNet b1.58 2B4T
+ * Technical Report", "Method Adaptation", describes one GPU kernel; the two
+ * here are this library's designs for B200.
+ *   kind   a bl_gemv_kernel value
+ * Returns the previous selection, or -1 (and changes nothing) for an unknown kind.
+ * Host only, no CUDA call.
+ */
+int bitlinear_set_gemv_kernel(int kind);
 
 /*
  * Check packed weights for the invalid code 3. SYNCHRONISES `stream`.

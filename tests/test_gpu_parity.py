@@ -444,3 +444,83 @@ def test_ffn_small_ragged(cuda_device):
     y = bl.ffn(P[0][0], P[0][1], P[1][0], P[1][1], P[2][0], P[2][1], x.to(cuda_device))
     ref = oracle.ffn_layer(P[0][2], P[0][3], P[1][2], P[1][3], P[2][2], P[2][3], bits(x))
     assert_bf16_exact(bits(y), ref["y"])
+
+
+# ----------------------------------------------------------------------------- tensor-core GEMV (M <= 16)
+
+@pytest.mark.parametrize("M", [1, 3, 8, 9, 16])
+@pytest.mark.parametrize("K,N", [(2560, 6912), (6912, 2560), (2560, 640), (256, 136), (768, 17), (8192, 1000)])
+def test_forward_gemv_tensor_core(cuda_device, K, N, M):
+    """The tcgen05 GEMV (weights unpacked into tensor memory, tokens as the MMA's
+    N = 8 / 16), forced on: ragged N, K with a half last stage (6912 = 13.5 x 512),
+    K split over clusters of 1 to 8 CTAs, residual and the int32 dump."""
+    W = make_weights(N, K, 0.02, seed=4000 + K + N)
+    Wp, gamma, Wp_ref, g_ref = pack_both(W, cuda_device)
+    x = synth.activations(M, K, seed=4100 + M, outliers=True)
+    res = synth.activations(M, N, seed=4200 + M, outliers=False)
+    with bl.gemv_kernel(bl.BL_GEMV_TENSOR):
+        check_forward_full(Wp, gamma, Wp_ref, g_ref, x, cuda_device, residual=res)
+    assert bl.get_device_error() == 0
+
+
+@pytest.mark.parametrize("M", [1, 16])
+@pytest.mark.parametrize("K,N", [(8192, 28672), (28672, 8192)])
+def test_forward_gemv_tensor_core_100b_sampled(cuda_device, K, N, M):
+    W = make_weights(N, K, synth.SIGMA_100B, seed=4300 + K)
+    Wp, gamma, Wp_ref, g_ref = pack_both(W, cuda_device)
+    x = synth.activations(M, K, seed=4400 + M, outliers=True)
+    rows = sample_indices(N, 256, seed=M + 11)
+    with bl.gemv_kernel(bl.BL_GEMV_TENSOR):
+        check_forward_sampled(Wp, gamma, Wp_ref, g_ref, x, cuda_device, rows, np.arange(M))
+
+
+@pytest.mark.parametrize("M", [2, 12])
+def test_forward_gemv_tensor_core_rowwise_and_segments(cuda_device, M):
+    K, N = 2560, 1024
+    W = make_weights(N, K, 0.02, seed=4500)
+    Wp, g = bl.pack_weights_rowwise(W.to(cuda_device))
+    Wp_ref, g_ref = oracle.pack_weights_rowwise(bits(W))
+    x = synth.activations(M, K, seed=4501 + M, outliers=True)
+    with bl.gemv_kernel(bl.BL_GEMV_TENSOR):
+        y, acc = bl.forward_rowwise(Wp, g, x.to(cuda_device), want_acc=True)
+    ref = oracle.forward_rowwise(Wp_ref, g_ref, bits(x))
+    assert np.array_equal(np_(acc), ref["acc"])
+    assert_bf16_exact(bits(y), ref["y"])
+    rows = [512, 256, 256]
+    parts = [make_weights(n, K, 0.02, seed=4510 + i) for i, n in enumerate(rows)]
+    dev_parts = [bl.pack_weights(p.to(cuda_device)) for p in parts]
+    ref_parts = [oracle.pack_weights(bits(p)) for p in parts]
+    with bl.gemv_kernel(bl.BL_GEMV_TENSOR):
+        yq = bl.forward_ex(torch.cat([p[0] for p in dev_parts]), torch.cat([p[1].reshape(1) for p in dev_parts]),
+                           rows, x.to(cuda_device), rmsnorm=True)
+    rq = oracle.forward_ex(np.concatenate([p[0] for p in ref_parts]), [p[1] for p in ref_parts], rows, bits(x),
+                           rmsnorm=True)
+    assert_bf16_exact(bits(yq), rq["y"])
+
+
+@pytest.mark.parametrize("M", [4, 16])
+def test_ffn_gemv_tensor_core(cuda_device, M):
+    """FFN projections on the tensor-core GEMV (fp32 gate/up outputs, then the
+    requantised down projection with the residual)."""
+    d, f = 2560, 6912
+    h = synth.activations(M, d, seed=4600 + M, outliers=False)
+    (Wg, gg, Wgr, ggr), (Wu, gu, Wur, gur), (Wd, gd, Wdr, gdr) = ffn_weights(11, d, f, cuda_device)
+    with bl.gemv_kernel(bl.BL_GEMV_TENSOR):
+        y = bl.ffn(Wg, gg, Wu, gu, Wd, gd, h.to(cuda_device), residual=h.to(cuda_device))
+    ref = oracle.ffn_layer(Wgr, ggr, Wur, gur, Wdr, gdr, bits(h), residual=bits(h))
+    assert_bf16_exact(bits(y), ref["y"])
+
+
+def test_gemv_kernel_choice_gives_the_same_bits(cuda_device):
+    """Every M <= 16 kernel computes the same integers and bf16 bits."""
+    K, N, M = 6912, 2560, 6
+    W = make_weights(N, K, 0.02, seed=4700)
+    Wp, gamma = bl.pack_weights(W.to(cuda_device))
+    x = synth.activations(M, K, seed=4701, outliers=True).to(cuda_device)
+    outs = []
+    for kind in (bl.BL_GEMV_STREAM, bl.BL_GEMV_TENSOR, bl.BL_GEMV_AUTO):
+        with bl.gemv_kernel(kind):
+            y, acc = bl.forward(Wp, gamma, x, want_acc=True)
+        outs.append((bits(y), np_(acc)))
+    for y, acc in outs[1:]:
+        assert np.array_equal(acc, outs[0][1]) and np.array_equal(y, outs[0][0])
