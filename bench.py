@@ -447,6 +447,33 @@ def run_extras(args, bl, synth, dev, hbm_peak, int8_peak):
         torch.cuda.empty_cache()
     out["stress_100b"] = big
 
+    # The three M <= 16 kernels side by side (bitlinear_set_gemv_kernel): the
+    # streamed dp4a / mma.sync GEMV (the automatic choice), the tensor-core GEMV
+    # with the weights in TMEM, and the lookup-table GEMV after the bitnet.cpp
+    # CPU kernels; cold weights as above.
+    kinds = (("stream", bl.BL_GEMV_STREAM), ("tensor", bl.BL_GEMV_TENSOR), ("lut", bl.BL_GEMV_LUT))
+    compared = {}
+    for K, N, sigma in ((2560, 6912, synth.SIGMA_2B), (8192, 28672, synth.SIGMA_100B)):
+        ncp = cold_copies(l2, K * N // 4)
+        cps = [bl.pack_weights(synth.weights(N, K, sigma, 70 + c, device=dev)) for c in range(ncp)]
+        for M in (1, 4, 16):
+            x = synth.activations(M, K, seed=M, device=dev)
+            y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+            ws = torch.empty(bl.workspace_bytes(bl.BL_OP_FORWARD, M, N, K), dtype=torch.uint8, device=dev)
+            row = {}
+            for name, kind in kinds:
+                with bl.gemv_kernel(kind):
+                    def fn():
+                        for Wp, g in cps:
+                            bl.forward(Wp, g, x, out=y, ws=ws)
+                    ms = time_graph(torch, fn, reps=3) / len(cps)
+                gbs = K * N / 4 / (ms * 1e-3) / 1e9
+                row[name] = {"us_per_call": round(ms * 1e3, 2), "hbm_frac": round(gbs / hbm_peak, 4)}
+            compared[f"{K}x{N}_M{M}"] = row
+        del cps
+        torch.cuda.empty_cache()
+    out["gemv_kernels_compared"] = compared
+
     # FFN chain: 30 layers, d=2560, f=6912, residual add
     d, f = 2560, 6912
     layers = []

@@ -5,7 +5,7 @@ of ``include/bitlinear.h``); this package is its Python binding plus the seeded
 synthetic input generators in ``synth``.
 """
 from .binding import (  # noqa: F401
-    BL_BF16, BL_FP32, BL_GEMV_AUTO, BL_GEMV_STREAM, BL_GEMV_TENSOR, BL_OK, BL_OP_FFN, BL_OP_FORWARD, BL_OP_PACK,
+    BL_BF16, BL_FP32, BL_GEMV_AUTO, BL_GEMV_LUT, BL_GEMV_STREAM, BL_GEMV_TENSOR, BL_OK, BL_OP_FFN, BL_OP_FORWARD, BL_OP_PACK,
     BL_OP_VALIDATE, LIB_PATH, SIGNATURES, STATUS_NAMES, BitLinearError, ffn, forward, forward_ex, forward_rowwise,
     gemv_kernel, get_device_error, lib, pack_weights, pack_weights_rowwise, quant_act, set_gemv_kernel,
     validate_packed, workspace_bytes,

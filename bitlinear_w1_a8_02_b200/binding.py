@@ -24,7 +24,7 @@ STATUS_NAMES = {
 }
 BL_BF16, BL_FP32 = 0, 1
 BL_OP_PACK, BL_OP_FORWARD, BL_OP_FFN, BL_OP_VALIDATE = 0, 1, 2, 3
-BL_GEMV_AUTO, BL_GEMV_STREAM, BL_GEMV_TENSOR = 0, 1, 2
+BL_GEMV_AUTO, BL_GEMV_STREAM, BL_GEMV_TENSOR, BL_GEMV_LUT = 0, 1, 2, 3
 
 # Every symbol include/bitlinear.h declares, with (restype, argtypes).
 _P = ctypes.c_void_p

@@ -108,7 +108,7 @@ bl_status check_ws(const void* ws, size_t ws_bytes, size_t need) {
 }
 
 // Which kernel runs a projection, and the activation-code layout it reads.
-enum class Path { GemvFast, GemvGeneric, GemmTc, GemvTc };
+enum class Path { GemvFast, GemvGeneric, GemmTc, GemvTc, GemvLut };
 
 // Process-wide choice of the M <= 16 kernel (bitlinear_set_gemv_kernel).
 std::atomic<int> g_gemv_kernel{BL_GEMV_AUTO};
@@ -129,6 +129,7 @@ inline Path choose_path(const uint8_t* Wp, int64_t N, int64_t K, int64_t M, cons
         const int kind = g_gemv_kernel.load(std::memory_order_relaxed);
         const bool tc_ok = bl::gemv_tc_ok(N, K, M, Wp, xq);
         if (kind == BL_GEMV_TENSOR && tc_ok) return Path::GemvTc;
+        if (kind == BL_GEMV_LUT && bl::gemv_lut_ok(N, K, M, Wp, xq)) return Path::GemvLut;
         if (kind == BL_GEMV_AUTO && tc_ok && prefer_gemv_tc(N, K, M)) return Path::GemvTc;
         return Path::GemvFast;
     }
@@ -138,7 +139,7 @@ inline Path choose_path(const uint8_t* Wp, int64_t N, int64_t K, int64_t M, cons
 inline int layout_of(Path p) {
     return (p == Path::GemmTc || p == Path::GemvTc) ? bl::XQ_G16T
            : p == Path::GemvFast                     ? bl::XQ_PLANES
-                                                     : bl::XQ_NATURAL;
+                                                     : bl::XQ_NATURAL;  // generic and lookup-table kernels
 }
 
 // One BitLinear projection of already-quantised codes `xq` (in layout_of(path)).
@@ -153,6 +154,8 @@ bl_status project(Path path, const uint8_t* Wp, const float* gamma, int64_t N, i
             return cuda_status(bl::launch_gemv(Wp, gamma, N, K, xq, scale, xsum, M, out, s));
         case Path::GemvTc:
             return cuda_status(bl::launch_gemv_tc(Wp, gamma, N, K, xq, scale, xsum, M, out, s));
+        case Path::GemvLut:
+            return cuda_status(bl::launch_gemv_lut(Wp, gamma, N, K, xq, scale, M, out, s));
         default:
             return cuda_status(bl::launch_gemv_generic(Wp, gamma, N, K, xq, scale, M, out, s));
     }
@@ -178,7 +181,7 @@ BL_API const char* bitlinear_status_string(bl_status st) {
 }
 
 BL_API int bitlinear_set_gemv_kernel(int kind) {
-    if (kind < BL_GEMV_AUTO || kind > BL_GEMV_TENSOR) return -1;
+    if (kind < BL_GEMV_AUTO || kind > BL_GEMV_LUT) return -1;
     return g_gemv_kernel.exchange(kind);
 }
 

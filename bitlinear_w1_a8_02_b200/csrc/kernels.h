@@ -102,6 +102,13 @@ cudaError_t launch_gemv_tc(const uint8_t* Wp, const float* gamma, int64_t N, int
 // K-split of the tensor-core GEMV (CTAs per cluster) for a shape, >= 1.
 int gemv_tc_split(int64_t N, int64_t K, int sms);
 
+// ---- lookup-table GEMV for up to 16 tokens (gemv_lut.cu)
+// xq: NATURAL layout codes (4-byte aligned). Requires K % 256 == 0 and a 16-byte
+// aligned Wp; any N. Launches ceil(M / 4) times (four tokens per table).
+bool gemv_lut_ok(int64_t N, int64_t K, int64_t M, const void* Wp, const void* xq);
+cudaError_t launch_gemv_lut(const uint8_t* Wp, const float* gamma, int64_t N, int64_t K, const int8_t* xq,
+                            const float* scale, int64_t M, const GemvOut& out, cudaStream_t s);
+
 // ---- FFN glue (ffn.cu)
 // h = relu(g)^2 * u; hn = subln(h); q2, s2, xsum2 = quant(hn) in `layout`.
 cudaError_t launch_ffn_finalise(const float* g, const float* u, int64_t M, int64_t f, int layout,

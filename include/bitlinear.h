@@ -81,7 +81,9 @@ typedef enum {
 typedef enum {
     BL_GEMV_AUTO = 0,   /* the library picks per call (default) */
     BL_GEMV_STREAM = 1, /* streamed GEMV: dp4a (one token) / mma.sync (2..16 tokens) on registers */
-    BL_GEMV_TENSOR = 2  /* tcgen05 GEMV: weights unpacked into tensor memory, tokens as the MMA's N */
+    BL_GEMV_TENSOR = 2, /* tcgen05 GEMV: weights unpacked into tensor memory, tokens as the MMA's N */
+    BL_GEMV_LUT = 3     /* lookup tables of activation partial sums indexed by packed weight nibbles
+                           (the T-MAC method of the bitnet.cpp CPU kernels); four tokens per pass */
 } bl_gemv_kernel;
 
 /* Human-readable name of a status. Never NULL; host only. */
@@ -266,10 +268,12 @@ bl_status bitlinear_forward_noalloc(const uint8_t* Wp, const float* gamma, int64
  * use for M <= 16 tokens; the choice is read when a call launches its kernels.
  * It exists to compare the kernels and to pin one in deployment; every kernel
  * computes the same integers and bf16 bits. A kernel that cannot take a call's
- * shape or alignment (both need K % 256 == 0 and 16-byte aligned Wp and x)
+ * shape or alignment (all need K % 256 == 0 and 16-byte aligned Wp and x)
  * leaves that call to the automatic choice. The paper card "BitNet b1.58 2B4T
- * Technical Report", "Method Adaptation", describes one GPU kernel; the two
- * here are this library's designs for B200.
+ * Technical Report", "Method Adaptation", describes one GPU kernel, the
+ * streamed and tensor-core GEMVs are this library's designs for B200, and the
+ * lookup-table GEMV follows the bitnet.cpp CPU kernels (dignews article on the
+ * release, section 3: lookup tables after T-MAC, lossless).
  *   kind   a bl_gemv_kernel value
  * Returns the previous selection, or -1 (and changes nothing) for an unknown kind.
  * Host only, no CUDA call.

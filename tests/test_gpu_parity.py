@@ -518,9 +518,51 @@ def test_gemv_kernel_choice_gives_the_same_bits(cuda_device):
     Wp, gamma = bl.pack_weights(W.to(cuda_device))
     x = synth.activations(M, K, seed=4701, outliers=True).to(cuda_device)
     outs = []
-    for kind in (bl.BL_GEMV_STREAM, bl.BL_GEMV_TENSOR, bl.BL_GEMV_AUTO):
+    for kind in (bl.BL_GEMV_STREAM, bl.BL_GEMV_TENSOR, bl.BL_GEMV_LUT, bl.BL_GEMV_AUTO):
         with bl.gemv_kernel(kind):
             y, acc = bl.forward(Wp, gamma, x, want_acc=True)
         outs.append((bits(y), np_(acc)))
     for y, acc in outs[1:]:
         assert np.array_equal(acc, outs[0][1]) and np.array_equal(y, outs[0][0])
+
+
+# ----------------------------------------------------------------------------- lookup-table GEMV (M <= 16)
+
+@pytest.mark.parametrize("M", [1, 2, 3, 4, 5, 16])
+@pytest.mark.parametrize("K,N", [(2560, 6912), (6912, 2560), (2560, 640), (256, 136), (13056, 33)])
+def test_forward_gemv_lookup_table(cuda_device, K, N, M):
+    """The T-MAC-style lookup-table GEMV, forced on: table segments of 128-768
+    words with a partial last chunk (K = 2560: 160 words; 6912: 432), several
+    segments (K = 13056 at one token: 816 words), one to four launches of up to
+    four tokens, residual and the int32 dump."""
+    W = make_weights(N, K, 0.02, seed=5000 + K + N)
+    Wp, gamma, Wp_ref, g_ref = pack_both(W, cuda_device)
+    x = synth.activations(M, K, seed=5100 + M, outliers=True)
+    res = synth.activations(M, N, seed=5200 + M, outliers=False)
+    with bl.gemv_kernel(bl.BL_GEMV_LUT):
+        check_forward_full(Wp, gamma, Wp_ref, g_ref, x, cuda_device, residual=res)
+    assert bl.get_device_error() == 0
+
+
+@pytest.mark.parametrize("M", [1, 4])
+@pytest.mark.parametrize("K,N", [(8192, 28672), (28672, 8192)])
+def test_forward_gemv_lookup_table_100b_sampled(cuda_device, K, N, M):
+    W = make_weights(N, K, synth.SIGMA_100B, seed=5300 + K)
+    Wp, gamma, Wp_ref, g_ref = pack_both(W, cuda_device)
+    x = synth.activations(M, K, seed=5400 + M, outliers=True)
+    rows = sample_indices(N, 256, seed=M + 13)
+    with bl.gemv_kernel(bl.BL_GEMV_LUT):
+        check_forward_sampled(Wp, gamma, Wp_ref, g_ref, x, cuda_device, rows, np.arange(M))
+
+
+def test_forward_gemv_lookup_table_rowwise(cuda_device):
+    K, N, M = 2560, 1000, 3
+    W = make_weights(N, K, 0.02, seed=5500)
+    Wp, g = bl.pack_weights_rowwise(W.to(cuda_device))
+    Wp_ref, g_ref = oracle.pack_weights_rowwise(bits(W))
+    x = synth.activations(M, K, seed=5501, outliers=True)
+    with bl.gemv_kernel(bl.BL_GEMV_LUT):
+        y, acc = bl.forward_rowwise(Wp, g, x.to(cuda_device), want_acc=True)
+    ref = oracle.forward_rowwise(Wp_ref, g_ref, bits(x))
+    assert np.array_equal(np_(acc), ref["acc"])
+    assert_bf16_exact(bits(y), ref["y"])
