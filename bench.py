@@ -286,9 +286,13 @@ def run_ours(args):
                 "bytes_per_launch": step_bytes // (LAYERS * len(DECODE_SHAPES)),
                 "peak_kind": peak_kind}
 
+    # the tensor-parallel FFN runs on every rank (its collectives need them all)
+    tp_extra = run_tp_extra(bl, synth, dev, rank, world, barrier, max_over_ranks) if world > 1 else None
     extras = {}
     if rank == 0 and not args.no_extras:
         extras = run_extras(args, bl, synth, dev, hbm_peak, int8_peak)
+    if tp_extra is not None:
+        extras["ffn_tp"] = tp_extra
 
     # ---- end to end through the public API with host buffers
     e2e = run_e2e(args, bl, dev, graph, xs, ys, step_bytes, world, barrier, max_over_ranks)
@@ -550,6 +554,54 @@ def run_extras(args, bl, synth, dev, hbm_peak, int8_peak):
     out["decoder_linears_2b_30_layers"] = linears
     del layers, dec
     torch.cuda.empty_cache()
+    return out
+
+
+def run_tp_extra(bl, synth, dev, rank, world, barrier, max_over_ranks, layers: int = 4):
+    """The FFN sub-layer split over the ranks (bitlinear_w1_a8_02_b200.tp): d = 2560,
+    f = 6912, each rank owning its shard of the hidden width, NCCL exchanges of the
+    subln statistics and the int32 accumulators; `layers` layers chained, at
+    M = 1 and 512. Device time on each rank, the max over ranks reported."""
+    import torch
+
+    from bitlinear_w1_a8_02_b200 import tp
+
+    d, f = 2560, 6912
+    c0, c1 = tp.shard_range(f, world, rank)
+    shards = []
+    for layer in range(layers):
+        sg, su, sd = synth.ffn_layer_seeds(layer)
+        Wg = synth.weights(f, d, synth.SIGMA_2B, sg, device=dev)
+        Wu = synth.weights(f, d, synth.SIGMA_2B, su, device=dev)
+        Wd = synth.weights(d, f, synth.SIGMA_2B, sd, device=dev)
+        shards.append(tp.pack_ffn_shard(Wg[c0:c1].contiguous(), Wu[c0:c1].contiguous(), Wd[:, c0:c1].contiguous(),
+                                        f, c0, c1))
+        del Wg, Wu, Wd
+    out = {"world": world, "shard_columns": [c0, c1], "layers": layers}
+    for M in (1, 512):
+        h0 = synth.activations(M, d, seed=1, outliers=False, device=dev)
+
+        def run():
+            h = h0
+            for sh in shards:
+                h = tp.ffn_tp(sh, h, residual=h)
+            return h
+        for _ in range(3):
+            run()
+        torch.cuda.synchronize()
+        barrier()
+        reps = 10
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(reps):
+            run()
+        b.record()
+        torch.cuda.synchronize()
+        ms = max_over_ranks(a.elapsed_time(b) / reps)
+        out[f"M{M}"] = {"ms_per_step": round(ms, 4), "us_per_layer": round(ms * 1e3 / layers, 2)}
+    torch.cuda.synchronize()
+    barrier()
     return out
 
 

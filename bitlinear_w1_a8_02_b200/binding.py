@@ -23,7 +23,7 @@ STATUS_NAMES = {
     9: "BL_ERR_BAD_CODE",
 }
 BL_BF16, BL_FP32 = 0, 1
-BL_OP_PACK, BL_OP_FORWARD, BL_OP_FFN, BL_OP_VALIDATE = 0, 1, 2, 3
+BL_OP_PACK, BL_OP_FORWARD, BL_OP_FFN, BL_OP_VALIDATE, BL_OP_FFN_TP_UP, BL_OP_FFN_TP_DOWN = 0, 1, 2, 3, 4, 5
 BL_GEMV_AUTO, BL_GEMV_STREAM, BL_GEMV_TENSOR, BL_GEMV_LUT = 0, 1, 2, 3
 
 # Every symbol include/bitlinear.h declares, with (restype, argtypes).
@@ -47,6 +47,11 @@ SIGNATURES = {
     "bitlinear_get_device_error": (_ST, [_P]),
     "bitlinear_selftest_timeout": (_ST, [_I, _P]),
     "bitlinear_set_gemv_kernel": (ctypes.c_int, [ctypes.c_int]),
+    "bitlinear_absmean_sum": (_ST, [_P, ctypes.c_int, _I, _I, _P, _P, _S, _P]),
+    "bitlinear_pack_weights_global": (_ST, [_P, ctypes.c_int, _I, _I, _P, _I, _P, _P, _P]),
+    "bitlinear_ffn_tp_up": (_ST, [_P, _P, _P, _P, _I, _I, _P, _I, _P, _P, _P, _P, _S, _P]),
+    "bitlinear_ffn_tp_down": (_ST, [_P, _I, _I, _I, _P, _I, _P, _P, _P, _P, _P, _S, _P]),
+    "bitlinear_ffn_tp_finish": (_ST, [_P, _P, _P, _P, _P, _I, _I, _P]),
 }
 
 
@@ -304,3 +309,91 @@ class gemv_kernel:
     def __exit__(self, *exc):
         set_gemv_kernel(self.prev)
         return False
+
+
+# ----------------------------------------------------------------------------- tensor-parallel pieces
+
+def _wdt(W: torch.Tensor) -> int:
+    if W.dtype == torch.bfloat16:
+        return BL_BF16
+    if W.dtype == torch.float32:
+        return BL_FP32
+    raise ValueError("W must be bf16 or fp32")
+
+
+def absmean_sum(W: torch.Tensor) -> torch.Tensor:
+    """fp64 sum of |W| of one weight shard [N, K]: a device float64 tensor [1]."""
+    _cuda(W, "W")
+    N, K = W.shape
+    out = torch.empty(1, dtype=torch.float64, device=W.device)
+    ws = _WS.get(W.device, workspace_bytes(BL_OP_PACK, 0, N, K))
+    st = lib().bitlinear_absmean_sum(_ptr(W), _wdt(W), N, K, _ptr(out), _ptr(ws), ws.numel(), _stream(W.device))
+    _check(st, "bitlinear_absmean_sum")
+    return out
+
+
+def pack_weights_global(W: torch.Tensor, total_sum: torch.Tensor, total_count: int):
+    """Pack a shard [N, K] with gamma = fp32(total_sum / total_count) of the whole
+    tensor (total_sum: device float64 [1]) -> (Wp uint8 [N, K/4], gamma fp32 [1])."""
+    _cuda(W, "W")
+    _cuda(total_sum, "total_sum", torch.float64)
+    N, K = W.shape
+    Wp = torch.empty((N, K // 4), dtype=torch.uint8, device=W.device)
+    gamma = torch.empty(1, dtype=torch.float32, device=W.device)
+    st = lib().bitlinear_pack_weights_global(_ptr(W), _wdt(W), N, K, _ptr(total_sum), int(total_count), _ptr(Wp),
+                                             _ptr(gamma), _stream(W.device))
+    _check(st, "bitlinear_pack_weights_global")
+    return Wp, gamma
+
+
+def ffn_tp_up(Wg, gg, Wu, gu, x: torch.Tensor):
+    """Rank-local gate/up of the FFN: (h fp32 [M, f_local], ss fp64 [M], hmax fp32 [M])."""
+    _cuda(x, "x", torch.bfloat16)
+    M, d = x.shape
+    fl = Wg.shape[0]
+    for t, name in ((Wg, "Wg"), (Wu, "Wu")):
+        _cuda(t, name, torch.uint8)
+    if Wg.shape != (fl, d // 4) or Wu.shape != (fl, d // 4):
+        raise ValueError("gate / up shard shapes do not match x")
+    h = torch.empty((M, fl), dtype=torch.float32, device=x.device)
+    ss = torch.empty(M, dtype=torch.float64, device=x.device)
+    hmax = torch.empty(M, dtype=torch.float32, device=x.device)
+    ws = _WS.get(x.device, workspace_bytes(BL_OP_FFN_TP_UP, M, fl, d))
+    st = lib().bitlinear_ffn_tp_up(_ptr(Wg), _ptr(gg), _ptr(Wu), _ptr(gu), d, fl, _ptr(x), M, _ptr(h), _ptr(ss),
+                                   _ptr(hmax), _ptr(ws), ws.numel(), _stream(x.device))
+    _check(st, "bitlinear_ffn_tp_up")
+    return h, ss, hmax
+
+
+def ffn_tp_down(Wd, h: torch.Tensor, ss_all: torch.Tensor, hmax_all: torch.Tensor, f_total: int):
+    """Rank-local requantisation (global statistics) and partial down projection:
+    (acc int32 [M, d], s2 fp32 [M])."""
+    _cuda(Wd, "Wd", torch.uint8)
+    _cuda(h, "h", torch.float32)
+    _cuda(ss_all, "ss_all", torch.float64)
+    _cuda(hmax_all, "hmax_all", torch.float32)
+    M, fl = h.shape
+    d = Wd.shape[0]
+    if Wd.shape != (d, fl // 4):
+        raise ValueError("down shard shape does not match h")
+    acc = torch.empty((M, d), dtype=torch.int32, device=h.device)
+    s2 = torch.empty(M, dtype=torch.float32, device=h.device)
+    ws = _WS.get(h.device, workspace_bytes(BL_OP_FFN_TP_DOWN, M, d, fl))
+    st = lib().bitlinear_ffn_tp_down(_ptr(Wd), d, fl, int(f_total), _ptr(h), M, _ptr(ss_all), _ptr(hmax_all),
+                                     _ptr(acc), _ptr(s2), _ptr(ws), ws.numel(), _stream(h.device))
+    _check(st, "bitlinear_ffn_tp_down")
+    return acc, s2
+
+
+def ffn_tp_finish(acc: torch.Tensor, gd, s2: torch.Tensor, residual: Optional[torch.Tensor] = None,
+                  out: Optional[torch.Tensor] = None):
+    """y = bf16([residual +] acc * (gd / s2)) on the accumulators summed over the ranks."""
+    _cuda(acc, "acc", torch.int32)
+    M, d = acc.shape
+    if residual is not None:
+        _cuda(residual, "residual", torch.bfloat16)
+    y = torch.empty((M, d), dtype=torch.bfloat16, device=acc.device) if out is None else out
+    st = lib().bitlinear_ffn_tp_finish(_ptr(acc), _ptr(gd), _ptr(s2), _ptr(residual), _ptr(y), M, d,
+                                       _stream(acc.device))
+    _check(st, "bitlinear_ffn_tp_finish")
+    return y

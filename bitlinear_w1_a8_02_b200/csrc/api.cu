@@ -67,6 +67,39 @@ inline FfnWs ffn_ws(int64_t M, int64_t f, int64_t d) {
     return w;
 }
 
+// Tensor-parallel FFN pieces. Up (sizes M, fl, d): codes of x, then g and u of
+// the rank's fl columns (fp32). Down (sizes M, d, fl): codes of the rank's
+// columns, their sums, and fp32 scratch for the projection's discarded dequantised
+// output (only its int32 accumulators are kept).
+struct TpUpWs {
+    size_t xq, scale, xsum, g, u, sk, sk_bytes, total;
+};
+inline TpUpWs tp_up_ws(int64_t M, int64_t fl, int64_t d) {
+    TpUpWs w;
+    w.xq = 0;
+    w.scale = align_up((size_t)(M * d));
+    w.xsum = w.scale + align_up((size_t)M * 4);
+    w.g = w.xsum + align_up((size_t)M * 4);
+    w.u = w.g + align_up((size_t)(M * fl) * 4);
+    w.sk = w.u + align_up((size_t)(M * fl) * 4);
+    w.sk_bytes = sk_bytes(M);
+    w.total = w.sk + w.sk_bytes;
+    return w;
+}
+struct TpDownWs {
+    size_t q2, xsum2, y32, sk, sk_bytes, total;
+};
+inline TpDownWs tp_down_ws(int64_t M, int64_t d, int64_t fl) {
+    TpDownWs w;
+    w.q2 = 0;
+    w.xsum2 = align_up((size_t)(M * fl));
+    w.y32 = w.xsum2 + align_up((size_t)M * 4);
+    w.sk = w.y32 + align_up((size_t)(M * d) * 4);
+    w.sk_bytes = sk_bytes(M);
+    w.total = w.sk + w.sk_bytes;
+    return w;
+}
+
 inline size_t pack_ws(int64_t N, int64_t K) {
     return align_up((size_t)bl::absmean_blocks(N * K) * sizeof(double));
 }
@@ -192,6 +225,8 @@ BL_API size_t bitlinear_workspace_bytes(int op, int64_t M, int64_t N, int64_t K)
         case BL_OP_FORWARD: return forward_ws(M, K).total;
         case BL_OP_FFN: return ffn_ws(M, N, K).total;
         case BL_OP_VALIDATE: return kWsAlign;
+        case BL_OP_FFN_TP_UP: return tp_up_ws(M, N, K).total;
+        case BL_OP_FFN_TP_DOWN: return tp_down_ws(M, N, K).total;
         default: return 0;
     }
 }
@@ -422,4 +457,101 @@ BL_API bl_status bitlinear_get_device_error(bl_stream_t stream) {
     unsigned v = 0;
     if (bl::read_and_clear_device_error(&v) != cudaSuccess) return BL_ERR_CUDA;
     return v ? BL_ERR_TIMEOUT : BL_OK;
+}
+
+// ---------------------------------------------------------------- tensor-parallel pieces
+
+BL_API bl_status bitlinear_absmean_sum(const void* W, int wdt, int64_t N, int64_t K, double* sum, void* ws,
+                                       size_t ws_bytes, bl_stream_t stream) {
+    if (wdt != BL_BF16 && wdt != BL_FP32) return BL_ERR_DTYPE;
+    if (N < 1 || K < 4 || K % 4 != 0 || N > kMaxN || K > kMaxK) return BL_ERR_SHAPE;
+    if (!W || !sum) return BL_ERR_NULL;
+    if (!aligned(W, 16) || !aligned(sum, 8)) return BL_ERR_ALIGN;
+    if (bl_status st = check_ws(ws, ws_bytes, pack_ws(N, K))) return st;
+    if (bl_status st = check_device()) return st;
+    return cuda_status(bl::launch_absmean_sum(W, wdt == BL_FP32, N * K, (double*)ws, sum, (cudaStream_t)stream));
+}
+
+BL_API bl_status bitlinear_pack_weights_global(const void* W, int wdt, int64_t N, int64_t K, const double* total_sum,
+                                               int64_t total_count, uint8_t* Wp, float* gamma, bl_stream_t stream) {
+    if (wdt != BL_BF16 && wdt != BL_FP32) return BL_ERR_DTYPE;
+    if (N < 1 || K < 4 || K % 4 != 0 || N > kMaxN || K > kMaxK || total_count < N * K) return BL_ERR_SHAPE;
+    if (!W || !total_sum || !Wp || !gamma) return BL_ERR_NULL;
+    if (!aligned(W, 16) || !aligned(total_sum, 8) || !aligned(gamma, 4)) return BL_ERR_ALIGN;
+    if (bl_status st = check_device()) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    BL_TRY(bl::launch_gamma_from_sum(total_sum, total_count, gamma, s));
+    BL_TRY(bl::launch_ternary_pack(W, wdt == BL_FP32, N, K, gamma, Wp, s));
+    return BL_OK;
+}
+
+BL_API bl_status bitlinear_ffn_tp_up(const uint8_t* Wg, const float* gg, const uint8_t* Wu, const float* gu,
+                                     int64_t d, int64_t fl, const uint16_t* x, int64_t M, float* h, double* ss,
+                                     float* hmax, void* ws, size_t ws_bytes, bl_stream_t stream) {
+    if (M < 0 || M > kMaxM || d < 4 || d % 4 != 0 || fl < 4 || fl % 4 != 0 || d > kMaxK || fl > kMaxN)
+        return BL_ERR_SHAPE;
+    if (M == 0) return BL_OK;
+    if (!Wg || !gg || !Wu || !gu || !x || !h || !ss || !hmax) return BL_ERR_NULL;
+    if (!aligned(gg, 4) || !aligned(gu, 4) || !aligned(x, 2) || !aligned(h, 4) || !aligned(ss, 8) ||
+        !aligned(hmax, 4))
+        return BL_ERR_ALIGN;
+    const TpUpWs w = tp_up_ws(M, fl, d);
+    if (bl_status st = check_ws(ws, ws_bytes, w.total)) return st;
+    if (bl_status st = check_device()) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    char* base = (char*)ws;
+    int8_t* xq = (int8_t*)(base + w.xq);
+    float* scale = (float*)(base + w.scale);
+    int32_t* xsum = (int32_t*)(base + w.xsum);
+    float* g = (float*)(base + w.g);
+    float* u = (float*)(base + w.u);
+    Path up = choose_path(Wg, fl, d, M, xq, x);  // gate and up share the codes, so a path
+    if (choose_path(Wu, fl, d, M, xq, x) != up) up = Path::GemvGeneric;
+    BL_TRY(bl::launch_act_quant(x, M, d, layout_of(up), xq, scale, xsum, s));
+    bl::GemvOut og;
+    og.y32 = g;
+    bl::GemvOut ou;
+    ou.y32 = u;
+    if (bl_status st = project(up, Wg, gg, fl, d, xq, scale, xsum, M, og, s, base + w.sk, w.sk_bytes)) return st;
+    if (bl_status st = project(up, Wu, gu, fl, d, xq, scale, xsum, M, ou, s, base + w.sk, w.sk_bytes)) return st;
+    return cuda_status(bl::launch_ffn_tp_hstats(g, u, M, fl, h, ss, hmax, s));
+}
+
+BL_API bl_status bitlinear_ffn_tp_down(const uint8_t* Wd, int64_t d, int64_t fl, int64_t f_total, const float* h,
+                                       int64_t M, const double* ss_all, const float* hmax_all, int32_t* acc,
+                                       float* s2, void* ws, size_t ws_bytes, bl_stream_t stream) {
+    if (M < 0 || M > kMaxM || d < 1 || d > kMaxN || fl < 4 || fl % 4 != 0 || fl > kMaxK || f_total < fl)
+        return BL_ERR_SHAPE;
+    if (M == 0) return BL_OK;
+    if (!Wd || !h || !ss_all || !hmax_all || !acc || !s2) return BL_ERR_NULL;
+    if (!aligned(h, 4) || !aligned(ss_all, 8) || !aligned(hmax_all, 4) || !aligned(acc, 4) || !aligned(s2, 4))
+        return BL_ERR_ALIGN;
+    const TpDownWs w = tp_down_ws(M, d, fl);
+    if (bl_status st = check_ws(ws, ws_bytes, w.total)) return st;
+    if (bl_status st = check_device()) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    char* base = (char*)ws;
+    int8_t* q2 = (int8_t*)(base + w.q2);
+    int32_t* xsum2 = (int32_t*)(base + w.xsum2);
+    const Path down = choose_path(Wd, d, fl, M, q2, nullptr);
+    BL_TRY(bl::launch_ffn_tp_requant(h, M, fl, f_total, ss_all, hmax_all, layout_of(down), q2, s2, xsum2, s));
+    // the projection dequantises into scratch (s2 stands in for gamma there: that
+    // output is discarded); the partial sums over the rank's columns go to acc
+    bl::GemvOut od;
+    od.y32 = (float*)(base + w.y32);
+    od.acc = acc;
+    return project(down, Wd, s2, d, fl, q2, s2, xsum2, M, od, s, base + w.sk, w.sk_bytes);
+}
+
+BL_API bl_status bitlinear_ffn_tp_finish(const int32_t* acc, const float* gd, const float* s2,
+                                         const uint16_t* residual, uint16_t* y, int64_t M, int64_t d,
+                                         bl_stream_t stream) {
+    if (M < 0 || M > kMaxM || d < 0 || d > kMaxN) return BL_ERR_SHAPE;
+    if (M == 0 || d == 0) return BL_OK;
+    if (!acc || !gd || !s2 || !y) return BL_ERR_NULL;
+    if (!aligned(acc, 4) || !aligned(gd, 4) || !aligned(s2, 4) || !aligned(y, 2) ||
+        (residual && !aligned(residual, 2)))
+        return BL_ERR_ALIGN;
+    if (bl_status st = check_device()) return st;
+    return cuda_status(bl::launch_ffn_tp_finish(acc, gd, s2, residual, y, M, d, (cudaStream_t)stream));
 }

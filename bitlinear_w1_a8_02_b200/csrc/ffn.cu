@@ -9,6 +9,13 @@
 //   q2, s2 = per-token absmax int8 quantisation of hn (as for x)
 //
 // One CTA per token; h is kept in shared memory between the passes.
+//
+// Tensor-parallel pieces (a rank owns fl of the f hidden columns; the pages give
+// no distributed detail, this is the library's split): h with the rank's share
+// of the per-token statistics sum h^2 and max |h|; the requantisation of the
+// rank's columns once those statistics are summed / maximised over the ranks;
+// and the dequantisation of the down projection's int32 accumulators once they
+// are summed over the ranks.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -90,6 +97,106 @@ __global__ void __launch_bounds__(kThreads) ffn_finalise_kernel(const float* __r
     }
 }
 
+// ---------------------------------------------------------------- tensor-parallel pieces
+// A rank owns fl of the f hidden columns. Its h, and per token its share of the
+// subln statistics: ss = sum_j h_j^2 (fp64, fixed order: thread strides, warp
+// butterfly, warps in index order) and hmax = max_j |h_j|.
+__global__ void __launch_bounds__(kThreads) ffn_tp_hstats_kernel(const float* __restrict__ g,
+                                                                  const float* __restrict__ u, int fl,
+                                                                  float* __restrict__ h, double* __restrict__ ss,
+                                                                  float* __restrict__ hmax) {
+    __shared__ double dscratch[kWarps];
+    __shared__ float fscratch[kWarps];
+    grid_dependency_wait();
+    grid_dependents_launch();
+    const int m = blockIdx.x;
+    double acc = 0.0;
+    float mx = 0.0f;
+    for (int j = threadIdx.x; j < fl; j += kThreads) {
+        const float gv = g[(size_t)m * fl + j];
+        const float t = gv > 0.0f ? gv : 0.0f;
+        const float hv = __fmul_rn(__fmul_rn(t, t), u[(size_t)m * fl + j]);
+        h[(size_t)m * fl + j] = hv;
+        acc = __dadd_rn(acc, __dmul_rn((double)hv, (double)hv));
+        mx = fmaxf(mx, fabsf(hv));
+    }
+    acc = block_sum<kWarps>(acc, dscratch);
+    mx = block_max<kWarps>(mx, fscratch);
+    if (threadIdx.x == 0) {
+        ss[m] = acc;
+        hmax[m] = mx;
+    }
+}
+
+// Requantisation of a rank's columns with the statistics of all ranks:
+// r = 1 / sqrtf(float(ss_all / f_total) + 1e-5), s2 = 127 / max(fl(hmax_all r), 1e-5)
+// (the largest |fl(h_j r)| of the whole row: rounding is monotonic and r > 0),
+// codes of fl(h_j r) in the consumer's layout, and their sum over the rank's columns.
+template <int LAYOUT>
+__global__ void __launch_bounds__(kThreads) ffn_tp_requant_kernel(const float* __restrict__ h, int fl, int64_t f_total,
+                                                                   const double* __restrict__ ss_all,
+                                                                   const float* __restrict__ hmax_all,
+                                                                   int8_t* __restrict__ q2, float* __restrict__ s2,
+                                                                   int32_t* __restrict__ xsum2) {
+    __shared__ int iscratch[kWarps];
+    grid_dependency_wait();
+    grid_dependents_launch();
+    const int m = blockIdx.x;
+    const float ms = __double2float_rn(__ddiv_rn(ss_all[m], (double)f_total));
+    const float r = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, kRmsEps)));
+    const float s = __fdiv_rn(kActRange, fmaxf(__fmul_rn(hmax_all[m], r), kActEps));
+    const float* hr = h + (size_t)m * fl;
+    int sum = 0;
+    if (LAYOUT == XQ_NATURAL) {
+        for (int j = threadIdx.x; j < fl; j += kThreads) {
+            const int q = quant_code(__fmul_rn(hr[j], r), s);
+            q2[(size_t)m * fl + j] = (int8_t)q;
+            sum += q;
+        }
+    } else {
+        const int fb = fl / 4;
+        for (int c = threadIdx.x; c < fl / 16; c += kThreads) {
+            unsigned w[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+            for (int b = 0; b < 4; ++b)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int q = quant_code(__fmul_rn(hr[16 * c + 4 * b + i], r), s);
+                    sum += q;
+                    w[i] |= (unsigned)(q & 255) << (8 * b);
+                }
+            if (LAYOUT == XQ_G16T) {
+                reinterpret_cast<uint4*>(q2 + (size_t)m * fl)[c] = make_uint4(w[0], w[1], w[2], w[3]);
+            } else {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) reinterpret_cast<unsigned*>(q2 + ((size_t)m * 4 + i) * fb)[c] = w[i];
+            }
+        }
+    }
+    sum = block_sum<kWarps>(sum, iscratch);
+    if (threadIdx.x == 0) {
+        s2[m] = s;
+        xsum2[m] = sum;
+    }
+}
+
+// y = bf16([residual +] float(acc) * (gd / s2)) on the accumulators summed over the ranks.
+__global__ void __launch_bounds__(kThreads) ffn_tp_finish_kernel(const int32_t* __restrict__ acc,
+                                                                  const float* __restrict__ gd,
+                                                                  const float* __restrict__ s2,
+                                                                  const uint16_t* __restrict__ residual,
+                                                                  uint16_t* __restrict__ y, int64_t M, int64_t d) {
+    grid_dependency_wait();
+    const float gamma = *gd;
+    const int64_t n = M * d;
+    for (int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x; i < n; i += (int64_t)gridDim.x * kThreads) {
+        const int64_t m = i / d;
+        float v = dequant(acc[i], __fdiv_rn(gamma, s2[m]));
+        if (residual) v = __fadd_rn(bf16_bits_to_f32(residual[i]), v);
+        y[i] = f32_to_bf16_bits(v);
+    }
+}
+
 template <int LAYOUT>
 cudaError_t launch_fin(const float* g, const float* u, int64_t M, int64_t f, int8_t* q2, float* s2,
                        int32_t* xsum2, cudaStream_t s) {
@@ -104,6 +211,37 @@ cudaError_t launch_fin(const float* g, const float* u, int64_t M, int64_t f, int
 }
 
 }  // namespace
+
+cudaError_t launch_ffn_tp_hstats(const float* g, const float* u, int64_t M, int64_t fl, float* h, double* ss,
+                                 float* hmax, cudaStream_t s) {
+    if (M == 0) return cudaSuccess;
+    return launch_pdl(ffn_tp_hstats_kernel, dim3((unsigned)M), dim3(kThreads), 0, s, g, u, (int)fl, h, ss, hmax);
+}
+
+cudaError_t launch_ffn_tp_requant(const float* h, int64_t M, int64_t fl, int64_t f_total, const double* ss_all,
+                                  const float* hmax_all, int layout, int8_t* q2, float* s2, int32_t* xsum2,
+                                  cudaStream_t s) {
+    if (M == 0) return cudaSuccess;
+    if (layout != XQ_NATURAL && fl % 16 != 0) return cudaErrorInvalidValue;
+    const dim3 g((unsigned)M), b(kThreads);
+    if (layout == XQ_PLANES)
+        return launch_pdl(ffn_tp_requant_kernel<XQ_PLANES>, g, b, 0, s, h, (int)fl, f_total, ss_all, hmax_all, q2, s2,
+                          xsum2);
+    if (layout == XQ_G16T)
+        return launch_pdl(ffn_tp_requant_kernel<XQ_G16T>, g, b, 0, s, h, (int)fl, f_total, ss_all, hmax_all, q2, s2,
+                          xsum2);
+    return launch_pdl(ffn_tp_requant_kernel<XQ_NATURAL>, g, b, 0, s, h, (int)fl, f_total, ss_all, hmax_all, q2, s2,
+                      xsum2);
+}
+
+cudaError_t launch_ffn_tp_finish(const int32_t* acc, const float* gd, const float* s2, const uint16_t* residual,
+                                 uint16_t* y, int64_t M, int64_t d, cudaStream_t s) {
+    if (M == 0 || d == 0) return cudaSuccess;
+    int64_t blocks = (M * d + kThreads - 1) / kThreads;
+    if (blocks > 148 * 16) blocks = 148 * 16;
+    return launch_pdl(ffn_tp_finish_kernel, dim3((unsigned)blocks), dim3(kThreads), 0, s, acc, gd, s2, residual, y,
+                      M, d);
+}
 
 cudaError_t launch_ffn_finalise(const float* g, const float* u, int64_t M, int64_t f, int layout,
                                 int8_t* q2, float* s2, int32_t* xsum2, cudaStream_t s) {

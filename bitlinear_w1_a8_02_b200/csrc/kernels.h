@@ -20,6 +20,10 @@ cudaError_t launch_absmean_rows(const void* W, bool fp32, int64_t N, int64_t K, 
 cudaError_t launch_count_bad_codes(const uint8_t* Wp, int64_t nbytes, unsigned long long* count,
                                    cudaStream_t s);
 
+// fp64 sum of |W| of one shard (absmean term), and gamma = fp32(total / count)
+cudaError_t launch_absmean_sum(const void* W, bool fp32, int64_t n, double* partial, double* sum, cudaStream_t s);
+cudaError_t launch_gamma_from_sum(const double* total_sum, int64_t count, float* gamma, cudaStream_t s);
+
 // ---- activation quantisation (actquant.cu); layout is an XqLayout
 // rmsnorm: quantise fl(x * r), r = 1 / sqrtf(float(sum_k x^2 / K) + 1e-5) per token
 // (unit-weight RMSNorm, sum in fp64), instead of x.
@@ -113,6 +117,15 @@ cudaError_t launch_gemv_lut(const uint8_t* Wp, const float* gamma, int64_t N, in
 // h = relu(g)^2 * u; hn = subln(h); q2, s2, xsum2 = quant(hn) in `layout`.
 cudaError_t launch_ffn_finalise(const float* g, const float* u, int64_t M, int64_t f, int layout,
                                 int8_t* q2, float* s2, int32_t* xsum2, cudaStream_t s);
+
+// tensor-parallel FFN pieces (ffn.cu): a rank owns fl of the f hidden columns
+cudaError_t launch_ffn_tp_hstats(const float* g, const float* u, int64_t M, int64_t fl, float* h, double* ss,
+                                 float* hmax, cudaStream_t s);
+cudaError_t launch_ffn_tp_requant(const float* h, int64_t M, int64_t fl, int64_t f_total, const double* ss_all,
+                                  const float* hmax_all, int layout, int8_t* q2, float* s2, int32_t* xsum2,
+                                  cudaStream_t s);
+cudaError_t launch_ffn_tp_finish(const int32_t* acc, const float* gd, const float* s2, const uint16_t* residual,
+                                 uint16_t* y, int64_t M, int64_t d, cudaStream_t s);
 
 // ---- device error word: set by bounded waits inside kernels that give up.
 // Address of the current device's word (for kernels), and a host read that

@@ -47,6 +47,20 @@ __global__ void absmean_final_kernel(const double* __restrict__ partial, int nbl
     if (threadIdx.x == 0) *gamma = __double2float_rn(__ddiv_rn(acc, (double)n));
 }
 
+// The fp64 sum itself (one shard's term of a per-tensor absmean split over ranks).
+__global__ void absmean_sum_kernel(const double* __restrict__ partial, int nblocks, double* __restrict__ sum) {
+    double acc = 0.0;
+    for (int i = threadIdx.x; i < nblocks; i += 32) acc = __dadd_rn(acc, partial[i]);
+    acc = warp_sum(acc);
+    if (threadIdx.x == 0) *sum = acc;
+}
+
+// gamma of a whole tensor from the fp64 sum and the count of all its shards.
+__global__ void gamma_from_sum_kernel(const double* __restrict__ total_sum, int64_t count,
+                                      float* __restrict__ gamma) {
+    *gamma = __double2float_rn(__ddiv_rn(*total_sum, (double)count));
+}
+
 // Per-row absmean: one CTA per row, fp64 sum in a fixed order (thread strides,
 // warp butterfly, warps in index order).
 template <bool FP32>
@@ -128,6 +142,21 @@ cudaError_t launch_absmean(const void* W, bool fp32, int64_t n, double* partial,
     else
         absmean_partial_kernel<false><<<g, kPackThreads, 0, s>>>(W, n, partial);
     absmean_final_kernel<<<1, 32, 0, s>>>(partial, g, n, gamma);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_absmean_sum(const void* W, bool fp32, int64_t n, double* partial, double* sum, cudaStream_t s) {
+    const int g = absmean_blocks(n);
+    if (fp32)
+        absmean_partial_kernel<true><<<g, kPackThreads, 0, s>>>(W, n, partial);
+    else
+        absmean_partial_kernel<false><<<g, kPackThreads, 0, s>>>(W, n, partial);
+    absmean_sum_kernel<<<1, 32, 0, s>>>(partial, g, sum);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gamma_from_sum(const double* total_sum, int64_t count, float* gamma, cudaStream_t s) {
+    gamma_from_sum_kernel<<<1, 1, 0, s>>>(total_sum, count, gamma);
     return cudaGetLastError();
 }
 

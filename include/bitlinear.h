@@ -74,7 +74,9 @@ typedef enum {
     BL_OP_PACK = 0,     /* sizes: N, K of the weight */
     BL_OP_FORWARD = 1,  /* sizes: M, N, K */
     BL_OP_FFN = 2,      /* sizes: M, N = f (hidden), K = d (model width) */
-    BL_OP_VALIDATE = 3  /* sizes ignored */
+    BL_OP_VALIDATE = 3, /* sizes ignored */
+    BL_OP_FFN_TP_UP = 4,    /* sizes: M, N = f_local (the rank's hidden columns), K = d */
+    BL_OP_FFN_TP_DOWN = 5   /* sizes: M, N = d, K = f_local */
 } bl_op;
 
 /* Kernels for M <= 16 tokens (bitlinear_set_gemv_kernel). */
@@ -279,6 +281,67 @@ bl_status bitlinear_forward_noalloc(const uint8_t* Wp, const float* gamma, int64
  * Host only, no CUDA call.
  */
 int bitlinear_set_gemv_kernel(int kind);
+
+/*
+ * Tensor-parallel pieces of the FFN sub-layer. The pages give no distributed
+ * detail (paper card "BitNet b1.58 2B4T Technical Report", "Limits"); this is
+ * the library's split of bitlinear_ffn over P ranks (one GPU each): rank r owns
+ * f_local of the f hidden columns, i.e. those rows of the gate and up weights
+ * and those columns of the down weight, packed with the gammas of the whole
+ * tensors. Per layer, between the calls, the caller exchanges (NCCL over
+ * NVLink, or any transport): the per-token sums ss (fp64, sum) and maxima hmax
+ * (fp32, max) after bitlinear_ffn_tp_up, and the int32 accumulators (sum, exact
+ * in any order) after bitlinear_ffn_tp_down. The result equals bitlinear_ffn on
+ * the whole weights bit for bit, up to the order of the fp64 sum of the ranks'
+ * ss (a different fp32 subln factor needs those sums to straddle an fp32
+ * rounding boundary).
+ *
+ * Packing a shard: the per-tensor gamma of the paper card's absmean ("Method
+ * Adaptation") is over the whole tensor, so each rank adds its fp64 sum of |W|
+ * (bitlinear_absmean_sum, into a device double) to the others' and packs its
+ * shard with that total (bitlinear_pack_weights_global).
+ */
+
+/* fp64 sum of |W| over one shard [N, K] of a weight tensor (bf16 or fp32, as
+ * bitlinear_pack_weights), written to *sum (device, 8-byte aligned), in a fixed
+ * order. ws: bitlinear_workspace_bytes(BL_OP_PACK, 0, N, K) bytes. */
+bl_status bitlinear_absmean_sum(const void* W, int wdt, int64_t N, int64_t K, double* sum,
+                                void* ws, size_t ws_bytes, bl_stream_t stream);
+
+/* Pack one shard [N, K] with the gamma of the whole tensor:
+ *   gamma = fp32(*total_sum / total_count)   (device double, fp64 division)
+ * total_sum: the fp64 sum of |W| over every shard; total_count: the element count
+ * of the whole tensor (>= N * K). Wp [N, K/4] and gamma [1] as bitlinear_pack_weights. */
+bl_status bitlinear_pack_weights_global(const void* W, int wdt, int64_t N, int64_t K, const double* total_sum,
+                                        int64_t total_count, uint8_t* Wp, float* gamma, bl_stream_t stream);
+
+/* Rank-local first half of the FFN: xq, s = quant(x) (x [M, d] whole on every
+ * rank); g, u = deq(Wg . xq), deq(Wu . xq) on the rank's f_local rows (fp32);
+ * h = max(g, 0)^2 * u -> h [M, f_local] fp32 (device); per token the rank's share of
+ * the subln statistics: ss[m] = sum_j h[m, j]^2 (fp64) and hmax[m] = max_j |h[m, j]|.
+ *   Wg, Wu  [f_local, d/4] packed shard rows; gg, gu [1] device fp32 (whole-tensor gammas)
+ *   ws      bitlinear_workspace_bytes(BL_OP_FFN_TP_UP, M, f_local, d) bytes */
+bl_status bitlinear_ffn_tp_up(const uint8_t* Wg, const float* gg, const uint8_t* Wu, const float* gu,
+                              int64_t d, int64_t f_local, const uint16_t* x, int64_t M, float* h, double* ss,
+                              float* hmax, void* ws, size_t ws_bytes, bl_stream_t stream);
+
+/* Rank-local second half, after ss and hmax are reduced over the ranks
+ * (ss_all = sum, hmax_all = max; device, [M]):
+ *   r  = 1 / sqrtf(float(ss_all / f_total) + 1e-5)
+ *   s2 = 127 / max(fl(hmax_all * r), 1e-5)          -> s2 [M] device fp32
+ *   q2 = clip(rint(fl(h * r) * s2))                  the rank's columns
+ *   acc[m, n] = sum_{j in the rank's columns} Wd[n, j] q2[m, j]  -> acc [M, d] int32
+ *   Wd  [d, f_local/4] packed shard columns (packed with the whole tensor's gamma)
+ *   ws  bitlinear_workspace_bytes(BL_OP_FFN_TP_DOWN, M, d, f_local) bytes */
+bl_status bitlinear_ffn_tp_down(const uint8_t* Wd, int64_t d, int64_t f_local, int64_t f_total, const float* h,
+                                int64_t M, const double* ss_all, const float* hmax_all, int32_t* acc, float* s2,
+                                void* ws, size_t ws_bytes, bl_stream_t stream);
+
+/* After acc is summed over the ranks: y = bf16([residual +] float(acc) * (gd / s2)).
+ *   acc [M, d] int32, s2 [M] fp32, gd [1] (whole-tensor gamma), residual [M, d] bf16
+ *   (may be NULL), y [M, d] bf16; all device. No workspace. */
+bl_status bitlinear_ffn_tp_finish(const int32_t* acc, const float* gd, const float* s2, const uint16_t* residual,
+                                  uint16_t* y, int64_t M, int64_t d, bl_stream_t stream);
 
 /*
  * Check packed weights for the invalid code 3. SYNCHRONISES `stream`.

@@ -65,6 +65,10 @@ def _l():
             "orc_ffn_layer": (ctypes.c_int, [P, F, P, F, P, F, I, I, P, I, P, P, P, P, P, P, P]),
             "orc_forward_ex": (ctypes.c_int, [P, P, P, I, I, P, I, I, P, P, P]),
             "orc_pack_weights_rowwise": (ctypes.c_int, [P, I, I, P, P]),
+            "orc_absmean_sum": (ctypes.c_double, [P, I]),
+            "orc_pack_weights_global": (ctypes.c_int, [P, I, I, ctypes.c_double, I, P, P]),
+            "orc_ffn_tp_up": (ctypes.c_int, [P, F, P, F, I, I, P, I, P, P, P]),
+            "orc_ffn_tp_down": (ctypes.c_int, [P, I, I, I, P, I, P, P, P, P]),
             "orc_forward_rowwise": (ctypes.c_int, [P, P, I, I, P, I, P, P, P]),
         }
         for name, (res, args) in sig.items():
@@ -313,3 +317,61 @@ def ffn_layer(Wg, gg, Wu, gu, Wd, gd, x_bf16, residual=None):
     if rc != 0:
         raise MemoryError("oracle ffn_layer failed")
     return dict(y=y, h=h, q2=q2, s2=s2, r=r, accd=accd)
+
+
+# --------------------------------------------------------------------------- tensor-parallel pieces
+
+def absmean_sum(W: np.ndarray) -> float:
+    """fp64 sum of |W| of one shard (fp32, or bf16 bits)."""
+    if W.dtype == np.uint16:
+        W = bf16_to_f32(W)
+    W = _c(W, np.float32)
+    return float(_l().orc_absmean_sum(_p(W), W.size))
+
+
+def pack_weights_global(W: np.ndarray, total_sum: float, total_count: int):
+    """Pack one shard with gamma = fp32(total_sum / total_count) of the whole tensor."""
+    if W.dtype == np.uint16:
+        W = bf16_to_f32(W)
+    W = _c(W, np.float32)
+    N, K = W.shape
+    Wp = np.empty((N, K // 4), np.uint8)
+    g = np.zeros(1, np.float32)
+    if _l().orc_pack_weights_global(_p(W), N, K, float(total_sum), int(total_count), _p(Wp), _p(g)) != 0:
+        raise MemoryError("oracle pack_weights_global failed")
+    return Wp, np.float32(g[0])
+
+
+def ffn_tp_up(Wg, gg, Wu, gu, x_bf16):
+    """Rank-local gate/up: returns (h [M, fl] fp32, ss [M] fp64, hmax [M] fp32)."""
+    Wg = _c(Wg, np.uint8)
+    Wu = _c(Wu, np.uint8)
+    x = _c(x_bf16, np.uint16)
+    M, d = x.shape
+    fl = Wg.shape[0]
+    assert Wg.shape == (fl, d // 4) and Wu.shape == (fl, d // 4)
+    h = np.empty((M, fl), np.float32)
+    ss = np.empty(M, np.float64)
+    hmax = np.empty(M, np.float32)
+    if _l().orc_ffn_tp_up(_p(Wg), float(np.float32(gg)), _p(Wu), float(np.float32(gu)), d, fl, _p(x), M, _p(h),
+                          _p(ss), _p(hmax)) != 0:
+        raise MemoryError("oracle ffn_tp_up failed")
+    return h, ss, hmax
+
+
+def ffn_tp_down(Wd, h, ss_all, hmax_all, f_total: int):
+    """Rank-local requantisation with the global statistics and the partial down
+    projection: returns (acc [M, d] int32, s2 [M] fp32)."""
+    Wd = _c(Wd, np.uint8)
+    h = _c(h, np.float32)
+    ss_all = _c(ss_all, np.float64)
+    hmax_all = _c(hmax_all, np.float32)
+    M, fl = h.shape
+    d = Wd.shape[0]
+    assert Wd.shape == (d, fl // 4)
+    acc = np.empty((M, d), np.int32)
+    s2 = np.empty(M, np.float32)
+    if _l().orc_ffn_tp_down(_p(Wd), d, fl, int(f_total), _p(h), M, _p(ss_all), _p(hmax_all), _p(acc),
+                            _p(s2)) != 0:
+        raise MemoryError("oracle ffn_tp_down failed")
+    return acc, s2

@@ -437,3 +437,103 @@ done:
     free(xf); free(xq); free(s); free(acc);
     return rc;
 }
+
+/* ------------------------------------------------------------------------- */
+/* Tensor-parallel pieces of the weight path and of the FFN sub-layer. The pages
+ * give no distributed detail (paper card, "Limits"); this is the library's
+ * split of the same computation over P ranks: rank r owns rows [c0, c1) of the
+ * gate and up weights and the same columns of the down weight. Composed over
+ * the ranks (sums and maxima exchanged between them), the pieces give exactly
+ * orc_pack_weights and orc_ffn_layer on the whole tensors.                   */
+
+/* fp64 sum of |W| over one shard (row-major order), the term each rank adds to
+ * the per-tensor absmean of [card] "Method Adaptation".                       */
+double orc_absmean_sum(const float* W, int64_t n) {
+    double s = 0.0;
+    for (int64_t i = 0; i < n; ++i) s += fabs((double)W[i]);
+    return s;
+}
+
+/* Ternarise and pack one shard with the gamma of the whole tensor:
+ * gamma = fp32(total_sum / total_count), the fp64 sum and count over all shards. */
+int orc_pack_weights_global(const float* W, int64_t N, int64_t K, double total_sum, int64_t total_count,
+                            uint8_t* Wp, float* gamma_out) {
+    int8_t* q = (int8_t*)malloc((size_t)(N * K));
+    if (!q) return -1;
+    float gamma = (float)(total_sum / (double)total_count);
+    orc_ternarize(W, N * K, gamma, q);
+    orc_pack(q, N, K, Wp);
+    free(q);
+    *gamma_out = gamma;
+    return 0;
+}
+
+/* Rank-local first half of the FFN: x is quantised whole (every rank holds it),
+ * the rank's fl gate and up rows give h = relu(g)^2 * u as in orc_ffn_layer, and
+ * per token the rank's share of the subln statistics: ss = sum_j h_j^2 (fp64,
+ * j in order) and hmax = max_j |h_j| over its fl columns.                      */
+int orc_ffn_tp_up(const uint8_t* Wg, float gg, const uint8_t* Wu, float gu, int64_t d, int64_t fl,
+                  const uint16_t* x, int64_t M, float* h, double* ss, float* hmax) {
+    float* xf = (float*)malloc(sizeof(float) * (size_t)(M * d));
+    int8_t* xq = (int8_t*)malloc((size_t)(M * d));
+    float* s = (float*)malloc(sizeof(float) * (size_t)M);
+    int32_t* accg = (int32_t*)malloc(sizeof(int32_t) * (size_t)(M * fl));
+    int32_t* accu = (int32_t*)malloc(sizeof(int32_t) * (size_t)(M * fl));
+    int rc = 0;
+    if (!xf || !xq || !s || !accg || !accu) {
+        rc = -1;
+        goto done;
+    }
+    orc_bf16_to_f32_array(x, M * d, xf);
+    orc_quant_act(xf, M, d, xq, s, NULL);
+    orc_int_gemm_packed(Wg, xq, M, fl, d, accg);
+    orc_int_gemm_packed(Wu, xq, M, fl, d, accu);
+    for (int64_t m = 0; m < M; ++m) {
+        float deqg = gg / s[m];
+        float dequ = gu / s[m];
+        double acc_ss = 0.0;
+        float mx = 0.0f;
+        for (int64_t j = 0; j < fl; ++j) {
+            float g = (float)accg[m * fl + j] * deqg;
+            float u = (float)accu[m * fl + j] * dequ;
+            float hv = orc_relu2_gate(g, u);
+            h[m * fl + j] = hv;
+            acc_ss += (double)hv * (double)hv;
+            if (fabsf(hv) > mx) mx = fabsf(hv);
+        }
+        ss[m] = acc_ss;
+        hmax[m] = mx;
+    }
+done:
+    free(xf); free(xq); free(s); free(accg); free(accu);
+    return rc;
+}
+
+/* Rank-local second half: with the statistics of all ranks (ss_all: the sum of
+ * the ranks' ss; hmax_all: their maximum) the subln factor and the
+ * requantisation scale are those of the whole h:
+ *   r  = 1 / sqrtf(float(ss_all / f_total) + eps)      (orc_subln_rms)
+ *   s2 = 127 / max(max_j |fl(h_j r)|, 1e-5) = 127 / max(fl(hmax_all r), 1e-5)
+ * (rounding is monotonic and r > 0, so the largest |fl(h_j r)| is fl(max|h_j| r));
+ * the rank quantises its columns fl(h_j r) with s2 and contracts them with its
+ * down columns: acc[m, n] = sum_{j in the rank's columns} Wd[n, j] q2[m, j].   */
+int orc_ffn_tp_down(const uint8_t* Wd, int64_t d, int64_t fl, int64_t f_total, const float* h, int64_t M,
+                    const double* ss_all, const float* hmax_all, int32_t* acc, float* s2) {
+    int8_t* q2 = (int8_t*)malloc((size_t)(M * fl));
+    if (!q2) return -1;
+    for (int64_t m = 0; m < M; ++m) {
+        float ms = (float)(ss_all[m] / (double)f_total);
+        float r = 1.0f / sqrtf(ms + ORC_RMS_EPS);
+        float sm = ORC_QB / fmaxf(hmax_all[m] * r, ORC_X_EPS);
+        for (int64_t j = 0; j < fl; ++j) {
+            float v = rintf((h[m * fl + j] * r) * sm);
+            if (v > 127.0f) v = 127.0f;
+            if (v < -128.0f) v = -128.0f;
+            q2[m * fl + j] = (int8_t)v;
+        }
+        s2[m] = sm;
+    }
+    orc_int_gemm_packed(Wd, q2, M, d, fl, acc);
+    free(q2);
+    return 0;
+}

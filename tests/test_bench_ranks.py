@@ -35,7 +35,7 @@ def _worker(rank, world, port, out):
 
 def test_max_over_ranks_with_gloo():
     world = 2
-    out = mp.Manager().dict()
+    out = mp.get_context("spawn").Manager().dict()  # no fork: CUDA may be initialised in this process
     mp.spawn(_worker, args=(world, _free_port(), out), nprocs=world, join=True)
     assert dict(out) == {0: 15.0, 1: 15.0}
 

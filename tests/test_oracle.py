@@ -439,3 +439,54 @@ def test_forward_rowwise_worked_2x4():
     # neither the per-tensor path nor a transposed gamma choice reproduces it
     for wrong in (np.full(2, gammas[0], np.float32), gammas[::-1].copy()):
         assert not np.array_equal(oracle.forward_rowwise(Wp, wrong, x)["y"], want)
+
+
+# ----------------------------------------------------------------------------- tensor-parallel pieces
+
+@pytest.mark.parametrize("P", [1, 2, 3])
+def test_ffn_tensor_parallel_pieces_compose_to_the_whole_layer(P):
+    """Shards of the hidden width, combined with sums (fp64 statistics, int32
+    accumulators) and maxima, give exactly the unsharded gammas, packed bytes, h,
+    requantisation scale, accumulators and output. A slip such as dividing the
+    sum of squares by the shard's width, a shard-local max, or a shard-local gamma
+    breaks one of these equalities."""
+    from bitlinear_w1_a8_02_b200 import tp
+    d, f, M = 64, 200, 5
+    Wg = bf16_bits(synth.weights(f, d, 0.02, 80))
+    Wu = bf16_bits(synth.weights(f, d, 0.02, 81))
+    Wd = bf16_bits(synth.weights(d, f, 0.02, 82))
+    x = bf16_bits(synth.activations(M, d, seed=83, outliers=True))
+    whole = [oracle.pack_weights(W) for W in (Wg, Wu, Wd)]
+    ref = oracle.ffn_layer(whole[0][0], whole[0][1], whole[1][0], whole[1][1], whole[2][0], whole[2][1], x,
+                           residual=x)
+    bounds = [tp.shard_range(f, P, r, align=4) for r in range(P)]
+    shards = []
+    for (c0, c1) in bounds:
+        parts = (Wg[c0:c1], Wu[c0:c1], np.ascontiguousarray(Wd[:, c0:c1]))
+        shards.append(parts)
+    packed = []
+    for i, W in enumerate((Wg, Wu, Wd)):
+        total = sum(oracle.absmean_sum(s[i]) for s in shards)
+        packed.append([oracle.pack_weights_global(s[i], total, W.size) for s in shards])
+        for r, (c0, c1) in enumerate(bounds):
+            assert packed[i][r][1] == whole[i][1]
+            want = whole[i][0][c0:c1] if i < 2 else whole[i][0][:, c0 // 4:c1 // 4]
+            assert np.array_equal(packed[i][r][0], want)
+    ups = [oracle.ffn_tp_up(packed[0][r][0], packed[0][r][1], packed[1][r][0], packed[1][r][1], x)
+           for r in range(P)]
+    assert np.array_equal(np.concatenate([u[0] for u in ups], axis=1), ref["h"])
+    ss = np.zeros(M, np.float64)
+    for u in ups:
+        ss = ss + u[1]
+    hmax = np.max(np.stack([u[2] for u in ups]), axis=0)
+    acc = np.zeros((M, d), np.int64)
+    s2 = None
+    for r in range(P):
+        a, s2r = oracle.ffn_tp_down(packed[2][r][0], ups[r][0], ss, hmax, f)
+        acc += a
+        assert s2 is None or np.array_equal(s2r, s2)
+        s2 = s2r
+    assert np.array_equal(s2, ref["s2"])
+    assert np.array_equal(acc.astype(np.int32), ref["accd"])
+    y = oracle.dequant(acc.astype(np.int32), packed[2][0][1], s2, residual=x)
+    assert np.array_equal(y, ref["y"])
