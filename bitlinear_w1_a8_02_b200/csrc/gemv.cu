@@ -118,6 +118,8 @@ struct GemvArgs {
     unsigned* err;         // device error word (bounded waits that give up)
     int norm;              // fused quantisation: unit-weight RMSNorm of x first
     int seg_chunks;        // 64-byte chunks per K segment of a streamed unit
+    int unit_rows;         // rows per streamed unit: 16, or 8 / 4 for one token with long rows
+    int rg_shift;          // one token: log2(threads per group of 4 rows) = log2(1024 / unit_rows)
     int pitch;             // shared-memory row pitch of a stage
     int codes_bytes;       // fused codes area at the start of dynamic shared memory
     // second weight stream (FFN up: Wp = gate, Wp2 = up; same rows, same codes)
@@ -310,6 +312,52 @@ __device__ void fused_quantise(const GemvArgs& a, int KB, uint8_t* codes, uint32
     }
 }
 
+// One token with a long row (BIG instantiation): each thread loads all of its
+// 16-element groups at once (at most kBigGroups), keeps them in registers for the
+// absmax and for the codes, so the token costs one round trip to L2 instead of
+// one per group and pass. Codes in the interleaved single-token layout.
+constexpr int kBigGroups = 8;
+
+__device__ void fused_quantise_big(const GemvArgs& a, int KB, uint8_t* codes, uint32_t* am_w, float* s_sh,
+                                   int* xs_sh, float* deq_sh) {
+    const int groups = KB / 4;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint4* xv = reinterpret_cast<const uint4*>(a.x);
+    const float gamma = threadIdx.x == 0 ? *a.gamma : 0.0f;
+    uint4 v[kBigGroups][2];
+#pragma unroll
+    for (int i = 0; i < kBigGroups; ++i) {
+        const int c = threadIdx.x + i * kThreads;
+        v[i][0] = v[i][1] = make_uint4(0u, 0u, 0u, 0u);
+        if (c < groups) {
+            v[i][0] = xv[2 * c];
+            v[i][1] = xv[2 * c + 1];
+        }
+    }
+    uint32_t mx = 0;  // zero groups (past the row) leave the maximum unchanged
+#pragma unroll
+    for (int i = 0; i < kBigGroups; ++i) mx = max(mx, absmax16(v[i][0], v[i][1]));
+    mx = __reduce_max_sync(0xffffffffu, mx);
+    if (lane == 0) am_w[warp] = mx;
+    consumer_sync();
+    uint32_t amb = am_w[0];
+#pragma unroll
+    for (int w = 1; w < kWarps; ++w) amb = max(amb, am_w[w]);
+    const float s = __fdiv_rn(kActRange, fmaxf(__uint_as_float(amb << 16), kActEps));
+    int sum = 0;
+#pragma unroll
+    for (int i = 0; i < kBigGroups; ++i) {
+        const int c = threadIdx.x + i * kThreads;
+        if (c < groups) sum += quant_bf16x16<true, false>(v[i][0], v[i][1], s, codes + 16 * c, KB, false, 1.0f);
+    }
+    sum = __reduce_add_sync(0xffffffffu, sum);
+    if (lane == 0) atomicAdd(&xs_sh[0], sum);
+    if (threadIdx.x == 0) {
+        s_sh[0] = s;
+        deq_sh[0] = __fdiv_rn(gamma, s);
+    }
+}
+
 // FFN glue inside the down projection (consumer threads): per token,
 // r = 1 / sqrtf(float(sum_j h_j^2 / f) + eps) from the up kernel's per-tile fp64
 // partials (fixed order: thread strides, warp butterfly, warps in index order),
@@ -397,8 +445,13 @@ __device__ __forceinline__ void bulk_copy(uint32_t dst, const void* src, uint32_
 // different banks.
 // XT: extended calls (row segments with their own gamma, RMSNorm of x); the
 // plain forward runs the instantiation without that code.
-template <int NT, int SRC, bool DUAL, bool DP, bool XT>
-__global__ void __launch_bounds__(kThreads + 32, NT == 1 ? 3 : 2) gemv_mma_kernel(const GemvArgs a) {
+// BIG: one token with a long row, quantised from registers (fused_quantise_big);
+// its registers allow two CTAs per SM.
+// Units of the single-token path hold a.unit_rows rows (16, or 8 / 4 for rows
+// longer than 2 KiB, so a unit stays a contiguous ~32 KiB and the tiles are fine
+// enough to balance the CTAs); every other path streams 16-row units.
+template <int NT, int SRC, bool DUAL, bool DP, bool XT, bool BIG = false>
+__global__ void __launch_bounds__(kThreads + 32, (NT == 1 && !BIG) ? 3 : 2) gemv_mma_kernel(const GemvArgs a) {
     constexpr int TOK = 8 * NT;
     constexpr bool FUSED = SRC != SRC_CODES;
     static_assert(!DP || (FUSED && NT == 1), "the dp4a path reads one token's codes from shared memory");
@@ -416,7 +469,8 @@ __global__ void __launch_bounds__(kThreads + 32, NT == 1 ? 3 : 2) gemv_mma_kerne
 
     const int N = a.N, KB = a.KB;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int ntiles = (N + 15) >> 4;
+    const int R = a.unit_rows;                         // rows per tile (16 except on the single-token path)
+    const int ntiles = (N + R - 1) / R;
     const int nchunks = KB >> 6;
     const int cps = a.seg_chunks;                     // chunks per K segment
     const int nseg = (nchunks + cps - 1) / cps;
@@ -424,8 +478,8 @@ __global__ void __launch_bounds__(kThreads + 32, NT == 1 ? 3 : 2) gemv_mma_kerne
     const int tok0 = blockIdx.y * TOK;
 
     uint8_t* codes = dyn;                              // fused: PLANES codes of the M tokens
-    uint8_t* stages = dyn + a.codes_bytes;             // kStages x NW x 16 rows x pitch
-    const int stage_bytes = NW * 16 * pitch;
+    uint8_t* stages = dyn + a.codes_bytes;             // kStages x NW x R rows x pitch
+    const int stage_bytes = NW * R * pitch;
     uint64_t* bars = reinterpret_cast<uint64_t*>(stages + kStages * stage_bytes);
     auto full = [&](int st) { return tc::smem_u32(bars + st); };
     auto empty = [&](int st) { return tc::smem_u32(bars + kStages + st); };
@@ -442,9 +496,9 @@ __global__ void __launch_bounds__(kThreads + 32, NT == 1 ? 3 : 2) gemv_mma_kerne
         for (int p = 0; p < kPrefetchAhead; ++p) {
             const int tile = blockIdx.x + p * gridDim.x;
             if (tile < ntiles) {
-                const int n0 = tile * 16;
-                prefetch_l2(a.Wp + (size_t)n0 * KB, (uint32_t)(min(16, N - n0) * KB));
-                if (DUAL) prefetch_l2(a.Wp2 + (size_t)n0 * KB, (uint32_t)(min(16, N - n0) * KB));
+                const int n0 = tile * R;
+                prefetch_l2(a.Wp + (size_t)n0 * KB, (uint32_t)(min(R, N - n0) * KB));
+                if (DUAL) prefetch_l2(a.Wp2 + (size_t)n0 * KB, (uint32_t)(min(R, N - n0) * KB));
             }
         }
     }
@@ -458,8 +512,8 @@ __global__ void __launch_bounds__(kThreads + 32, NT == 1 ? 3 : 2) gemv_mma_kerne
             bool stop = false;
             bool waited = false;
             for (int tile = blockIdx.x; tile < ntiles && !stop; tile += gridDim.x) {
-                const int n0 = tile * 16;
-                const int rows = min(16, N - n0);
+                const int n0 = tile * R;
+                const int rows = min(R, N - n0);
                 for (int sg = 0; sg < nseg; ++sg, ++g) {
                     const int st = g % kStages;
                     if (g >= kStages &&
@@ -483,7 +537,7 @@ __global__ void __launch_bounds__(kThreads + 32, NT == 1 ? 3 : 2) gemv_mma_kerne
                         bulk_copy(dst + r * pitch, a.Wp + (size_t)(n0 + r) * KB + c0 * 64, segb, full(st));
                     if (DUAL)
                         for (int r = 0; r < rows; ++r)
-                            bulk_copy(dst + (16 + r) * pitch, a.Wp2 + (size_t)(n0 + r) * KB + c0 * 64, segb,
+                            bulk_copy(dst + (R + r) * pitch, a.Wp2 + (size_t)(n0 + r) * KB + c0 * 64, segb,
                                       full(st));
                 }
             }
@@ -534,7 +588,10 @@ __global__ void __launch_bounds__(kThreads + 32, NT == 1 ? 3 : 2) gemv_mma_kerne
 
     grid_dependency_wait();
     if (SRC == SRC_X) {
-        fused_quantise<DUAL, DP, XT>(a, KB, codes, am_sh, ss_sh, s_sh, xs_sh, deq_sh, deq2_sh);
+        if constexpr (BIG)
+            fused_quantise_big(a, KB, codes, am_sh[0], s_sh, xs_sh, deq_sh);
+        else
+            fused_quantise<DUAL, DP, XT>(a, KB, codes, am_sh, ss_sh, s_sh, xs_sh, deq_sh, deq2_sh);
     } else if (SRC == SRC_H) {
         finalise_quantise<DP>(a, KB, codes, s_sh, xs_sh, r_sh, deq_sh);
     } else if (threadIdx.x < TOK && tok0 + (int)threadIdx.x < a.M) {
@@ -547,12 +604,13 @@ __global__ void __launch_bounds__(kThreads + 32, NT == 1 ? 3 : 2) gemv_mma_kerne
 
     uint32_t g = 0;
     for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
-        const int n0 = tile * 16;
+        const int n0 = tile * R;
         if constexpr (DP) {
-            // One token: thread (row group rg, lane tl of 64) owns rows 4 rg .. 4 rg + 3
-            // of the unit and its words j = tl, tl + 64, ...; per word one dp4a per
-            // field against the interleaved plane words of the token.
-            const int rg = threadIdx.x >> 6, tl = threadIdx.x & 63;
+            // One token: thread (row group rg, lane tl of T = 1024 / R) owns rows
+            // 4 rg .. 4 rg + 3 of the unit and its words j = tl, tl + T, ...; per word
+            // one dp4a per field against the interleaved plane words of the token.
+            const int rg = threadIdx.x >> a.rg_shift, tl = threadIdx.x & ((1 << a.rg_shift) - 1);
+            const int tstride = 1 << a.rg_shift;
             int acc[4][4] = {}, acc2[DUAL ? 4 : 1][4] = {};
             for (int sg = 0; sg < nseg; ++sg, ++g) {
                 const int st = g % kStages;
@@ -566,14 +624,14 @@ __global__ void __launch_bounds__(kThreads + 32, NT == 1 ? 3 : 2) gemv_mma_kerne
                 const uint8_t* wr = stages + st * stage_bytes + 4 * rg * pitch;
                 const uint4* xw = reinterpret_cast<const uint4*>(codes) + sg * cps * 16;
 #pragma unroll 2
-                for (int j = tl; j < words; j += 64) {
+                for (int j = tl; j < words; j += tstride) {
                     const uint4 xv = xw[j];
 #pragma unroll
                     for (int r = 0; r < 4; ++r) {
                         const uint32_t w = *reinterpret_cast<const uint32_t*>(wr + r * pitch + 4 * j);
                         dp4a_fields(acc[r], w, xv);
                         if constexpr (DUAL) {
-                            const uint32_t w2 = *reinterpret_cast<const uint32_t*>(wr + (16 + r) * pitch + 4 * j);
+                            const uint32_t w2 = *reinterpret_cast<const uint32_t*>(wr + (R + r) * pitch + 4 * j);
                             dp4a_fields(acc2[r], w2, xv);
                         }
                     }
@@ -704,7 +762,7 @@ __global__ void __launch_bounds__(kThreads + 32, NT == 1 ? 3 : 2) gemv_mma_kerne
             for (int idx = threadIdx.x; idx < 16 * TOK; idx += kThreads) {
                 const int r = idx & 15, cl = idx >> 4;
                 const int n = n0 + r, m = tok0 + cl;
-                if (n >= N || m >= a.M) continue;
+                if (r >= R || n >= N || m >= a.M) continue;
                 int sum = 0;
 #pragma unroll
                 for (int w = 0; w < kWarps; ++w) sum += red[w][r][cl];
@@ -770,9 +828,9 @@ int sm_count() {
     return n;
 }
 
-template <int NT, int SRC, bool DUAL, bool DP = false, bool XT = false>
+template <int NT, int SRC, bool DUAL, bool DP = false, bool XT = false, bool BIG = false>
 cudaError_t launch_variant(const GemvArgs& a, dim3 grid, size_t smem, cudaStream_t s) {
-    auto kern = gemv_mma_kernel<NT, SRC, DUAL, DP, XT>;
+    auto kern = gemv_mma_kernel<NT, SRC, DUAL, DP, XT, BIG>;
     static bool done[64];
     int dev = 0;
     cudaGetDevice(&dev);
@@ -798,22 +856,27 @@ struct StreamPlan {
     unsigned grid_x;
 };
 
+// unit_rows: 16, or 8 / 4 for the single-token path (whose threads then cover
+// one or two groups of four rows); a unit keeps at most 32 KiB of weights.
 cudaError_t plan_stream(GemvArgs& a, int64_t N, int64_t K, int64_t M, int nw, bool codes_in_smem,
-                        StreamPlan& p) {
+                        StreamPlan& p, int unit_rows = 16, int max_per_sm = 4) {
     cudaError_t e = device_error_word(&a.err);
     if (e != cudaSuccess) return e;
-    // K segments of at most kMaxSegChunks chunks, as even as possible
+    a.unit_rows = unit_rows;
+    a.rg_shift = unit_rows == 16 ? 6 : unit_rows == 8 ? 7 : 8;
+    // K segments of at most kMaxSegChunks * 16 / unit_rows chunks, as even as possible
+    const int max_seg = kMaxSegChunks * 16 / unit_rows;
     const int nchunks = (int)(K / 256);
-    const int nseg = (nchunks + kMaxSegChunks - 1) / kMaxSegChunks;
+    const int nseg = (nchunks + max_seg - 1) / max_seg;
     a.seg_chunks = (nchunks + nseg - 1) / nseg;
     const int segb = a.seg_chunks * 64;
     a.pitch = (segb % 128 == 0) ? segb + 64 : segb;  // rows g, g+1 on different banks
     a.codes_bytes = codes_in_smem ? (int)((M * (K + 64) + 127) / 128 * 128) : 0;
-    p.smem = (size_t)a.codes_bytes + (size_t)kStages * nw * 16 * a.pitch + 2 * kStages * 8;
-    const int ntiles = (int)((N + 15) / 16);
+    p.smem = (size_t)a.codes_bytes + (size_t)kStages * nw * unit_rows * a.pitch + 2 * kStages * 8;
+    const int ntiles = (int)((N + unit_rows - 1) / unit_rows);
     // as many CTAs per SM as shared memory allows (228 KiB per SM, static + reserve per CTA)
     int per_sm = (int)((228 * 1024) / (p.smem + 10 * 1024));
-    per_sm = per_sm < 1 ? 1 : per_sm > 4 ? 4 : per_sm;
+    per_sm = per_sm < 1 ? 1 : per_sm > max_per_sm ? max_per_sm : per_sm;
     const int cap = per_sm * sm_count();
     p.grid_x = (unsigned)(ntiles < cap ? ntiles : cap);
     return cudaSuccess;
@@ -857,16 +920,24 @@ cudaError_t launch_gemv(const uint8_t* Wp, const float* gamma, int64_t N, int64_
     a.Xp = Xp;
     a.scale = scale;
     a.xsum = xsum;
+    const bool xt = a.norm || out.seg_end[0] < N || out.per_row;
+    // One token: units of whole rows of up to 32 KiB (16, 8 or 4 rows), and for a
+    // long row (8192 <= K <= 32768) the quantiser that keeps x in registers (its
+    // register budget allows two CTAs per SM).
+    const bool one = x_fused && M == 1;
+    const int64_t KB = K / 4;
+    const int unit_rows = one ? (KB <= 2048 ? 16 : KB <= 4096 ? 8 : 4) : 16;
+    const bool big = one && !xt && K >= 8192 && K / 16 <= (int64_t)kBigGroups * kThreads;
     StreamPlan p;
-    cudaError_t e = plan_stream(a, N, K, M, 1, x_fused != nullptr, p);
+    cudaError_t e = plan_stream(a, N, K, M, 1, x_fused != nullptr, p, unit_rows, big ? 2 : 4);
     if (e != cudaSuccess) return e;
     const dim3 g1(p.grid_x, 1), g2(p.grid_x, (unsigned)((M + 15) / 16));
-    const bool xt = a.norm || out.seg_end[0] < N || out.per_row;
     if (xt) {
         if (x_fused) return launch_fused<SRC_X, false, true>(a, g1, p.smem, s);
         if (M <= 8) return launch_variant<1, SRC_CODES, false, false, true>(a, g1, p.smem, s);
         return launch_variant<2, SRC_CODES, false, false, true>(a, g2, p.smem, s);
     }
+    if (big) return launch_variant<1, SRC_X, false, true, false, true>(a, g1, p.smem, s);
     if (x_fused) return launch_fused<SRC_X, false>(a, g1, p.smem, s);
     if (M <= 8) return launch_variant<1, SRC_CODES, false>(a, g1, p.smem, s);
     return launch_variant<2, SRC_CODES, false>(a, g2, p.smem, s);

@@ -566,3 +566,33 @@ def test_forward_gemv_lookup_table_rowwise(cuda_device):
     ref = oracle.forward_rowwise(Wp_ref, g_ref, bits(x))
     assert np.array_equal(np_(acc), ref["acc"])
     assert_bf16_exact(bits(y), ref["y"])
+
+
+# ----------------------------------------------------------------------------- one token, long rows
+
+@pytest.mark.parametrize("K", [4608, 8192, 12288, 20480, 32768, 36864])
+@pytest.mark.parametrize("N", [1001, 300])
+def test_forward_single_token_long_rows(cuda_device, K, N):
+    """M = 1 on the streamed dp4a GEMV with units of whole rows (16 rows up to
+    2 KiB per row, 8 up to 4 KiB, 4 beyond; two K segments past 8 KiB) and the
+    register-resident quantiser for 8192 <= K <= 32768; N ragged for every unit
+    height."""
+    W = make_weights(N, K, 0.01, seed=6000 + K + N)
+    Wp, gamma, Wp_ref, g_ref = pack_both(W, cuda_device)
+    x = synth.activations(1, K, seed=6100 + K, outliers=True)
+    res = synth.activations(1, N, seed=6200 + N, outliers=False)
+    check_forward_full(Wp, gamma, Wp_ref, g_ref, x, cuda_device, residual=res)
+
+
+@pytest.mark.parametrize("K", [12288, 28672])
+def test_forward_ex_single_token_long_rows_rmsnorm(cuda_device, K):
+    rows = [256, 64, 64]
+    parts = [make_weights(n, K, 0.01, seed=6300 + i) for i, n in enumerate(rows)]
+    dev_parts = [bl.pack_weights(p.to(cuda_device)) for p in parts]
+    ref_parts = [oracle.pack_weights(bits(p)) for p in parts]
+    x = synth.activations(1, K, seed=6310, outliers=True)
+    yq = bl.forward_ex(torch.cat([p[0] for p in dev_parts]), torch.cat([p[1].reshape(1) for p in dev_parts]),
+                       rows, x.to(cuda_device), rmsnorm=True)
+    rq = oracle.forward_ex(np.concatenate([p[0] for p in ref_parts]), [p[1] for p in ref_parts], rows, bits(x),
+                           rmsnorm=True)
+    assert_bf16_exact(bits(yq), rq["y"])
