@@ -46,11 +46,11 @@ METRIC = "W1.58A8 BitLinear: decode GEMV HBM GB/s (% peak); prefill int8 TOPS (%
 DECODE_SHAPES = [(2560, 2560), (2560, 640), (2560, 6912), (6912, 2560)]  # (K, N)
 LAYERS = 30
 # DRAM bytes (read + write) per launch of the decode GEMV, averaged over the
-# step's four shapes: ncu captures of one launch per shape read 1,666,048 +
-# 436,992 + 4,451,072 + 4,459,776 bytes (0 written) for 2,723,840 packed bytes
+# step's four shapes: ncu captures of one launch per shape read 1,666,816 +
+# 437,248 + 4,452,352 + 4,460,544 bytes (0 written) for 2,723,840 packed bytes
 # per launch on average (x 1.011). Set to None whenever the kernel changes until
 # a new capture is taken.
-GEMV_TRAFFIC_PER_LAUNCH = 2753472
+GEMV_TRAFFIC_PER_LAUNCH = 2754240
 # The pages' only latency figure, quoted beside the whole-decoder-layer number as
 # context (not a target): whole-model CPU decode, ms per output token.
 PAGES_CPU_MS_PER_TOKEN = 29.0
