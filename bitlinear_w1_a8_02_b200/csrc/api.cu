@@ -409,6 +409,23 @@ BL_API bl_status bitlinear_ffn(const uint8_t* Wg, const float* gg, const uint8_t
         od.residual = residual;
         return cuda_status(bl::launch_ffn_down_fused(Wd, gd, d, f, g, part_ss, part_max, M, od, s));
     }
+    if (up == Path::GemmTc) {
+        // M > 16: gate and up in one tensor-core launch whose epilogue writes h (in
+        // the g slot) and per-tile partials of sum h^2 and max |h| (in the u slot);
+        // then the subln + requantisation from the partials, and the down projection.
+        const int nparts = bl::gemm_dual_parts(f);
+        bl::FfnUpOut fo;
+        fo.h = g;
+        fo.part_ss = (double*)u;
+        fo.part_max = (float*)((char*)u + align_up((size_t)M * nparts * sizeof(double)));
+        BL_TRY(bl::launch_act_quant(x, M, d, bl::XQ_G16T, xq, scale, xsum, s));
+        BL_TRY(bl::launch_gemm_tc_dual(Wg, gg, Wu, gu, f, d, xq, scale, xsum, M, fo, s));
+        BL_TRY(bl::launch_ffn_requant_parts(g, fo.part_ss, fo.part_max, nparts, M, f, layout_of(down), q2, s2, xsum2, s));
+        bl::GemvOut od;
+        od.y = y;
+        od.residual = residual;
+        return project(down, Wd, gd, d, f, q2, s2, xsum2, M, od, s, base + w.sk, w.sk_bytes);
+    }
     bl::GemvOut og;
     og.y32 = g;
     bl::GemvOut ou;

@@ -132,19 +132,15 @@ __global__ void __launch_bounds__(kThreads) ffn_tp_hstats_kernel(const float* __
 // r = 1 / sqrtf(float(ss_all / f_total) + 1e-5), s2 = 127 / max(fl(hmax_all r), 1e-5)
 // (the largest |fl(h_j r)| of the whole row: rounding is monotonic and r > 0),
 // codes of fl(h_j r) in the consumer's layout, and their sum over the rank's columns.
+// Codes of token m's fl columns fl(h_j r) with scale s = 127 / max(fl(hmax r), 1e-5),
+// r = 1 / sqrtf(float(ss / f_total) + 1e-5), in LAYOUT; s2[m] and the codes' sum.
 template <int LAYOUT>
-__global__ void __launch_bounds__(kThreads) ffn_tp_requant_kernel(const float* __restrict__ h, int fl, int64_t f_total,
-                                                                   const double* __restrict__ ss_all,
-                                                                   const float* __restrict__ hmax_all,
-                                                                   int8_t* __restrict__ q2, float* __restrict__ s2,
-                                                                   int32_t* __restrict__ xsum2) {
-    __shared__ int iscratch[kWarps];
-    grid_dependency_wait();
-    grid_dependents_launch();
-    const int m = blockIdx.x;
-    const float ms = __double2float_rn(__ddiv_rn(ss_all[m], (double)f_total));
+__device__ __forceinline__ void requant_row(const float* __restrict__ h, int m, int fl, int64_t f_total, double ss,
+                                            float hmax, int8_t* __restrict__ q2, float* __restrict__ s2,
+                                            int32_t* __restrict__ xsum2, int* iscratch) {
+    const float ms = __double2float_rn(__ddiv_rn(ss, (double)f_total));
     const float r = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, kRmsEps)));
-    const float s = __fdiv_rn(kActRange, fmaxf(__fmul_rn(hmax_all[m], r), kActEps));
+    const float s = __fdiv_rn(kActRange, fmaxf(__fmul_rn(hmax, r), kActEps));
     const float* hr = h + (size_t)m * fl;
     int sum = 0;
     if (LAYOUT == XQ_NATURAL) {
@@ -178,6 +174,46 @@ __global__ void __launch_bounds__(kThreads) ffn_tp_requant_kernel(const float* _
         s2[m] = s;
         xsum2[m] = sum;
     }
+}
+
+template <int LAYOUT>
+__global__ void __launch_bounds__(kThreads) ffn_tp_requant_kernel(const float* __restrict__ h, int fl, int64_t f_total,
+                                                                   const double* __restrict__ ss_all,
+                                                                   const float* __restrict__ hmax_all,
+                                                                   int8_t* __restrict__ q2, float* __restrict__ s2,
+                                                                   int32_t* __restrict__ xsum2) {
+    __shared__ int iscratch[kWarps];
+    grid_dependency_wait();
+    grid_dependents_launch();
+    const int m = blockIdx.x;
+    requant_row<LAYOUT>(h, m, fl, f_total, ss_all[m], hmax_all[m], q2, s2, xsum2, iscratch);
+}
+
+// The FFN's subln and requantisation after the fused gate+up GEMM: the token's
+// per-tile partials of sum h^2 (fp64) and max |h| reduced in a fixed order
+// (thread strides, warp butterfly, warps in index order), then requant_row.
+template <int LAYOUT>
+__global__ void __launch_bounds__(kThreads) ffn_requant_parts_kernel(const float* __restrict__ h,
+                                                                      const double* __restrict__ part_ss,
+                                                                      const float* __restrict__ part_max, int nparts,
+                                                                      int f, int8_t* __restrict__ q2,
+                                                                      float* __restrict__ s2,
+                                                                      int32_t* __restrict__ xsum2) {
+    __shared__ double dscratch[kWarps];
+    __shared__ float fscratch[kWarps];
+    __shared__ int iscratch[kWarps];
+    grid_dependency_wait();
+    grid_dependents_launch();
+    const int m = blockIdx.x;
+    double ss = 0.0;
+    float mx = 0.0f;
+    for (int p = threadIdx.x; p < nparts; p += kThreads) {
+        ss = __dadd_rn(ss, part_ss[(size_t)m * nparts + p]);
+        mx = fmaxf(mx, part_max[(size_t)m * nparts + p]);
+    }
+    ss = block_sum<kWarps>(ss, dscratch);
+    mx = block_max<kWarps>(mx, fscratch);
+    requant_row<LAYOUT>(h, m, f, f, ss, mx, q2, s2, xsum2, iscratch);
 }
 
 // y = bf16([residual +] float(acc) * (gd / s2)) on the accumulators summed over the ranks.
@@ -231,6 +267,22 @@ cudaError_t launch_ffn_tp_requant(const float* h, int64_t M, int64_t fl, int64_t
         return launch_pdl(ffn_tp_requant_kernel<XQ_G16T>, g, b, 0, s, h, (int)fl, f_total, ss_all, hmax_all, q2, s2,
                           xsum2);
     return launch_pdl(ffn_tp_requant_kernel<XQ_NATURAL>, g, b, 0, s, h, (int)fl, f_total, ss_all, hmax_all, q2, s2,
+                      xsum2);
+}
+
+cudaError_t launch_ffn_requant_parts(const float* h, const double* part_ss, const float* part_max, int nparts,
+                                     int64_t M, int64_t f, int layout, int8_t* q2, float* s2, int32_t* xsum2,
+                                     cudaStream_t s) {
+    if (M == 0) return cudaSuccess;
+    if (layout != XQ_NATURAL && f % 16 != 0) return cudaErrorInvalidValue;
+    const dim3 g((unsigned)M), b(kThreads);
+    if (layout == XQ_PLANES)
+        return launch_pdl(ffn_requant_parts_kernel<XQ_PLANES>, g, b, 0, s, h, part_ss, part_max, nparts, (int)f, q2,
+                          s2, xsum2);
+    if (layout == XQ_G16T)
+        return launch_pdl(ffn_requant_parts_kernel<XQ_G16T>, g, b, 0, s, h, part_ss, part_max, nparts, (int)f, q2, s2,
+                          xsum2);
+    return launch_pdl(ffn_requant_parts_kernel<XQ_NATURAL>, g, b, 0, s, h, part_ss, part_max, nparts, (int)f, q2, s2,
                       xsum2);
 }
 

@@ -196,12 +196,18 @@ __device__ __forceinline__ void store_row_chunk(const uint32_t (&v)[32], int xs,
 // flight share activation tiles and the whole packed weight stays in L2.
 // PR: one gamma per output row (the per-row variant); without it that code is
 // compiled out of the epilogue.
-template <int BN, bool SK, bool PR>
+// DUAL: the FFN's gate and up projections in one launch. Each 256-row weight
+// tile holds 128 rows of the gate weight (tmB) and the same 128 rows of the up
+// weight (tmB2); the epilogue forms h = max(g, 0)^2 * u of those 128 hidden
+// columns and, per token, the tile's sum of h^2 (fp64, columns in order) and max
+// |h| (FfnUpOut). Data-parallel tiles only.
+template <int BN, bool SK, bool PR, bool DUAL = false>
 __global__ void __launch_bounds__(THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   int M, int N, int K, const float* __restrict__ gamma_p,
+                   const __grid_constant__ CUtensorMap tmB2, int M, int N, int K, const float* __restrict__ gamma_p,
                    const float* __restrict__ scale, const int32_t* __restrict__ xsum, GemvOut out,
-                   unsigned* err, uint32_t* __restrict__ partials) {
+                   unsigned* err, uint32_t* __restrict__ partials, FfnUpOut up) {
+    static_assert(!DUAL || (BN == 256 && !SK && !PR), "the gate+up tiles are 128 + 128 rows, data-parallel");
     constexpr int P_BYTES = TileCfg<BN>::P_BYTES;
     constexpr int U_BYTES = TileCfg<BN>::U_BYTES;
     constexpr int UNPACK_VEC = TileCfg<BN>::UNPACK_VEC;
@@ -225,7 +231,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     auto aempty = [&](int a) { return bar(2 * TSTAGES + 2 * USTAGES + 2 + a); };  // drained
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int n_tiles = (N + BN - 1) / BN;
+    constexpr int TN = DUAL ? BN / 2 : BN;  // output columns per tile
+    const int n_tiles = (N + TN - 1) / TN;
     const int num_tiles = n_tiles * ((M + BM - 1) / BM);
     const int nkb = (K + BK - 1) / BK;
 
@@ -259,11 +266,12 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (lane == 0) {
             tc::prefetch_tmap(&tmA);
             tc::prefetch_tmap(&tmB);
+            if (DUAL) tc::prefetch_tmap(&tmB2);
             uint32_t g = 0;
             WorkIter<SK> it(nkb, num_tiles, gridDim.x, blockIdx.x);
             int tile, kb0, kb1;
             while (!aborted(&abort_sh) && it.next(tile, kb0, kb1)) {
-                const int m0 = (tile / n_tiles) * BM, n0 = (tile % n_tiles) * BN;
+                const int m0 = (tile / n_tiles) * BM, n0 = (tile % n_tiles) * TN;
                 for (int kb = kb0; kb < kb1; ++kb, ++g) {
                     const int s = g % TSTAGES;
                     if (g >= TSTAGES &&
@@ -274,6 +282,9 @@ __global__ void __launch_bounds__(THREADS, 1)
                     tc::mbar_arrive_expect_tx(tfull(s), A_BYTES + P_BYTES);
                     tc::tma_load_2d(tc::smem_u32(sA + s * A_BYTES), &tmA, kb * BK, m0, tfull(s));
                     tc::tma_load_2d(tc::smem_u32(sP + s * P_BYTES), &tmB, kb * (BK / 4), n0, tfull(s));
+                    if (DUAL)  // up rows into the second half of the weight tile
+                        tc::tma_load_2d(tc::smem_u32(sP + s * P_BYTES + (BN / 2) * (BK / 4)), &tmB2, kb * (BK / 4), n0,
+                                        tfull(s));
                 }
             }
             if (aborted(&abort_sh)) {
@@ -386,9 +397,60 @@ __global__ void __launch_bounds__(THREADS, 1)
                 break;
             }
             tc::fence_after_sync();
-            const int m0 = (tile / n_tiles) * BM, n0 = (tile % n_tiles) * BN;
+            const int m0 = (tile / n_tiles) * BM, n0 = (tile % n_tiles) * TN;
             const int m = m0 + q * 32 + lane;
             const bool mv = m < M;
+            if constexpr (DUAL) {
+                // h of this token's 128 hidden columns; gate in columns 0..127 of the
+                // accumulator, up in 128..255
+                const uint32_t tb = tmem + (static_cast<uint32_t>(q * 32) << 16) + a * BN;
+                const float dg = mv ? __fdiv_rn(gamma, scale[m]) : 0.0f;
+                const float du = mv ? __fdiv_rn(*up.gamma_u, scale[m]) : 0.0f;
+                const int xs = mv ? xsum[m] : 0;
+                double ss = 0.0;
+                float mx = 0.0f;
+#pragma unroll 1
+                for (int c = 0; c < TN / 32; ++c) {
+                    uint32_t vg[32], vu[32];
+                    tc::tmem_ld_32x32(tb + c * 32, vg);
+                    tc::tmem_ld_32x32(tb + TN + c * 32, vu);
+                    tc::tmem_ld_wait();
+                    const int nb = n0 + c * 32;
+                    if (!mv || nb >= N) continue;
+                    float hv[32];
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const float gv = dequant(static_cast<int>(vg[j]) - xs, dg);
+                        const float uv = dequant(static_cast<int>(vu[j]) - xs, du);
+                        const float t0 = gv > 0.0f ? gv : 0.0f;
+                        hv[j] = __fmul_rn(__fmul_rn(t0, t0), uv);
+                    }
+                    const int cnt = min(32, N - nb);
+                    float* hrow = up.h + (size_t)m * N + nb;
+                    if (cnt == 32 && (N & 3) == 0) {  // 16-byte stores
+#pragma unroll
+                        for (int j = 0; j < 32; j += 4)
+                            *reinterpret_cast<float4*>(hrow + j) = make_float4(hv[j], hv[j + 1], hv[j + 2], hv[j + 3]);
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 32; ++j)
+                            if (j < cnt) hrow[j] = hv[j];
+                    }
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        if (j >= cnt) break;
+                        ss = __dadd_rn(ss, __dmul_rn((double)hv[j], (double)hv[j]));
+                        mx = fmaxf(mx, fabsf(hv[j]));
+                    }
+                }
+                if (mv) {
+                    up.part_ss[(size_t)m * n_tiles + (tile % n_tiles)] = ss;
+                    up.part_max[(size_t)m * n_tiles + (tile % n_tiles)] = mx;
+                }
+                tc::fence_before_sync();
+                tc::mbar_arrive(aempty(a));
+                continue;
+            }
             const bool whole = !SK || (kb0 == 0 && kb1 == nkb);
             // a piece of a split tile goes to slot 2c (the CTA's first piece) or 2c + 1,
             // column-major, so that the 32 rows of a warp store one 128-byte line
@@ -608,13 +670,51 @@ cudaError_t launch_bn(const uint8_t* Wp, const float* gamma, int64_t N, int64_t 
     const int64_t units = tiles * ((K + BK - 1) / BK);
     const int64_t work = sk ? units : tiles;
     const unsigned grid = (unsigned)(work < sms ? work : sms);
-    kern<<<grid, THREADS, smem, s>>>(mapA, mapB, (int)M, (int)N, (int)K, gamma, scale, xsum, out, err, partials);
+    kern<<<grid, THREADS, smem, s>>>(mapA, mapB, mapB, (int)M, (int)N, (int)K, gamma, scale, xsum, out, err, partials,
+                                     FfnUpOut());
     e = cudaGetLastError();
     if (e != cudaSuccess || !sk) return e;
     return launch_pdl(gemm_sk_fixup_kernel<BN, PR>, dim3((unsigned)tiles, BN / 32), dim3(512), 0, s, (int)M, (int)N,
                       (int)K, (int)grid, (const uint32_t*)partials, gamma, scale, xsum, out);
 }
 }  // namespace
+
+cudaError_t launch_gemm_tc_dual(const uint8_t* Wg, const float* gg, const uint8_t* Wu, const float* gu, int64_t f,
+                                int64_t d, const int8_t* xq_g16t, const float* scale, const int32_t* xsum, int64_t M,
+                                const FfnUpOut& up, cudaStream_t s) {
+    if (M == 0 || f == 0) return cudaSuccess;
+    if (!gemm_tc_ok(f, d, Wg, xq_g16t) || !gemm_tc_ok(f, d, Wu, xq_g16t)) return cudaErrorInvalidValue;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    int sms = 148;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) sms = 148;
+    constexpr int BN = 256;
+    constexpr size_t smem = TileCfg<BN>::SMEM_BYTES;
+    CUtensorMap mapA, mapG, mapU;
+    if (!make_map(&mapA, xq_g16t, (uint64_t)M, (uint64_t)d, BM, BK, true) ||
+        !make_map(&mapG, Wg, (uint64_t)f, (uint64_t)(d / 4), BN / 2, BK / 4, false) ||
+        !make_map(&mapU, Wu, (uint64_t)f, (uint64_t)(d / 4), BN / 2, BK / 4, false))
+        return cudaErrorInvalidValue;
+    unsigned* err = nullptr;
+    cudaError_t e = device_error_word(&err);
+    if (e != cudaSuccess) return e;
+    auto kern = gemm_tc_kernel<BN, false, false, true>;
+    static bool attr_set[64];
+    if (dev >= 64 || !attr_set[dev]) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        if (dev < 64) attr_set[dev] = true;
+    }
+    const int64_t tiles = ((f + BN / 2 - 1) / (BN / 2)) * ((M + BM - 1) / BM);
+    const unsigned grid = (unsigned)(tiles < sms ? tiles : sms);
+    FfnUpOut u = up;
+    u.gamma_u = gu;
+    kern<<<grid, THREADS, smem, s>>>(mapA, mapG, mapU, (int)M, (int)f, (int)d, gg, scale, xsum, GemvOut(), err,
+                                     nullptr, u);
+    return cudaGetLastError();
+}
+
+int gemm_dual_parts(int64_t f) { return (int)((f + 127) / 128); }
 
 // Tile width: 256 weight rows per tile unless narrower tiles finish sooner. The
 // estimate is waves x relative time of one tile; a narrower tile still loads the

@@ -91,6 +91,20 @@ cudaError_t launch_gemm_tc(const uint8_t* Wp, const float* gamma, int64_t N, int
                            const GemvOut& out, cudaStream_t s, void* sk_ws = nullptr, size_t sk_ws_bytes = 0);
 size_t gemm_sk_workspace_bytes(int sms);
 
+// The FFN's gate and up projections in one tensor-core launch (M > 16): h =
+// max(g, 0)^2 * u [M, f] fp32 and, per token and 128-column tile,
+// part_ss = sum h^2 (fp64) and part_max = max |h| ([M, gemm_dual_parts(f)]).
+struct FfnUpOut {
+    float* h = nullptr;
+    double* part_ss = nullptr;
+    float* part_max = nullptr;
+    const float* gamma_u = nullptr;  // gamma of the up weight (the gate's is the launch's gamma)
+};
+cudaError_t launch_gemm_tc_dual(const uint8_t* Wg, const float* gg, const uint8_t* Wu, const float* gu, int64_t f,
+                                int64_t d, const int8_t* xq_g16t, const float* scale, const int32_t* xsum, int64_t M,
+                                const FfnUpOut& up, cudaStream_t s);
+int gemm_dual_parts(int64_t f);
+
 // 2-D uint8 TMA tensor map over [rows, cols] (cols contiguous), box [box_rows,
 // box_cols], optionally 128-byte swizzled; false when the driver refuses it.
 bool make_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows,
@@ -124,6 +138,11 @@ cudaError_t launch_ffn_tp_hstats(const float* g, const float* u, int64_t M, int6
 cudaError_t launch_ffn_tp_requant(const float* h, int64_t M, int64_t fl, int64_t f_total, const double* ss_all,
                                   const float* hmax_all, int layout, int8_t* q2, float* s2, int32_t* xsum2,
                                   cudaStream_t s);
+// subln + requantisation of h from per-tile partials (sum h^2 fp64, max |h|),
+// reduced in a fixed order per token; codes in `layout`.
+cudaError_t launch_ffn_requant_parts(const float* h, const double* part_ss, const float* part_max, int nparts,
+                                     int64_t M, int64_t f, int layout, int8_t* q2, float* s2, int32_t* xsum2,
+                                     cudaStream_t s);
 cudaError_t launch_ffn_tp_finish(const int32_t* acc, const float* gd, const float* s2, const uint16_t* residual,
                                  uint16_t* y, int64_t M, int64_t d, cudaStream_t s);
 

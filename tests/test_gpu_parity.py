@@ -596,3 +596,21 @@ def test_forward_ex_single_token_long_rows_rmsnorm(cuda_device, K):
     rq = oracle.forward_ex(np.concatenate([p[0] for p in ref_parts]), [p[1] for p in ref_parts], rows, bits(x),
                            rmsnorm=True)
     assert_bf16_exact(bits(yq), rq["y"])
+
+
+# ----------------------------------------------------------------------------- FFN, gate+up in one tensor-core launch
+
+@pytest.mark.parametrize("M,d,f", [(17, 256, 200), (40, 512, 1000), (300, 2560, 6912), (129, 4096, 1024)])
+def test_ffn_dual_gemm(cuda_device, M, d, f):
+    """M > 16: gate and up in one launch (128 + 128 weight rows per tile) whose
+    epilogue forms h and the per-tile sum h^2 / max |h|; then the requantisation
+    from those partials and the down projection (generic kernel for f = 200 and
+    1000, tensor cores otherwise). f = 200 and 1000 leave a partial last tile."""
+    Wg, Wu, Wd = (make_weights(f, d, 0.02, 7000 + d), make_weights(f, d, 0.02, 7001 + d),
+                  make_weights(d, f, 0.02, 7002 + d))
+    P = [pack_both(W, cuda_device) for W in (Wg, Wu, Wd)]
+    x = synth.activations(M, d, seed=7003 + M, outliers=False)
+    y = bl.ffn(P[0][0], P[0][1], P[1][0], P[1][1], P[2][0], P[2][1], x.to(cuda_device), residual=x.to(cuda_device))
+    ref = oracle.ffn_layer(P[0][2], P[0][3], P[1][2], P[1][3], P[2][2], P[2][3], bits(x), residual=bits(x))
+    assert_bf16_exact(bits(y), ref["y"])
+    assert bl.get_device_error() == 0
