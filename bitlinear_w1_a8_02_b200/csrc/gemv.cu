@@ -458,7 +458,11 @@ __global__ void __launch_bounds__(kThreads + 32, (NT == 1 && !BIG) ? 3 : 2) gemv
     static_assert(!DP || (FUSED && NT == 1), "the dp4a path reads one token's codes from shared memory");
     constexpr int NW = DUAL ? 2 : 1;  // weight streams
     extern __shared__ __align__(128) uint8_t dyn[];
-    __shared__ int red[kWarps][16][TOK];
+    // per-tile partial sums of the warps; double-buffered for one token group
+    // (tile t + 1 fills the other buffer while tile t's epilogue may still read
+    // its own, so one named barrier per tile suffices)
+    constexpr int RB = (NT == 1 && !DUAL) ? 2 : 1;
+    __shared__ int red_buf[RB][kWarps][16][TOK];
     __shared__ int red2[DUAL ? kWarps : 1][16][TOK];
     __shared__ float s_sh[TOK];
     __shared__ int xs_sh[TOK];
@@ -604,7 +608,9 @@ __global__ void __launch_bounds__(kThreads + 32, (NT == 1 && !BIG) ? 3 : 2) gemv
     consumer_sync();  // codes, code sums and dequantisation factors are ready
 
     uint32_t g = 0;
-    for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+    int it = 0;  // tiles done by this CTA
+    for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
+        auto& red = red_buf[RB == 2 ? (it & 1) : 0];
         const int n0 = tile * R;
         if constexpr (DP) {
             // One token: thread (row group rg, lane tl of T = 1024 / R) owns rows
@@ -781,7 +787,7 @@ __global__ void __launch_bounds__(kThreads + 32, (NT == 1 && !BIG) ? 3 : 2) gemv
                 if (a.out.acc) a.out.acc[o] = accv;
             }
         }
-        consumer_sync();
+        if (RB == 1) consumer_sync();  // the single buffer is reused by the next tile
     }
 }
 
