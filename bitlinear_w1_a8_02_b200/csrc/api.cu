@@ -9,6 +9,8 @@
 #include <atomic>
 
 #include <cuda_runtime.h>
+
+#include <algorithm>
 #include <stdint.h>
 
 #include "common.cuh"
@@ -27,23 +29,28 @@ inline size_t align_up(size_t v) { return (v + kWsAlign - 1) / kWsAlign * kWsAli
 inline bool aligned(const void* p, size_t a) { return (uintptr_t)p % a == 0; }
 
 // Workspace carving -----------------------------------------------------------
-// Tensor-core projections (M > 16) may split tiles across CTAs (stream-K) and
-// need scratch for the pieces; the smaller paths do not. Sized for 148 SMs
-// without asking the device (workspace sizes are host-only arithmetic); a device
-// with more SMs finds the scratch too small and keeps the data-parallel split.
+// A tensor-core projection (M > 16) whose shape takes the stream-K split needs
+// scratch for the pieces of split tiles; other shapes and the smaller paths do
+// not. The split is decided, and the scratch sized, for 148 SMs without asking
+// the device (workspace sizes are host-only arithmetic); a device with more SMs
+// finds the scratch too small and keeps the data-parallel split.
 constexpr int kStreamKSms = 148;
-inline size_t sk_bytes(int64_t M) { return M > 16 ? align_up(bl::gemm_sk_workspace_bytes(kStreamKSms)) : 0; }
+inline size_t sk_bytes(int64_t M, int64_t N, int64_t K) {
+    return M > 16 && bl::gemm_use_stream_k(M, N, K, kStreamKSms)
+               ? align_up(bl::gemm_sk_workspace_bytes(kStreamKSms))
+               : 0;
+}
 
 struct ForwardWs {
     size_t xq, scale, xsum, sk, sk_bytes, total;
 };
-inline ForwardWs forward_ws(int64_t M, int64_t K) {
+inline ForwardWs forward_ws(int64_t M, int64_t N, int64_t K) {
     ForwardWs w;
     w.xq = 0;
     w.scale = align_up((size_t)(M * K));
     w.xsum = w.scale + align_up((size_t)M * 4);
     w.sk = w.xsum + align_up((size_t)M * 4);
-    w.sk_bytes = sk_bytes(M);
+    w.sk_bytes = sk_bytes(M, N, K);
     w.total = w.sk + w.sk_bytes;
     return w;
 }
@@ -62,7 +69,9 @@ inline FfnWs ffn_ws(int64_t M, int64_t f, int64_t d) {
     w.s2 = w.q2 + align_up((size_t)(M * f));
     w.xsum2 = w.s2 + align_up((size_t)M * 4);
     w.sk = w.xsum2 + align_up((size_t)M * 4);
-    w.sk_bytes = sk_bytes(M);
+    // the down projection (M, d, f); gate and up with the split only on paths
+    // without the fused gate + up launch
+    w.sk_bytes = std::max(sk_bytes(M, d, f), sk_bytes(M, f, d));
     w.total = w.sk + w.sk_bytes;
     return w;
 }
@@ -82,7 +91,7 @@ inline TpUpWs tp_up_ws(int64_t M, int64_t fl, int64_t d) {
     w.g = w.xsum + align_up((size_t)M * 4);
     w.u = w.g + align_up((size_t)(M * fl) * 4);
     w.sk = w.u + align_up((size_t)(M * fl) * 4);
-    w.sk_bytes = sk_bytes(M);
+    w.sk_bytes = sk_bytes(M, fl, d);
     w.total = w.sk + w.sk_bytes;
     return w;
 }
@@ -95,7 +104,7 @@ inline TpDownWs tp_down_ws(int64_t M, int64_t d, int64_t fl) {
     w.xsum2 = align_up((size_t)(M * fl));
     w.y32 = w.xsum2 + align_up((size_t)M * 4);
     w.sk = w.y32 + align_up((size_t)(M * d) * 4);
-    w.sk_bytes = sk_bytes(M);
+    w.sk_bytes = sk_bytes(M, d, fl);
     w.total = w.sk + w.sk_bytes;
     return w;
 }
@@ -222,7 +231,7 @@ BL_API size_t bitlinear_workspace_bytes(int op, int64_t M, int64_t N, int64_t K)
     if (M < 0 || N < 0 || K < 0) return 0;
     switch (op) {
         case BL_OP_PACK: return pack_ws(N, K);
-        case BL_OP_FORWARD: return forward_ws(M, K).total;
+        case BL_OP_FORWARD: return forward_ws(M, N, K).total;
         case BL_OP_FFN: return ffn_ws(M, N, K).total;
         case BL_OP_VALIDATE: return kWsAlign;
         case BL_OP_FFN_TP_UP: return tp_up_ws(M, N, K).total;
@@ -280,7 +289,7 @@ namespace {
 bl_status forward_impl(const uint8_t* Wp, const float* gamma, int64_t N, int64_t K, const uint16_t* x,
                        int64_t M, bool rmsnorm, bl::GemvOut out, void* ws, size_t ws_bytes,
                        cudaStream_t s) {
-    const ForwardWs w = forward_ws(M, K);
+    const ForwardWs w = forward_ws(M, N, K);
     if (bl_status st = check_ws(ws, ws_bytes, w.total)) return st;
     if (bl_status st = check_device()) return st;
     char* base = (char*)ws;

@@ -90,6 +90,9 @@ cudaError_t launch_gemm_tc(const uint8_t* Wp, const float* gamma, int64_t N, int
                            const int8_t* xq_g16t, const float* scale, const int32_t* xsum, int64_t M,
                            const GemvOut& out, cudaStream_t s, void* sk_ws = nullptr, size_t sk_ws_bytes = 0);
 size_t gemm_sk_workspace_bytes(int sms);
+// Whether launch_gemm_tc splits tiles across CTAs (stream-K) for this shape on
+// `sms` SMs, given enough workspace.
+bool gemm_use_stream_k(int64_t M, int64_t N, int64_t K, int sms);
 
 // The FFN's gate and up projections in one tensor-core launch (M > 16): h =
 // max(g, 0)^2 * u [M, f] fp32 and, per token and 128-column tile,

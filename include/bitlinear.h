@@ -145,9 +145,10 @@ bl_status bitlinear_quant_act(const uint16_t* x, int64_t M, int64_t K,
  * bandwidth-bound GEMV (K % 256 == 0, Wp and x 16-byte aligned), quantising x
  * inside the same kernel for M <= 4 when the codes of all M tokens fit in 48 KiB
  * (M * (K + 64) bytes); larger M runs the tensor-core GEMM (K % 64 == 0, same
- * alignment, any N), which for M > 16 also uses the workspace for split-tile
- * partial sums; other shapes take a generic kernel. Every path gives the same
- * bits.
+ * alignment, any N), which for shapes whose tiles would leave most of the
+ * last wave idle splits tiles across CTAs and keeps their partial sums in the
+ * workspace (bitlinear_workspace_bytes includes that scratch only for such
+ * shapes); other shapes take a generic kernel. Every path gives the same bits.
  */
 bl_status bitlinear_forward(const uint8_t* Wp, const float* gamma, int64_t N, int64_t K,
                             const uint16_t* x, int64_t M, const uint16_t* residual,

@@ -59,11 +59,14 @@ def test_workspace_sizes():
     assert f(bl.BL_OP_FORWARD, -1, 1, 4) == 0
     for op in (bl.BL_OP_FORWARD, bl.BL_OP_FFN):
         assert f(op, 1, 2560, 2560) % 256 == 0
-    # tensor-core calls (M > 16) carry the stream-K scratch: two 128 x 256 int32
-    # slots per SM, sized for 148 SMs without asking a device
+    # tensor-core shapes that take the stream-K split carry its scratch (two
+    # 128 x 256 int32 slots per SM, sized for 148 SMs without asking a device);
+    # shapes that keep the data-parallel split and the M <= 16 paths do not
     sk = 2 * 148 * 128 * 256 * 4
-    assert f(bl.BL_OP_FORWARD, 17, 2560, 2560) >= 17 * 2560 + sk
-    assert f(bl.BL_OP_FFN, 17, 6912, 2560) >= sk
+    assert f(bl.BL_OP_FORWARD, 512, 2560, 6912) >= 512 * 6912 + sk   # 40 tiles of 54 k-blocks
+    assert f(bl.BL_OP_FFN, 512, 6912, 2560) >= sk                     # its down projection
+    assert f(bl.BL_OP_FORWARD, 17, 2560, 2560) < sk                   # 20 k-blocks: data-parallel
+    assert f(bl.BL_OP_FORWARD, 4096, 6912, 2560) < sk                 # 864 tiles fill the waves
     assert f(bl.BL_OP_FORWARD, 16, 2560, 2560) < sk
 
 
