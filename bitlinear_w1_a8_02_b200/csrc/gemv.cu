@@ -319,15 +319,16 @@ __device__ void fused_quantise(const GemvArgs& a, int KB, uint8_t* codes, uint32
 // one per group and pass. Codes in the interleaved single-token layout.
 constexpr int kBigGroups = 8;
 
+template <int G>
 __device__ void fused_quantise_big(const GemvArgs& a, int KB, uint8_t* codes, uint32_t* am_w, float* s_sh,
                                    int* xs_sh, float* deq_sh) {
     const int groups = KB / 4;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint4* xv = reinterpret_cast<const uint4*>(a.x);
     const float gamma = threadIdx.x == 0 ? *a.gamma : 0.0f;
-    uint4 v[kBigGroups][2];
+    uint4 v[G][2];
 #pragma unroll
-    for (int i = 0; i < kBigGroups; ++i) {
+    for (int i = 0; i < G; ++i) {
         const int c = threadIdx.x + i * kThreads;
         v[i][0] = v[i][1] = make_uint4(0u, 0u, 0u, 0u);
         if (c < groups) {
@@ -337,7 +338,7 @@ __device__ void fused_quantise_big(const GemvArgs& a, int KB, uint8_t* codes, ui
     }
     uint32_t mx = 0;  // zero groups (past the row) leave the maximum unchanged
 #pragma unroll
-    for (int i = 0; i < kBigGroups; ++i) mx = max(mx, absmax16(v[i][0], v[i][1]));
+    for (int i = 0; i < G; ++i) mx = max(mx, absmax16(v[i][0], v[i][1]));
     mx = __reduce_max_sync(0xffffffffu, mx);
     if (lane == 0) am_w[warp] = mx;
     consumer_sync();
@@ -347,7 +348,7 @@ __device__ void fused_quantise_big(const GemvArgs& a, int KB, uint8_t* codes, ui
     const float s = __fdiv_rn(kActRange, fmaxf(__uint_as_float(amb << 16), kActEps));
     int sum = 0;
 #pragma unroll
-    for (int i = 0; i < kBigGroups; ++i) {
+    for (int i = 0; i < G; ++i) {
         const int c = threadIdx.x + i * kThreads;
         if (c < groups) sum += quant_bf16x16<true, false>(v[i][0], v[i][1], s, codes + 16 * c, KB, false, 1.0f);
     }
@@ -451,8 +452,8 @@ __device__ __forceinline__ void bulk_copy(uint32_t dst, const void* src, uint32_
 // Units of the single-token path hold a.unit_rows rows (16, or 8 / 4 for rows
 // longer than 2 KiB, so a unit stays a contiguous ~32 KiB and the tiles are fine
 // enough to balance the CTAs); every other path streams 16-row units.
-template <int NT, int SRC, bool DUAL, bool DP, bool XT, bool BIG = false>
-__global__ void __launch_bounds__(kThreads + 32, (NT == 1 && !BIG) ? 3 : 2) gemv_mma_kernel(const GemvArgs a) {
+template <int NT, int SRC, bool DUAL, bool DP, bool XT, int BIG = 0>
+__global__ void __launch_bounds__(kThreads + 32, (NT == 1 && BIG <= 2) ? 3 : 2) gemv_mma_kernel(const GemvArgs a) {
     constexpr int TOK = 8 * NT;
     constexpr bool FUSED = SRC != SRC_CODES;
     static_assert(!DP || (FUSED && NT == 1), "the dp4a path reads one token's codes from shared memory");
@@ -593,8 +594,8 @@ __global__ void __launch_bounds__(kThreads + 32, (NT == 1 && !BIG) ? 3 : 2) gemv
 
     grid_dependency_wait();
     if (SRC == SRC_X) {
-        if constexpr (BIG)
-            fused_quantise_big(a, KB, codes, am_sh[0], s_sh, xs_sh, deq_sh);
+        if constexpr (BIG > 0)
+            fused_quantise_big<BIG>(a, KB, codes, am_sh[0], s_sh, xs_sh, deq_sh);
         else
             fused_quantise<DUAL, DP, XT>(a, KB, codes, am_sh, ss_sh, s_sh, xs_sh, deq_sh, deq2_sh);
     } else if (SRC == SRC_H) {
@@ -835,7 +836,7 @@ int sm_count() {
     return n;
 }
 
-template <int NT, int SRC, bool DUAL, bool DP = false, bool XT = false, bool BIG = false>
+template <int NT, int SRC, bool DUAL, bool DP = false, bool XT = false, int BIG = 0>
 cudaError_t launch_variant(const GemvArgs& a, dim3 grid, size_t smem, cudaStream_t s) {
     auto kern = gemv_mma_kernel<NT, SRC, DUAL, DP, XT, BIG>;
     static bool done[64];
@@ -948,7 +949,10 @@ cudaError_t launch_gemv(const uint8_t* Wp, const float* gamma, int64_t N, int64_
     const int unit_rows = one ? (KB <= 2048 ? 16 : KB <= 4096 ? 8 : 4) : 16;
     const bool big = one && !xt && K >= 8192 && K / 16 <= (int64_t)kBigGroups * kThreads;
     StreamPlan p;
-    cudaError_t e = plan_stream(a, N, K, M, 1, x_fused != nullptr, p, unit_rows, big ? 2 : 4);
+    // a token of at most 8192 codes needs two register groups per thread, which
+    // leaves room for three CTAs per SM; longer tokens need eight (two CTAs)
+    const bool big2 = big && K / 16 <= 2 * kThreads;
+    cudaError_t e = plan_stream(a, N, K, M, 1, x_fused != nullptr, p, unit_rows, big && !big2 ? 2 : 4);
     if (e != cudaSuccess) return e;
     const dim3 g1(p.grid_x, 1), g2(p.grid_x, (unsigned)((M + 15) / 16));
     if (xt) {
@@ -956,7 +960,8 @@ cudaError_t launch_gemv(const uint8_t* Wp, const float* gamma, int64_t N, int64_
         if (M <= 8) return launch_variant<1, SRC_CODES, false, false, true>(a, g1, p.smem, s);
         return launch_variant<2, SRC_CODES, false, false, true>(a, g2, p.smem, s);
     }
-    if (big) return launch_variant<1, SRC_X, false, true, false, true>(a, g1, p.smem, s);
+    if (big2) return launch_variant<1, SRC_X, false, true, false, 2>(a, g1, p.smem, s);
+    if (big) return launch_variant<1, SRC_X, false, true, false, kBigGroups>(a, g1, p.smem, s);
     if (x_fused) return launch_fused<SRC_X, false>(a, g1, p.smem, s);
     if (M <= 8) return launch_variant<1, SRC_CODES, false>(a, g1, p.smem, s);
     return launch_variant<2, SRC_CODES, false>(a, g2, p.smem, s);
