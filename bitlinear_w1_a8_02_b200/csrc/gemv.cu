@@ -947,10 +947,11 @@ cudaError_t launch_gemv(const uint8_t* Wp, const float* gamma, int64_t N, int64_
     const bool one = x_fused && M == 1;
     const int64_t KB = K / 4;
     const int unit_rows = one ? (KB <= 2048 ? 16 : KB <= 4096 ? 8 : 4) : 16;
-    const bool big = one && !xt && K >= 8192 && K / 16 <= (int64_t)kBigGroups * kThreads;
+    const bool big = one && !xt && K / 16 <= (int64_t)kBigGroups * kThreads;
     StreamPlan p;
     // a token of at most 8192 codes needs two register groups per thread, which
     // leaves room for three CTAs per SM; longer tokens need eight (two CTAs)
+    const bool big1 = big && K / 16 <= kThreads;
     const bool big2 = big && K / 16 <= 2 * kThreads;
     cudaError_t e = plan_stream(a, N, K, M, 1, x_fused != nullptr, p, unit_rows, big && !big2 ? 2 : 4);
     if (e != cudaSuccess) return e;
@@ -960,6 +961,7 @@ cudaError_t launch_gemv(const uint8_t* Wp, const float* gamma, int64_t N, int64_
         if (M <= 8) return launch_variant<1, SRC_CODES, false, false, true>(a, g1, p.smem, s);
         return launch_variant<2, SRC_CODES, false, false, true>(a, g2, p.smem, s);
     }
+    if (big1) return launch_variant<1, SRC_X, false, true, false, 1>(a, g1, p.smem, s);
     if (big2) return launch_variant<1, SRC_X, false, true, false, 2>(a, g1, p.smem, s);
     if (big) return launch_variant<1, SRC_X, false, true, false, kBigGroups>(a, g1, p.smem, s);
     if (x_fused) return launch_fused<SRC_X, false>(a, g1, p.smem, s);
