@@ -319,13 +319,14 @@ __device__ void fused_quantise(const GemvArgs& a, int KB, uint8_t* codes, uint32
 // one per group and pass. Codes in the interleaved single-token layout.
 constexpr int kBigGroups = 8;
 
-template <int G>
+template <int G, bool DUAL>
 __device__ void fused_quantise_big(const GemvArgs& a, int KB, uint8_t* codes, uint32_t* am_w, float* s_sh,
-                                   int* xs_sh, float* deq_sh) {
+                                   int* xs_sh, float* deq_sh, float* deq2_sh) {
     const int groups = KB / 4;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint4* xv = reinterpret_cast<const uint4*>(a.x);
     const float gamma = threadIdx.x == 0 ? *a.gamma : 0.0f;
+    const float gamma2 = DUAL && threadIdx.x == 0 ? *a.gamma2 : 0.0f;
     uint4 v[G][2];
 #pragma unroll
     for (int i = 0; i < G; ++i) {
@@ -357,6 +358,7 @@ __device__ void fused_quantise_big(const GemvArgs& a, int KB, uint8_t* codes, ui
     if (threadIdx.x == 0) {
         s_sh[0] = s;
         deq_sh[0] = __fdiv_rn(gamma, s);
+        if (DUAL) deq2_sh[0] = __fdiv_rn(gamma2, s);
     }
 }
 
@@ -595,7 +597,7 @@ __global__ void __launch_bounds__(kThreads + 32, (NT == 1 && BIG <= 2) ? 3 : 2) 
     grid_dependency_wait();
     if (SRC == SRC_X) {
         if constexpr (BIG > 0)
-            fused_quantise_big<BIG>(a, KB, codes, am_sh[0], s_sh, xs_sh, deq_sh);
+            fused_quantise_big<BIG, DUAL>(a, KB, codes, am_sh[0], s_sh, xs_sh, deq_sh, deq2_sh);
         else
             fused_quantise<DUAL, DP, XT>(a, KB, codes, am_sh, ss_sh, s_sh, xs_sh, deq_sh, deq2_sh);
     } else if (SRC == SRC_H) {
@@ -981,10 +983,18 @@ cudaError_t launch_ffn_up_fused(const uint8_t* Wg, const float* gg, const uint8_
     a.h = h;
     a.part_ss = part_ss;
     a.part_max = part_max;
+    // one token: the register quantiser (one L2 round trip for x), as in launch_gemv
+    const int groups = M == 1 && d / 16 <= (int64_t)kBigGroups * kThreads
+                           ? (d / 16 <= kThreads ? 1 : d / 16 <= 2 * kThreads ? 2 : kBigGroups)
+                           : 0;
     StreamPlan p;
-    cudaError_t e = plan_stream(a, f, d, M, 2, true, p);
+    cudaError_t e = plan_stream(a, f, d, M, 2, true, p, 16, groups == kBigGroups ? 2 : 4);
     if (e != cudaSuccess) return e;
-    return launch_fused<SRC_X, true>(a, dim3(p.grid_x, 1), p.smem, s);
+    const dim3 g1(p.grid_x, 1);
+    if (groups == 1) return launch_variant<1, SRC_X, true, true, false, 1>(a, g1, p.smem, s);
+    if (groups == 2) return launch_variant<1, SRC_X, true, true, false, 2>(a, g1, p.smem, s);
+    if (groups == kBigGroups) return launch_variant<1, SRC_X, true, true, false, kBigGroups>(a, g1, p.smem, s);
+    return launch_fused<SRC_X, true>(a, g1, p.smem, s);
 }
 
 cudaError_t launch_ffn_down_fused(const uint8_t* Wd, const float* gd, int64_t d, int64_t f,
