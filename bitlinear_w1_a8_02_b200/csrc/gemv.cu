@@ -313,6 +313,75 @@ __device__ void fused_quantise(const GemvArgs& a, int KB, uint8_t* codes, uint32
     }
 }
 
+// Up to four tokens with K <= 4096, so one 16-element group per thread and token
+// (instantiation BIG = -1): every token's group is loaded at once, one named
+// barrier serves the absmax (and RMSNorm sum) of all tokens, then each token is
+// quantised from registers. Per token the reductions are those of
+// fused_quantise, in the same order, so the codes and scales are the same bits.
+template <bool DUAL, bool IL, bool XT>
+__device__ void fused_quantise_few(const GemvArgs& a, int KB, uint8_t* codes, uint32_t (*am_sh)[kWarps],
+                                   double (*ss_sh)[kWarps], float* s_sh, int* xs_sh, float* deq_sh,
+                                   float* deq2_sh) {
+    const int M = a.M, groups = KB / 4;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int c0 = threadIdx.x;
+    const uint4* xv = reinterpret_cast<const uint4*>(a.x);
+    float gamma = 0.0f, gamma2 = 0.0f;
+    if (threadIdx.x == 0) {
+        gamma = *a.gamma;
+        if (DUAL) gamma2 = *a.gamma2;
+    }
+    const bool norm = XT && a.norm;
+    uint4 v[kFusedMaxTokens][2];
+#pragma unroll
+    for (int m = 0; m < kFusedMaxTokens; ++m) {
+        v[m][0] = v[m][1] = make_uint4(0u, 0u, 0u, 0u);
+        if (m < M && c0 < groups) {
+            v[m][0] = xv[(size_t)m * 2 * groups + 2 * c0];
+            v[m][1] = xv[(size_t)m * 2 * groups + 2 * c0 + 1];
+        }
+    }
+#pragma unroll
+    for (int m = 0; m < kFusedMaxTokens; ++m) {
+        if (m >= M) break;
+        uint32_t mx = absmax16(v[m][0], v[m][1]);  // 0 when this thread has no group
+        double ss = norm ? sumsq16(v[m][0], v[m][1]) : 0.0;
+        mx = __reduce_max_sync(0xffffffffu, mx);
+        if (norm) ss = warp_sum(ss);
+        if (lane == 0) {
+            am_sh[m][warp] = mx;
+            if (XT) ss_sh[m][warp] = ss;
+        }
+    }
+    consumer_sync();
+#pragma unroll
+    for (int m = 0; m < kFusedMaxTokens; ++m) {
+        if (m >= M) break;
+        uint32_t amb = am_sh[m][0];
+#pragma unroll
+        for (int w = 1; w < kWarps; ++w) amb = max(amb, am_sh[m][w]);
+        float amax = __uint_as_float(amb << 16), r = 1.0f;
+        if (norm) {  // unit-weight RMSNorm: max |fl(x r)| = fl(max |x| r)
+            double tot = ss_sh[m][0];
+#pragma unroll
+            for (int w = 1; w < kWarps; ++w) tot += ss_sh[m][w];
+            const float ms = __double2float_rn(__ddiv_rn(tot, (double)(4 * KB)));
+            r = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, kRmsEps)));
+            amax = __fmul_rn(amax, r);
+        }
+        const float s = __fdiv_rn(kActRange, fmaxf(amax, kActEps));
+        int sum = 0;
+        if (c0 < groups) sum = quant_bf16x16<IL, XT>(v[m][0], v[m][1], s, group_codes<IL>(codes, m, c0, KB), KB, norm, r);
+        sum = __reduce_add_sync(0xffffffffu, sum);
+        if (lane == 0) atomicAdd(&xs_sh[m], sum);
+        if (threadIdx.x == 0) {
+            s_sh[m] = s;
+            deq_sh[m] = __fdiv_rn(gamma, s);
+            if (DUAL) deq2_sh[m] = __fdiv_rn(gamma2, s);
+        }
+    }
+}
+
 // One token with a long row (BIG instantiation): each thread loads all of its
 // 16-element groups at once (at most kBigGroups), keeps them in registers for the
 // absmax and for the codes, so the token costs one round trip to L2 instead of
@@ -598,6 +667,8 @@ __global__ void __launch_bounds__(kThreads + 32, (NT == 1 && BIG <= 2) ? 3 : 2) 
     if (SRC == SRC_X) {
         if constexpr (BIG > 0)
             fused_quantise_big<BIG, DUAL>(a, KB, codes, am_sh[0], s_sh, xs_sh, deq_sh, deq2_sh);
+        else if constexpr (BIG < 0)
+            fused_quantise_few<DUAL, DP, XT>(a, KB, codes, am_sh, ss_sh, s_sh, xs_sh, deq_sh, deq2_sh);
         else
             fused_quantise<DUAL, DP, XT>(a, KB, codes, am_sh, ss_sh, s_sh, xs_sh, deq_sh, deq2_sh);
     } else if (SRC == SRC_H) {
@@ -856,6 +927,13 @@ cudaError_t launch_variant(const GemvArgs& a, dim3 grid, size_t smem, cudaStream
 // spend 7 of its 8 token columns on padding).
 template <int SRC, bool DUAL, bool XT = false>
 cudaError_t launch_fused(const GemvArgs& a, dim3 grid, size_t smem, cudaStream_t s) {
+    // K <= 4096 from x: the quantiser that loads every token's group at once
+    if constexpr (SRC == SRC_X) {
+        if (a.KB / 4 <= kThreads) {
+            if (a.M == 1) return launch_variant<1, SRC, DUAL, true, XT, -1>(a, grid, smem, s);
+            return launch_variant<1, SRC, DUAL, false, XT, -1>(a, grid, smem, s);
+        }
+    }
     if (a.M == 1) return launch_variant<1, SRC, DUAL, true, XT>(a, grid, smem, s);
     return launch_variant<1, SRC, DUAL, false, XT>(a, grid, smem, s);
 }
