@@ -1026,7 +1026,9 @@ cudaError_t launch_gemv(const uint8_t* Wp, const float* gamma, int64_t N, int64_
     // register budget allows two CTAs per SM).
     const bool one = x_fused && M == 1;
     const int64_t KB = K / 4;
-    const int unit_rows = one ? (KB <= 2048 ? 16 : KB <= 4096 ? 8 : 4) : 16;
+    // (8-row units also when 16-row tiles would leave SMs without one: 2560 -> 640
+    // runs 80 CTAs instead of 40)
+    const int unit_rows = one ? (KB <= 2048 ? ((N + 15) / 16 < sm_count() ? 8 : 16) : KB <= 4096 ? 8 : 4) : 16;
     const bool big = one && !xt && K / 16 <= (int64_t)kBigGroups * kThreads;
     StreamPlan p;
     // a token of at most 8192 codes needs two register groups per thread, which
