@@ -46,11 +46,11 @@ METRIC = "W1.58A8 BitLinear: decode GEMV HBM GB/s (% peak); prefill int8 TOPS (%
 DECODE_SHAPES = [(2560, 2560), (2560, 640), (2560, 6912), (6912, 2560)]  # (K, N)
 LAYERS = 30
 # DRAM bytes (read + write) per launch of the decode GEMV, averaged over the
-# step's four shapes: ncu captures of one launch per shape read 1,666,816 +
-# 437,248 + 4,452,352 + 4,460,544 bytes (0 written) for 2,723,840 packed bytes
-# per launch on average (x 1.011). Set to None whenever the kernel changes until
+# step's four shapes: ncu captures of one launch per shape read 1,664,512 +
+# 435,200 + 4,450,048 + 4,460,032 bytes (0 written) for 2,723,840 packed bytes
+# per launch on average (x 1.0105). Set to None whenever the kernel changes until
 # a new capture is taken.
-GEMV_TRAFFIC_PER_LAUNCH = 2754240
+GEMV_TRAFFIC_PER_LAUNCH = 2752448
 # The pages' only latency figure, quoted beside the whole-decoder-layer number as
 # context (not a target): whole-model CPU decode, ms per output token.
 PAGES_CPU_MS_PER_TOKEN = 29.0
@@ -281,7 +281,8 @@ def run_ours(args):
     achieved = (step_bytes / (LAYERS * len(DECODE_SHAPES))) / per_launch_s / 1e9
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
                 "frac": round(achieved / hbm_peak, 4), "traffic": GEMV_TRAFFIC_PER_LAUNCH,
-                "kernel": "gemv_mma_kernel<1,SRC_X,0,dp4a,0> (quantise + ternary GEMV + dequant, one launch per call)",
+                "kernel": "gemv_mma_kernel<1,SRC_X,0,dp4a,0,BIG=1|2> (register quantiser + ternary GEMV + dequant, "
+                          "one launch per call)",
                 "us_per_launch": round(per_launch_s * 1e6, 3),
                 "bytes_per_launch": step_bytes // (LAYERS * len(DECODE_SHAPES)),
                 "peak_kind": peak_kind}
