@@ -382,10 +382,11 @@ __device__ void fused_quantise_few(const GemvArgs& a, int KB, uint8_t* codes, ui
     }
 }
 
-// One token with a long row (BIG instantiation): each thread loads all of its
-// 16-element groups at once (at most kBigGroups), keeps them in registers for the
-// absmax and for the codes, so the token costs one round trip to L2 instead of
-// one per group and pass. Codes in the interleaved single-token layout.
+// One token (BIG = G instantiation): each thread loads all of its G 16-element
+// groups at once (at most kBigGroups), keeps them in registers for the absmax and
+// for the codes, so the token costs one round trip to L2 instead of one per group
+// and pass. Codes in the interleaved single-token layout. DUAL: the FFN's gate
+// and up projections share the codes; each gets its own gamma / s.
 constexpr int kBigGroups = 8;
 
 template <int G, bool DUAL>
@@ -518,11 +519,15 @@ __device__ __forceinline__ void bulk_copy(uint32_t dst, const void* src, uint32_
 // different banks.
 // XT: extended calls (row segments with their own gamma, RMSNorm of x); the
 // plain forward runs the instantiation without that code.
-// BIG: one token with a long row, quantised from registers (fused_quantise_big);
-// its registers allow two CTAs per SM.
+// BIG: how x is quantised when the kernel does it (SRC_X). G > 0: one token from
+// registers, G 16-element groups per thread (fused_quantise_big; with G = 8 the
+// registers allow two CTAs per SM, otherwise three); -1: up to four tokens with
+// K <= 4096, one group per thread and token (fused_quantise_few); 0: the
+// two-pass loop (fused_quantise).
 // Units of the single-token path hold a.unit_rows rows (16, or 8 / 4 for rows
 // longer than 2 KiB, so a unit stays a contiguous ~32 KiB and the tiles are fine
-// enough to balance the CTAs); every other path streams 16-row units.
+// enough to balance the CTAs; 8 also when 16-row tiles would leave SMs without
+// one); every other path streams 16-row units.
 template <int NT, int SRC, bool DUAL, bool DP, bool XT, int BIG = 0>
 __global__ void __launch_bounds__(kThreads + 32, (NT == 1 && BIG <= 2) ? 3 : 2) gemv_mma_kernel(const GemvArgs a) {
     constexpr int TOK = 8 * NT;
