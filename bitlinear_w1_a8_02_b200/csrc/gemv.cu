@@ -432,6 +432,78 @@ __device__ void fused_quantise_big(const GemvArgs& a, int KB, uint8_t* codes, ui
     }
 }
 
+// One token with f <= 8192 (the BIG = 2 instantiation of the down projection):
+// the partials and this thread's two groups of h are requested together, so the
+// token costs one round trip to L2 instead of one for the partials and one for
+// h; the reductions are those of finalise_quantise, in the same order.
+template <bool IL>
+__device__ void finalise_quantise_one(const GemvArgs& a, int KB, uint8_t* codes, float* s_sh, int* xs_sh,
+                                      float* r_sh, float* deq_sh) {
+    const int f = 4 * KB, groups = KB / 4;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    __shared__ double dred[kWarps];
+    __shared__ float fred[kWarps];
+    float gamma = 0.0f;
+    if (threadIdx.x == 0) gamma = *a.gamma;
+    const float4* hr = reinterpret_cast<const float4*>(a.hin);
+    float4 h[2][4];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const int c = threadIdx.x + i * kThreads;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) h[i][q] = c < groups ? hr[4 * c + q] : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    double ss = 0.0;
+    float hmax = 0.0f;
+#pragma unroll 1
+    for (int p = threadIdx.x; p < a.hin_parts; p += kThreads) {
+        ss = __dadd_rn(ss, a.hin_ss[p]);
+        hmax = fmaxf(hmax, a.hin_max[p]);
+    }
+    ss = warp_sum(ss);
+    hmax = warp_max(hmax);
+    if (lane == 0) {
+        dred[warp] = ss;
+        fred[warp] = hmax;
+    }
+    consumer_sync();
+    if (threadIdx.x == 0) {
+        double tot = dred[0];
+        float mx = fred[0];
+#pragma unroll 1
+        for (int w = 1; w < kWarps; ++w) {
+            tot = __dadd_rn(tot, dred[w]);
+            mx = fmaxf(mx, fred[w]);
+        }
+        const float ms = __double2float_rn(__ddiv_rn(tot, (double)f));
+        const float r = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, kRmsEps)));
+        const float s = __fdiv_rn(kActRange, fmaxf(__fmul_rn(mx, r), kActEps));
+        r_sh[0] = r;
+        s_sh[0] = s;
+        deq_sh[0] = __fdiv_rn(gamma, s);
+    }
+    consumer_sync();
+    const float r = r_sh[0], s = s_sh[0];
+    int sum = 0;
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const int c = threadIdx.x + i * kThreads;
+        if (c < groups) {
+            float v[16];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                v[4 * q] = __fmul_rn(h[i][q].x, r);
+                v[4 * q + 1] = __fmul_rn(h[i][q].y, r);
+                v[4 * q + 2] = __fmul_rn(h[i][q].z, r);
+                v[4 * q + 3] = __fmul_rn(h[i][q].w, r);
+            }
+            sum += quant_pack16<IL>(v, s, group_codes<IL>(codes, 0, c, KB), KB);
+        }
+    }
+    sum = __reduce_add_sync(0xffffffffu, sum);
+    if (lane == 0) atomicAdd(&xs_sh[0], sum);
+}
+
 // FFN glue inside the down projection (consumer threads): per token,
 // r = 1 / sqrtf(float(sum_j h_j^2 / f) + eps) from the up kernel's per-tile fp64
 // partials (fixed order: thread strides, warp butterfly, warps in index order),
@@ -677,7 +749,10 @@ __global__ void __launch_bounds__(kThreads + 32, (NT == 1 && BIG <= 2) ? 3 : 2) 
         else
             fused_quantise<DUAL, DP, XT>(a, KB, codes, am_sh, ss_sh, s_sh, xs_sh, deq_sh, deq2_sh);
     } else if (SRC == SRC_H) {
-        finalise_quantise<DP>(a, KB, codes, s_sh, xs_sh, r_sh, deq_sh);
+        if constexpr (BIG > 0)
+            finalise_quantise_one<DP>(a, KB, codes, s_sh, xs_sh, r_sh, deq_sh);
+        else
+            finalise_quantise<DP>(a, KB, codes, s_sh, xs_sh, r_sh, deq_sh);
     } else if (threadIdx.x < TOK && tok0 + (int)threadIdx.x < a.M) {
         const float s = a.scale[tok0 + threadIdx.x];
         s_sh[threadIdx.x] = s;
@@ -1095,6 +1170,8 @@ cudaError_t launch_ffn_down_fused(const uint8_t* Wd, const float* gd, int64_t d,
     StreamPlan p;
     cudaError_t e = plan_stream(a, d, f, M, 1, true, p);
     if (e != cudaSuccess) return e;
+    if (M == 1 && f / 16 <= 2 * kThreads)  // one token: partials and h in one round trip
+        return launch_variant<1, SRC_H, false, true, false, 2>(a, dim3(p.grid_x, 1), p.smem, s);
     return launch_fused<SRC_H, false>(a, dim3(p.grid_x, 1), p.smem, s);
 }
 
