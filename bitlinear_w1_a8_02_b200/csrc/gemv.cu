@@ -515,12 +515,14 @@ __device__ void finalise_quantise(const GemvArgs& a, int KB, uint8_t* codes, flo
                                   float* r_sh, float* deq_sh) {
     const int f = 4 * KB;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    __shared__ double dred[kWarps];
-    __shared__ float fred[kWarps];
+    __shared__ double dred[kFusedMaxTokens][kWarps];
+    __shared__ float fred[kFusedMaxTokens][kWarps];
     float gamma = 0.0f;
-    if (threadIdx.x == 0) gamma = *a.gamma;
-#pragma unroll 1
-    for (int m = 0; m < a.M; ++m) {
+    if (threadIdx.x < kFusedMaxTokens) gamma = *a.gamma;
+    // every token's partials in one pass (their loads overlap), one barrier for all
+#pragma unroll
+    for (int m = 0; m < kFusedMaxTokens; ++m) {
+        if (m >= a.M) break;
         double ss = 0.0;
         float hmax = 0.0f;
 #pragma unroll 1
@@ -531,27 +533,28 @@ __device__ void finalise_quantise(const GemvArgs& a, int KB, uint8_t* codes, flo
         ss = warp_sum(ss);
         hmax = warp_max(hmax);
         if (lane == 0) {
-            dred[warp] = ss;
-            fred[warp] = hmax;
+            dred[m][warp] = ss;
+            fred[m][warp] = hmax;
         }
-        consumer_sync();
-        if (threadIdx.x == 0) {
-            double tot = dred[0];
-            float mx = fred[0];
-#pragma unroll 1
-            for (int w = 1; w < kWarps; ++w) {
-                tot = __dadd_rn(tot, dred[w]);
-                mx = fmaxf(mx, fred[w]);
-            }
-            const float ms = __double2float_rn(__ddiv_rn(tot, (double)f));
-            const float r = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, kRmsEps)));
-            const float s = __fdiv_rn(kActRange, fmaxf(__fmul_rn(mx, r), kActEps));
-            r_sh[m] = r;
-            s_sh[m] = s;
-            deq_sh[m] = __fdiv_rn(gamma, s);
-        }
-        consumer_sync();
     }
+    consumer_sync();
+    if (threadIdx.x < a.M && threadIdx.x < kFusedMaxTokens) {  // thread m: token m's r, s2 (warps in order)
+        const int m = threadIdx.x;
+        double tot = dred[m][0];
+        float mx = fred[m][0];
+#pragma unroll 1
+        for (int w = 1; w < kWarps; ++w) {
+            tot = __dadd_rn(tot, dred[m][w]);
+            mx = fmaxf(mx, fred[m][w]);
+        }
+        const float ms = __double2float_rn(__ddiv_rn(tot, (double)f));
+        const float r = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, kRmsEps)));
+        const float s = __fdiv_rn(kActRange, fmaxf(__fmul_rn(mx, r), kActEps));
+        r_sh[m] = r;
+        s_sh[m] = s;
+        deq_sh[m] = __fdiv_rn(gamma, s);
+    }
+    consumer_sync();
     const int groups = KB / 4;
 #pragma unroll 1
     for (int m = 0; m < a.M; ++m) {
