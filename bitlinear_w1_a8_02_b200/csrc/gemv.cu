@@ -685,7 +685,11 @@ __global__ void __launch_bounds__(kThreads + 32, (NT == 1 && BIG <= 2) ? 3 : 2) 
                     const int c0 = sg * cps;
                     const uint32_t segb = (uint32_t)(min(cps, nchunks - c0) * 64);
                     tc::mbar_arrive_expect_tx(full(st), segb * rows * NW);
-                    if (!waited) {  // everything above touches shared memory only
+                    // The first kStages units are copied before the dependency wait: the
+                    // packed weights are not written by a kernel that lets this one start
+                    // early (the library's early-triggering kernels never write them),
+                    // so the ring fills while the previous kernel finishes.
+                    if (!waited && g >= (uint32_t)kStages) {
                         grid_dependency_wait();
                         waited = true;
                     }

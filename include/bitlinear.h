@@ -25,6 +25,14 @@
  *     bitlinear_get_device_error, which say so.
  *   - No C++ exception crosses this boundary. A failed launch returns BL_ERR_CUDA.
  *   - Calls on different streams may overlap only if their workspaces differ.
+ *   - Kernels launch with programmatic dependent launch: a call's kernel may start
+ *     while the previous kernel in the stream finishes, and waits for it before
+ *     reading its inputs x / h or writing anything. The packed weights (Wp, Wg,
+ *     Wu, Wd) are the exception: the streamed GEMV starts copying them before that
+ *     wait. So packed weights must not be written by the kernel just before the
+ *     call in the same stream if that kernel triggers programmatic dependent launch
+ *     early (the library's own kernels that do never write weights; the packing
+ *     calls, host copies and ordinary kernels complete before a call starts).
  *
  * Packed weight format (this library's reading; the paper card, "Method
  * Adaptation", only fixes four ternary weights per 8-bit value): Wp is [N, K/4]
