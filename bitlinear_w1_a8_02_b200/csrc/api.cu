@@ -302,11 +302,8 @@ bl_status forward_impl(const uint8_t* Wp, const float* gamma, int64_t N, int64_t
     if ((path == Path::GemmTc && !bl::gemm_segments_ok(out, N)) ||
         ((path == Path::GemvFast || path == Path::GemvTc) && !bl::gemv_segments_ok(out, N)))
         path = Path::GemvGeneric;
-    // one kernel (quantise + GEMV) up to 4 tokens, except 4 tokens with K > 4096, where
-    // the in-kernel quantisation of every CTA costs more than the separate act-quant
-    // launch (6912 -> 2560 at M = 4: 6.90 us fused, 6.16 us with act-quant; 2 and 3
-    // tokens: 4.83 / 5.90 us fused, 6.05 / 6.10 us with it)
-    if (path == Path::GemvFast && bl::gemv_fused_ok(M, K) && (M <= 3 || K <= 4096))
+    // one kernel (quantise + GEMV) up to 4 tokens where that beats the separate act-quant
+    if (path == Path::GemvFast && bl::gemv_fused_ok(M, K) && bl::gemv_fused_pays(M, N, K))
         return cuda_status(bl::launch_gemv(Wp, gamma, N, K, nullptr, nullptr, nullptr, M, out, s, x, rmsnorm));
     BL_TRY(bl::launch_act_quant(x, M, K, layout_of(path), xq, scale, xsum, s, rmsnorm));
     return project(path, Wp, gamma, N, K, xq, scale, xsum, M, out, s, base + w.sk, w.sk_bytes);

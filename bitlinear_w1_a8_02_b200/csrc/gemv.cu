@@ -1091,6 +1091,16 @@ bool gemv_segments_ok(const GemvOut& out, int64_t N) {
     return true;
 }
 
+// The single kernel (quantise + GEMV) for the forward: every CTA quantises all M
+// tokens, which costs more than the separate act-quant launch only for four
+// tokens with K > 4096 on a grid of at most two 16-row tiles per SM (measured:
+// 6912 -> 2560 at M = 4, 160 tiles: 6.90 us fused, 6.16 us with act-quant;
+// 8192 -> 28672 at M = 4, 1792 tiles: 17.1 us fused, 22.7 us with it; two and
+// three tokens are faster fused at 6912 -> 2560 too).
+bool gemv_fused_pays(int64_t M, int64_t N, int64_t K) {
+    return M <= 3 || K <= 4096 || (N + 15) / 16 > 2 * (int64_t)sm_count();
+}
+
 bool gemv_fused_ok(int64_t M, int64_t K) {
     return M >= 1 && M <= kFusedMaxTokens && (size_t)M * (K + 64) <= (size_t)kFusedSmemLimit;
 }

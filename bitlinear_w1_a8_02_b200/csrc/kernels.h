@@ -57,6 +57,8 @@ __host__ __device__ __forceinline__ int gamma_index(const GemvOut& o, int n) {
 // (16-byte aligned bf16 x, gemv_fused_ok(M, K)), are computed inside the kernel.
 bool gemv_fast_ok(int64_t N, int64_t K);
 bool gemv_fused_ok(int64_t M, int64_t K);
+// gemv_fused_ok and also faster than the separate act-quant launch for this shape
+bool gemv_fused_pays(int64_t M, int64_t N, int64_t K);
 bool gemv_segments_ok(const GemvOut& out, int64_t N);  // segment ends on 16-row tiles
 cudaError_t launch_gemv(const uint8_t* Wp, const float* gamma, int64_t N, int64_t K,
                         const int8_t* Xp, const float* scale, const int32_t* xsum, int64_t M,

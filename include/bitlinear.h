@@ -151,8 +151,9 @@ bl_status bitlinear_quant_act(const uint16_t* x, int64_t M, int64_t K,
  *   ws        device workspace of bitlinear_workspace_bytes(BL_OP_FORWARD, M, N, K) bytes
  * Kernel choice: M <= 16 streams the packed weights once through a
  * bandwidth-bound GEMV (K % 256 == 0, Wp and x 16-byte aligned), quantising x
- * inside the same kernel for M <= 4 (M <= 3 when K > 4096) when the codes of all
- * M tokens fit in 48 KiB (M * (K + 64) bytes); larger M runs the tensor-core GEMM (K % 64 == 0, same
+ * inside the same kernel for M <= 4 (not for four tokens with K > 4096 on small
+ * N, where the separate quantisation is faster) when the codes of all M tokens
+ * fit in 48 KiB (M * (K + 64) bytes); larger M runs the tensor-core GEMM (K % 64 == 0, same
  * alignment, any N), which for shapes whose tiles would leave most of the
  * last wave idle splits tiles across CTAs and keeps their partial sums in the
  * workspace (bitlinear_workspace_bytes includes that scratch only for such
