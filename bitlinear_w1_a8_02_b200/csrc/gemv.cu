@@ -313,12 +313,14 @@ __device__ void fused_quantise(const GemvArgs& a, int KB, uint8_t* codes, uint32
     }
 }
 
-// Up to four tokens with K <= 4096, so one 16-element group per thread and token
-// (instantiation BIG = -1): every token's group is loaded at once, one named
-// barrier serves the absmax (and RMSNorm sum) of all tokens, then each token is
-// quantised from registers. Per token the reductions are those of
-// fused_quantise, in the same order, so the codes and scales are the same bits.
-template <bool DUAL, bool IL, bool XT>
+// Up to MT tokens with G 16-element groups per thread and token (instantiations
+// BIG = -1: four tokens, K <= 4096; BIG = -2: two tokens, K <= 8192): every
+// token's groups are loaded at once, one named barrier serves the absmax (and
+// RMSNorm sum) of all tokens, then each token is quantised from registers. Per
+// token the reductions are those of fused_quantise (a thread's groups in order,
+// then the warp, then the warps in order), so the codes and scales are the same
+// bits.
+template <bool DUAL, bool IL, bool XT, int MT, int G>
 __device__ void fused_quantise_few(const GemvArgs& a, int KB, uint8_t* codes, uint32_t (*am_sh)[kWarps],
                                    double (*ss_sh)[kWarps], float* s_sh, int* xs_sh, float* deq_sh,
                                    float* deq2_sh) {
@@ -332,20 +334,28 @@ __device__ void fused_quantise_few(const GemvArgs& a, int KB, uint8_t* codes, ui
         if (DUAL) gamma2 = *a.gamma2;
     }
     const bool norm = XT && a.norm;
-    uint4 v[kFusedMaxTokens][2];
+    uint4 v[MT][G][2];
 #pragma unroll
-    for (int m = 0; m < kFusedMaxTokens; ++m) {
-        v[m][0] = v[m][1] = make_uint4(0u, 0u, 0u, 0u);
-        if (m < M && c0 < groups) {
-            v[m][0] = xv[(size_t)m * 2 * groups + 2 * c0];
-            v[m][1] = xv[(size_t)m * 2 * groups + 2 * c0 + 1];
+    for (int m = 0; m < MT; ++m)
+#pragma unroll
+        for (int i = 0; i < G; ++i) {
+            const int c = c0 + i * kThreads;
+            v[m][i][0] = v[m][i][1] = make_uint4(0u, 0u, 0u, 0u);
+            if (m < M && c < groups) {
+                v[m][i][0] = xv[(size_t)m * 2 * groups + 2 * c];
+                v[m][i][1] = xv[(size_t)m * 2 * groups + 2 * c + 1];
+            }
         }
-    }
 #pragma unroll
-    for (int m = 0; m < kFusedMaxTokens; ++m) {
+    for (int m = 0; m < MT; ++m) {
         if (m >= M) break;
-        uint32_t mx = absmax16(v[m][0], v[m][1]);  // 0 when this thread has no group
-        double ss = norm ? sumsq16(v[m][0], v[m][1]) : 0.0;
+        uint32_t mx = 0;  // 0 when this thread has no group
+        double ss = 0.0;
+#pragma unroll
+        for (int i = 0; i < G; ++i) {
+            mx = max(mx, absmax16(v[m][i][0], v[m][i][1]));
+            if (norm) ss += sumsq16(v[m][i][0], v[m][i][1]);
+        }
         mx = __reduce_max_sync(0xffffffffu, mx);
         if (norm) ss = warp_sum(ss);
         if (lane == 0) {
@@ -355,7 +365,7 @@ __device__ void fused_quantise_few(const GemvArgs& a, int KB, uint8_t* codes, ui
     }
     consumer_sync();
 #pragma unroll
-    for (int m = 0; m < kFusedMaxTokens; ++m) {
+    for (int m = 0; m < MT; ++m) {
         if (m >= M) break;
         uint32_t amb = am_sh[m][0];
 #pragma unroll
@@ -371,7 +381,12 @@ __device__ void fused_quantise_few(const GemvArgs& a, int KB, uint8_t* codes, ui
         }
         const float s = __fdiv_rn(kActRange, fmaxf(amax, kActEps));
         int sum = 0;
-        if (c0 < groups) sum = quant_bf16x16<IL, XT>(v[m][0], v[m][1], s, group_codes<IL>(codes, m, c0, KB), KB, norm, r);
+#pragma unroll
+        for (int i = 0; i < G; ++i) {
+            const int c = c0 + i * kThreads;
+            if (c < groups)
+                sum += quant_bf16x16<IL, XT>(v[m][i][0], v[m][i][1], s, group_codes<IL>(codes, m, c, KB), KB, norm, r);
+        }
         sum = __reduce_add_sync(0xffffffffu, sum);
         if (lane == 0) atomicAdd(&xs_sh[m], sum);
         if (threadIdx.x == 0) {
@@ -751,8 +766,11 @@ __global__ void __launch_bounds__(kThreads + 32, (NT == 1 && BIG <= 2) ? 3 : 2) 
     if (SRC == SRC_X) {
         if constexpr (BIG > 0)
             fused_quantise_big<BIG, DUAL>(a, KB, codes, am_sh[0], s_sh, xs_sh, deq_sh, deq2_sh);
-        else if constexpr (BIG < 0)
-            fused_quantise_few<DUAL, DP, XT>(a, KB, codes, am_sh, ss_sh, s_sh, xs_sh, deq_sh, deq2_sh);
+        else if constexpr (BIG == -1)
+            fused_quantise_few<DUAL, DP, XT, kFusedMaxTokens, 1>(a, KB, codes, am_sh, ss_sh, s_sh, xs_sh, deq_sh,
+                                                                 deq2_sh);
+        else if constexpr (BIG == -2)
+            fused_quantise_few<DUAL, DP, XT, 2, 2>(a, KB, codes, am_sh, ss_sh, s_sh, xs_sh, deq_sh, deq2_sh);
         else
             fused_quantise<DUAL, DP, XT>(a, KB, codes, am_sh, ss_sh, s_sh, xs_sh, deq_sh, deq2_sh);
     } else if (SRC == SRC_H) {
@@ -1019,6 +1037,10 @@ cudaError_t launch_fused(const GemvArgs& a, dim3 grid, size_t smem, cudaStream_t
         if (a.KB / 4 <= kThreads) {
             if (a.M == 1) return launch_variant<1, SRC, DUAL, true, XT, -1>(a, grid, smem, s);
             return launch_variant<1, SRC, DUAL, false, XT, -1>(a, grid, smem, s);
+        }
+        if (a.M <= 2 && a.KB / 4 <= 2 * kThreads) {  // two tokens, K <= 8192
+            if (a.M == 1) return launch_variant<1, SRC, DUAL, true, XT, -2>(a, grid, smem, s);
+            return launch_variant<1, SRC, DUAL, false, XT, -2>(a, grid, smem, s);
         }
     }
     if (a.M == 1) return launch_variant<1, SRC, DUAL, true, XT>(a, grid, smem, s);

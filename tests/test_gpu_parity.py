@@ -124,6 +124,24 @@ def test_forward_batched_decode(cuda_device, K, N, M):
     check_forward_full(Wp, gamma, Wp_ref, g_ref, x, cuda_device)
 
 
+@pytest.mark.parametrize("K,N,M", [(8192, 28672, 4), (6912, 2560, 4), (6912, 2560, 3), (2560, 2560, 3)])
+def test_forward_few_tokens_quantiser_routes(cuda_device, K, N, M):
+    """2 to 4 tokens take one of three quantisation routes: the in-kernel
+    quantiser that loads every token's group at once (K <= 4096), the per-token
+    in-kernel loop (K > 4096, or four tokens on a large grid: 8192 -> 28672 has
+    1792 16-row tiles), or the separate act-quant kernel (four tokens with
+    K > 4096 on a grid of at most two tiles per SM: 6912 -> 2560). All must give
+    the oracle's bits; the large shape is checked on sampled rows."""
+    W = make_weights(N, K, synth.SIGMA_100B if K * N > 10**8 else 0.02, seed=7000 + K + M)
+    Wp, gamma, Wp_ref, g_ref = pack_both(W, cuda_device)
+    x = synth.activations(M, K, seed=7100 + M, outliers=True)
+    if K * N > 10**8:
+        rows = sample_indices(N, 256, seed=M + 71)
+        check_forward_sampled(Wp, gamma, Wp_ref, g_ref, x, cuda_device, rows, np.arange(M))
+    else:
+        check_forward_full(Wp, gamma, Wp_ref, g_ref, x, cuda_device)
+
+
 @pytest.mark.parametrize("M", [17, 512, 2048, 4096])
 @pytest.mark.parametrize("K,N", [(2560, 6912), (6912, 2560)])
 def test_forward_prefill_sampled(cuda_device, K, N, M):
