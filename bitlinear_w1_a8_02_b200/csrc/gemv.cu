@@ -612,8 +612,8 @@ __device__ __forceinline__ void bulk_copy(uint32_t dst, const void* src, uint32_
 // BIG: how x is quantised when the kernel does it (SRC_X). G > 0: one token from
 // registers, G 16-element groups per thread (fused_quantise_big; with G = 8 the
 // registers allow two CTAs per SM, otherwise three); -1: up to four tokens with
-// K <= 4096, one group per thread and token (fused_quantise_few); 0: the
-// two-pass loop (fused_quantise).
+// K <= 4096, one group per thread and token, -2: two tokens with K <= 8192, two
+// groups (fused_quantise_few); 0: the two-pass loop (fused_quantise).
 // Units of the single-token path hold a.unit_rows rows (16, or 8 / 4 for rows
 // longer than 2 KiB, so a unit stays a contiguous ~32 KiB and the tiles are fine
 // enough to balance the CTAs; 8 also when 16-row tiles would leave SMs without
