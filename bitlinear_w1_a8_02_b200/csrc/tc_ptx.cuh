@@ -1,6 +1,6 @@
 // Inline-PTX wrappers for the sm_100a pieces the tensor-core kernels use:
-// mbarriers (with bounded waits), TMA tile loads and L2 prefetches (no
-// multicast), tcgen05 TMEM allocation, MMA issue/commit (A from shared memory
+// mbarriers (with bounded waits), TMA tile loads into this CTA's own shared
+// memory and L2 prefetches, tcgen05 TMEM allocation, MMA issue/commit (A from shared memory
 // or from TMEM), TMEM loads and stores, cluster barriers and asynchronous adds
 // into a peer CTA's shared memory, and the shared-memory matrix descriptor of
 // the 128-byte-swizzled K-major operand layout.
