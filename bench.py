@@ -45,6 +45,10 @@ sys.path.insert(0, ROOT)
 METRIC = "W1.58A8 BitLinear: decode GEMV HBM GB/s (% peak); prefill int8 TOPS (% peak)"
 DECODE_SHAPES = [(2560, 2560), (2560, 640), (2560, 6912), (6912, 2560)]  # (K, N)
 LAYERS = 30
+# the headline workload and its inputs, named the same way by both arms
+WORKLOAD = ("decode_2b: M=1, (K,N) in {(2560,2560),(2560,640),(2560,6912),(6912,2560)}, "
+            "30 layer copies each, 120 BitLinear calls per step")
+DATA = "synthetic (seeded N(0,0.02^2) weights, N(0,1) activations with 1% x20 outlier channels)"
 # DRAM bytes (read + write) per launch of the decode GEMV, averaged over the
 # step's four shapes: ncu captures of one launch per shape read 1,664,512 +
 # 435,712 + 4,449,792 + 4,460,288 bytes (0 written) for 2,723,840 packed bytes
@@ -311,9 +315,8 @@ def run_ours(args):
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
-        "data": "synthetic (seeded N(0,0.02^2) weights, N(0,1) activations with 1% x20 outlier channels)",
-        "config": {"workload": "decode_2b: M=1, (K,N) in {(2560,2560),(2560,640),(2560,6912),(6912,2560)}, "
-                               "30 layer copies each, 120 BitLinear calls per step",
+        "data": DATA,
+        "config": {"workload": WORKLOAD,
                    "M": 1, "layers": LAYERS, "calls_per_step": LAYERS * len(DECODE_SHAPES),
                    "packed_bytes_per_step": step_bytes,
                    "l2": "inputs larger than L2: 327 MB of packed weights per step vs 126 MB L2",
@@ -731,9 +734,9 @@ def run_reference(args):
         "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
-        "data": "synthetic",
-        "config": {"workload": "decode_2b: M=1, (K,N) in {(2560,2560),(2560,640),(2560,6912),(6912,2560)}",
-                   "M": 1, "sample": sample},
+        "data": DATA,
+        "config": {"workload": WORKLOAD, "M": 1, "layers": LAYERS,
+                   "calls_per_step": LAYERS * len(DECODE_SHAPES), "sample": sample},
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
