@@ -38,6 +38,13 @@ def test_bf16_rounding_matches_torch():
     ours = oracle.f32_to_bf16(vals)
     ref = bf16_bits(torch.from_numpy(vals).to(torch.bfloat16))
     assert np.array_equal(ours, ref)
+    # NaNs whose payload sits only in the low half, or that rounding up would carry
+    # into the sign, stay NaNs of the same sign (exponent all ones, mantissa not 0)
+    nans = np.array([0x7F800001, 0xFF800001, 0x7FFFFFFF, 0xFFFFFFFF, 0x7FC00000], np.uint32).view(np.float32)
+    out = oracle.f32_to_bf16(nans).astype(np.uint32)
+    assert np.all((out & 0x7F80) == 0x7F80) and np.all((out & 0x007F) != 0)
+    assert (out >> 15).tolist() == [0, 1, 0, 1, 0]
+    assert np.all(np.isnan(torch.from_numpy(nans).to(torch.bfloat16).float().numpy()))
     back = oracle.bf16_to_f32(ours)
     assert np.array_equal(back, torch.from_numpy(ours.view(np.int16)).view(torch.bfloat16).float().numpy())
 
@@ -104,6 +111,8 @@ def test_worked_4x4_example():
     out = oracle.forward(Wp, gamma, bf16_bits(torch.tensor(g["x"]).to(torch.bfloat16)))
     assert out["acc"].tolist() == g["acc"]
     assert np.array_equal(out["y"], y)
+    assert out["xq"].tolist() == g["xq"] and out["xsum"].tolist() == g["xsum"]
+    assert out["s"].tolist() == np.array(g["s"], np.float32).tolist()
 
 
 # ----------------------------------------------------------------------------- weights
@@ -127,6 +136,11 @@ def test_absmean_closed_forms():
     W = (np.arange(1, 4097, dtype=np.float32) * np.float32(2.0 ** -12)) * np.where(np.arange(4096) % 2, 1, -1)
     exact = math.fsum(abs(float(v)) for v in W) / W.size
     assert oracle.absmean(W.astype(np.float32)) == np.float32(exact)
+    # one rounding, of the fp64 quotient: sum = 3 + 5 * 2^-23 (exact in fp64), and
+    # sum / 3 = 1 + (5/3) 2^-23 rounds to 1 + 2 * 2^-23. Rounding the sum to fp32
+    # first would give 3 + 4 * 2^-23 (a tie, to even), then 1 + 2^-23.
+    W3 = np.array([1.0, 1.0, 1.0 + 5 * 2.0 ** -23], np.float32)
+    assert oracle.absmean(W3) == np.float32(1.0 + 2.0 ** -22)
     # all-zero W: gamma = 0, every code 0
     Z = np.zeros((3, 8), np.float32)
     Wp, g = oracle.pack_weights(Z)
@@ -234,6 +248,12 @@ def test_relu2_gate_values():
     assert oracle.relu2_gate(2.0, 3.0) == 12.0
     assert oracle.relu2_gate(-2.0, 3.0) == 0.0
     assert oracle.relu2_gate(0.5, -4.0) == -1.0
+    # The square is rounded to fp32 before u multiplies it. With t = 1 + 2^-12 the
+    # exact square 1 + 2^-11 + 2^-24 lies halfway between two fp32 values and rounds
+    # to the even one, 1 + 2^-11; times u = 1 + 2^-11 that is 1 + 2^-10 + 2^-22,
+    # exact. Multiplying t * (t * u), or rounding the exact triple product once,
+    # gives 1 + 2^-10 + 2^-22 + 2^-23 instead.
+    assert oracle.relu2_gate(1 + 2.0 ** -12, 1 + 2.0 ** -11) == 1 + 2.0 ** -10 + 2.0 ** -22
 
 
 def test_subln_rms_closed_form():
@@ -490,3 +510,70 @@ def test_ffn_tensor_parallel_pieces_compose_to_the_whole_layer(P):
     assert np.array_equal(acc.astype(np.int32), ref["accd"])
     y = oracle.dequant(acc.astype(np.int32), packed[2][0][1], s2, residual=x)
     assert np.array_equal(y, ref["y"])
+
+
+def test_pack_weights_global_keeps_the_eps():
+    """Two one-row shards of the tensor of the eps example: mean |W| = 1/4 over the
+    whole tensor, and w0 / (1/4 + 1e-5) < 0.5 gives code 0, where w0 / (1/4) =
+    0.5 + 2^-18 would give 1. Codes [0, 1, 1, 1] are stored as q + 1 = [1, 2, 2, 2]
+    at bits 0, 2, 4, 6: 1 + 2*4 + 2*16 + 2*64 = 169 (170 without the eps)."""
+    row = [0.125 + 2.0 ** -20, 0.375 - 2.0 ** -20, 0.25, 0.25]
+    shards = [np.array([row], np.float32), np.array([row], np.float32)]
+    total = sum(oracle.absmean_sum(w) for w in shards)
+    assert total == 2.0
+    for w in shards:
+        Wp, g = oracle.pack_weights_global(w, total, 8)
+        assert g == np.float32(0.25)
+        assert Wp.tolist() == [[169]]
+
+
+def test_ffn_tensor_parallel_statistics_are_exact_sums():
+    """A rank's subln statistics: ss is the fp64 sum of the exact squares of its h
+    (each square of an fp32 value is exact in fp64), so it agrees with the
+    correctly rounded sum to within the rounding of 200 fp64 additions; squares
+    rounded to fp32 first would be off by ~1e-8 relative. hmax is max |h|."""
+    d, f, M = 64, 200, 5
+    Wg, gg = oracle.pack_weights(bf16_bits(synth.weights(f, d, 0.02, 80)))
+    Wu, gu = oracle.pack_weights(bf16_bits(synth.weights(f, d, 0.02, 81)))
+    x = bf16_bits(synth.activations(M, d, seed=83, outliers=True))
+    h, ss, hmax = oracle.ffn_tp_up(Wg, gg, Wu, gu, x)
+    assert np.count_nonzero(h) > M * f // 4
+    for m in range(M):
+        exact = math.fsum(float(v) ** 2 for v in h[m])
+        assert abs(ss[m] - exact) <= 1e-12 * exact
+        assert hmax[m] == np.abs(h[m]).max()
+
+
+def test_ffn_tensor_parallel_requantisation_rounds_like_the_whole_layer():
+    """The rank-local requantisation with the global statistics reproduces, code for
+    code, the subln then per-token quantisation of the whole layer: hn = fl(h r),
+    then rint(fl(hn s2)). h is drawn uniform in [-1, 1] (codes spread over the whole
+    int8 range) and large enough that the other rounding order, rint(fl(h fl(r
+    s2))), moves some code; the test checks that it does. The down weights are a
+    row of +1 and a row of seeded ternary codes, so a moved code changes acc."""
+    rng = np.random.default_rng(5)
+    M, fl = 10, 262144
+    h = rng.uniform(-1.0, 1.0, (M, fl)).astype(np.float32)
+    # an all-zero token and one so small that max |h r| < 1e-5: both take the
+    # scale floor, s2 = 127 / 1e-5, as the whole layer's quantisation does
+    h[8] = 0.0
+    h[9] *= np.float32(1e-9)
+    codes = np.stack([np.ones(fl, np.int8), rng.integers(-1, 2, fl).astype(np.int8)])
+    Wd = oracle.pack(codes)
+    q2 = np.empty((M, fl), np.int8)
+    s2 = np.empty(M, np.float32)
+    moved = 0
+    for m in range(M):
+        r, hn = oracle.subln_rms(h[m])
+        xq, s, _ = oracle.quant_act(hn[None, :])
+        q2[m], s2[m] = xq[0], s[0]
+        other = np.clip(np.rint(h[m] * np.float32(r * s[0])), -128, 127).astype(np.int8)
+        moved += int(np.count_nonzero(other != q2[m]))
+    assert moved > 0
+    # ss in the order the whole layer sums it (sequential fp64 over j), hmax exact
+    ss = np.cumsum(h.astype(np.float64) ** 2, axis=1)[:, -1]
+    hmax = np.abs(h).max(axis=1)
+    acc, s2_tp = oracle.ffn_tp_down(Wd, h, ss, hmax, fl)
+    assert s2[8] == s2[9] == np.float32(127.0) / np.float32(1e-5)
+    assert np.array_equal(s2_tp, s2)
+    assert np.array_equal(acc, (q2.astype(np.int64) @ codes.T.astype(np.int64)).astype(np.int32))
