@@ -8,7 +8,7 @@ against it. A pin set is adequate when every mistake makes some pin fail. The
 repository's own oracle and tests are never modified.
 
 Two entries are equivalent mutants and are expected to survive: the lower clip of
-an int8 code at -128 never binds, because with s = 127 / max |x| every product
+an int8 code at -128 never binds: with s = 127 / max |x|, every product satisfies
 |x * s| <= 127 * (1 + 2^-24)^2 < 127.5, so rint gives codes in
 [-127, 127] (``test_quant_act_invariants`` checks that range).
 
