@@ -18,10 +18,12 @@
 // weight word and a word of plane i cover the same k.
 //
 // Work split: persistent CTAs walk units of 16 output rows x one K segment
-// (at most 2 KiB of each row); the 8 warps of a CTA split a unit in 64-byte column
-// chunks, partial sums meet in shared memory and the dequantisation epilogue is
-// fused. Before the dependency wait each CTA asks for its first tiles to be
-// prefetched into L2, so DRAM already streams while the previous kernel ends.
+// (at most 32 KiB of packed weights: 2 KiB of each row; a single token uses 8- or
+// 4-row units for long rows or few row tiles); the 8 warps of a CTA split a unit
+// in 64-byte column chunks, partial sums meet in shared memory and the
+// dequantisation epilogue is fused. Before the dependency wait each CTA asks for
+// its first tiles to be prefetched into L2, so DRAM already streams while the
+// previous kernel ends.
 //
 // Single token (DP): an 8-column MMA would spend 7 columns on padding, so each
 // thread instead owns 4 rows of the unit and every 64th packed word, and runs one
@@ -30,8 +32,11 @@
 //
 // Fused activation quantisation: when the codes of all M (<= 4) tokens fit in
 // shared memory, each CTA quantises x itself (absmax per token, then PLANES codes
-// into shared memory), so a forward call is one kernel. Otherwise the codes come
-// from the act-quant kernel through the workspace.
+// into shared memory), so a forward call is one kernel. Where x fits in the
+// threads' registers (one token; two or four tokens of short rows) it is read
+// once and quantised from registers after one barrier; otherwise a two-pass loop
+// reads it twice. Without fusion the codes come from the act-quant kernel
+// through the workspace.
 //
 // Extended calls (XT): row segments with their own gamma (stacked projections),
 // one gamma per row, and a unit-weight RMSNorm of x before the quantisation are
@@ -39,10 +44,13 @@
 // as before (its prologue runs once per launch from a cold instruction cache).
 //
 // Programmatic dependent launch: before waiting for the previous kernel in the
-// stream (griddepcontrol.wait) a CTA only issues L2 prefetches of its weights,
-// which cannot observe stale data (L2 is the point of coherence), and sets up its
-// barriers; the producer arms its first stage before it waits. Every global load
-// of other data and every store comes after the wait.
+// stream (griddepcontrol.wait) a CTA issues L2 prefetches of its weights, which
+// cannot observe stale data (L2 is the point of coherence), sets up its barriers,
+// and its producer copies the first kStages weight units into the ring. The
+// packed weights are read-only to every kernel of the library, so a kernel that
+// lets this one start early is not writing them; the public header states the
+// same condition for a caller's own kernels. Every global load of other data and
+// every store comes after the wait.
 #include "common.cuh"
 #include "kernels.h"
 #include "tc_ptx.cuh"
@@ -57,7 +65,7 @@ constexpr int kPrefetchAhead = 2;          // tiles of lookahead per CTA
 constexpr int kFusedSmemLimit = 48 * 1024;  // codes of all tokens in shared memory
 constexpr int kFusedMaxTokens = 4;          // beyond this the separate quantiser is faster
 constexpr int kStages = 2;                  // shared-memory ring of streamed weight units (2 CTAs per SM)
-constexpr int kMaxSegChunks = 32;           // at most 2 KiB of each row per unit
+constexpr int kMaxSegChunks = 32;           // 64-byte chunks of each row per 16-row unit (2 KiB)
 constexpr uint64_t kWaitLimitNs = 1000000000ull;
 constexpr size_t kMaxDynSmem = 200 * 1024;  // dynamic shared memory limit set on every instantiation
 
@@ -602,8 +610,8 @@ __device__ __forceinline__ void bulk_copy(uint32_t dst, const void* src, uint32_
         : "memory");
 }
 
-// The weight stream: a unit is one 16-row tile restricted to one K segment of
-// at most 32 chunks (2 KiB per row). The producer warp copies the unit's row
+// The weight stream: a unit is one tile of unit_rows rows restricted to one K
+// segment of at most 32 KiB (32 chunks of 64 bytes per row at 16 rows). The producer warp copies the unit's row
 // segments into a ring of kStages shared-memory stages; the row pitch is
 // congruent to 64 mod 128 bytes so rows g and g + 1 of a quarter-warp fall on
 // different banks.
