@@ -8,7 +8,10 @@
 //   hn = h * r                              unit RMSNorm weight, no bias
 //   q2, s2 = per-token absmax int8 quantisation of hn (as for x)
 //
-// One CTA per token; h is kept in shared memory between the passes.
+// Separate gate and up projections (ffn_finalise_kernel): one CTA per token, h
+// kept in shared memory between its passes. After the fused gate+up GEMM (more
+// than 16 tokens), whose epilogue writes h and per-tile partials of sum h^2 and
+// max |h|, ffn_requant_parts_kernel reduces the partials and requantises.
 //
 // Tensor-parallel pieces (a rank owns fl of the f hidden columns; the pages give
 // no distributed detail, this is the library's split): h with the rank's share
@@ -128,12 +131,11 @@ __global__ void __launch_bounds__(kThreads) ffn_tp_hstats_kernel(const float* __
     }
 }
 
-// Requantisation of a rank's columns with the statistics of all ranks:
-// r = 1 / sqrtf(float(ss_all / f_total) + 1e-5), s2 = 127 / max(fl(hmax_all r), 1e-5)
-// (the largest |fl(h_j r)| of the whole row: rounding is monotonic and r > 0),
-// codes of fl(h_j r) in the consumer's layout, and their sum over the rank's columns.
-// Codes of token m's fl columns fl(h_j r) with scale s = 127 / max(fl(hmax r), 1e-5),
-// r = 1 / sqrtf(float(ss / f_total) + 1e-5), in LAYOUT; s2[m] and the codes' sum.
+// Requantisation of token m's fl columns from the statistics of the whole row
+// (ss = sum h^2 over all f_total columns, hmax = max |h|):
+// r = 1 / sqrtf(float(ss / f_total) + 1e-5), s2 = 127 / max(fl(hmax r), 1e-5)
+// (the largest |fl(h_j r)| of the row: rounding is monotonic and r > 0); writes the
+// codes of fl(h_j r) in LAYOUT, s2[m] and the codes' sum over the fl columns.
 template <int LAYOUT>
 __device__ __forceinline__ void requant_row(const float* __restrict__ h, int m, int fl, int64_t f_total, double ss,
                                             float hmax, int8_t* __restrict__ q2, float* __restrict__ s2,

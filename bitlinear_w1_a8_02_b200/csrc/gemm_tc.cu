@@ -4,15 +4,17 @@
 // Paper card "BitNet b1.58 2B4T Technical Report", "Method Adaptation": packed
 // int8 weights are loaded into on-chip memory and unpacked right before the
 // int8 matmul (pack-store-load-unpack-compute). On B200 this becomes:
-//   TMA:     packed weight tile [256 rows x 32 bytes] and activation-code tile
+//   TMA:     packed weight tile [BN rows x 32 bytes, BN = 256, or 128 / 64 when
+//            wider tiles cannot fill the SMs] and activation-code tile
 //            [128 tokens x 128 codes] -> shared memory (one mbarrier per stage);
 //   unpack:  four warps turn every packed 32-bit word into 16 code bytes
 //            (three shifts and four ANDs) and store them straight into the
 //            128-byte-swizzled K-major operand layout the tensor core reads;
 //   MMA:     one thread issues tcgen05.mma kind::i8 (A = codes s8, B = weight
-//            codes u8 in {0,1,2}) into a 128 x 256 int32 accumulator in TMEM;
-//   epilogue: the same four warps read TMEM (tcgen05.ld), subtract the code
-//            offset (sum_k xq), dequantise and store bf16 / fp32 / int32.
+//            codes u8 in {0,1,2}) into a 128 x BN int32 accumulator in TMEM;
+//   epilogue: four more warps read TMEM (tcgen05.ld), subtract the code offset
+//            (sum_k xq), dequantise and store bf16 / fp32 / int32, while the
+//            next tile accumulates into the second TMEM accumulator.
 // The activation codes are in the G16T layout (each 16-code group stored as a
 // transposed 4x4 byte block), which is exactly the order a packed word unpacks
 // into, so no byte shuffling is needed anywhere.
