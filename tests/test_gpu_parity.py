@@ -602,6 +602,32 @@ def test_forward_single_token_long_rows(cuda_device, K, N):
     check_forward_full(Wp, gamma, Wp_ref, g_ref, x, cuda_device, residual=res)
 
 
+@pytest.mark.parametrize("M", [1, 2])
+@pytest.mark.parametrize("norm", [False, True])
+def test_forward_ex_two_tokens_register_quantiser(cuda_device, M, norm):
+    """One or two tokens with 4096 < K <= 8192 on the extended calls: the
+    in-kernel quantiser that keeps both tokens' x in registers (two groups of 16
+    per thread), with and without the RMSNorm, for stacked segments with their own
+    gammas and for one gamma per row."""
+    K, rows = 6912, [1024, 256, 256]
+    Wp, gam, Wp_ref, g_ref = stacked(rows, K, 97, cuda_device)
+    x = synth.activations(M, K, seed=98 + M, outliers=True)
+    y, acc = bl.forward_ex(Wp, gam, rows, x.to(cuda_device), rmsnorm=norm, want_acc=True)
+    ref = oracle.forward_ex(Wp_ref, g_ref, rows, bits(x), rmsnorm=norm)
+    assert np.array_equal(np_(acc), ref["acc"]), "int32 accumulators"
+    assert_bf16_exact(bits(y), ref["y"])
+    if not norm:
+        W = make_weights(1000, K, 0.02, seed=99)
+        Wr, gr = bl.pack_weights_rowwise(W.to(cuda_device))
+        Wr_ref, gr_ref = oracle.pack_weights_rowwise(bits(W))
+        res = synth.activations(M, 1000, seed=100 + M, outliers=False)
+        y, acc = bl.forward_rowwise(Wr, gr, x.to(cuda_device), residual=res.to(cuda_device), want_acc=True)
+        ref = oracle.forward_rowwise(Wr_ref, gr_ref, bits(x), residual=bits(res))
+        assert np.array_equal(np_(acc), ref["acc"])
+        assert_bf16_exact(bits(y), ref["y"])
+    assert bl.get_device_error() == 0
+
+
 @pytest.mark.parametrize("K", [12288, 28672])
 def test_forward_ex_single_token_long_rows_rmsnorm(cuda_device, K):
     rows = [256, 64, 64]
