@@ -464,6 +464,27 @@ def test_ffn_small_ragged(cuda_device):
     assert_bf16_exact(bits(y), ref["y"])
 
 
+@pytest.mark.parametrize("M,d,f", [(1, 6912, 2560), (1, 12288, 1024), (1, 2560, 12288), (2, 6912, 2560),
+                                   (3, 6912, 2560), (4, 8192, 1024)])
+def test_ffn_fused_prologue_routes(cuda_device, M, d, f):
+    """The two-kernel FFN (up to 4 tokens) with each of its quantiser forms:
+    gate+up with 2 and 8 register groups for one token (d = 6912, 12288), with two
+    groups for two tokens (d = 6912), and the two-pass loop for three and four
+    tokens with d > 4096; the down projection's one-token form for f <= 8192 and
+    its two-pass loop beyond (f = 12288)."""
+    Wg, Wu, Wd = (make_weights(f, d, 0.02, 7100 + d), make_weights(f, d, 0.02, 7200 + d),
+                  make_weights(d, f, 0.02, 7300 + f))
+    P = [pack_both(W, cuda_device) for W in (Wg, Wu, Wd)]
+    x = synth.activations(M, d, seed=7400 + M, outliers=True)
+    res = synth.activations(M, d, seed=7500 + M, outliers=False)
+    y = bl.ffn(P[0][0], P[0][1], P[1][0], P[1][1], P[2][0], P[2][1], x.to(cuda_device),
+               residual=res.to(cuda_device))
+    ref = oracle.ffn_layer(P[0][2], P[0][3], P[1][2], P[1][3], P[2][2], P[2][3], bits(x), residual=bits(res))
+    assert_bf16_close(bits(y), ref["y"])
+    assert_bf16_exact(bits(y), ref["y"])
+    assert bl.get_device_error() == 0
+
+
 # ----------------------------------------------------------------------------- tensor-core GEMV (M <= 16)
 
 @pytest.mark.parametrize("M", [1, 3, 8, 9, 16])
