@@ -196,7 +196,7 @@ bl_status bitlinear_forward_rowwise(const uint8_t* Wp, const float* gammas, int6
  * digest, BitLinear list). The query, key and value projections read the same
  * normalised x; the output projection reads the subln-normalised attention
  * output and adds the residual.
- *   y[m, n] = [residual[m, n] +] bf16(acc[m, n] * gammas[seg(n)] / s_m)
+ *   y[m, n] = bf16([residual[m, n] +] float(acc[m, n]) * (gammas[seg(n)] / s_m))
  *   xq, s   = quant(rmsnorm ? x * r : x),  r = 1 / sqrtf(float(sum_k x^2 / K) + 1e-5)
  *             per token (sum in fp64; x * r kept in fp32 and quantised as in
  *             bitlinear_forward)
@@ -263,9 +263,8 @@ bl_status bitlinear_ffn(const uint8_t* Wg, const float* gg, const uint8_t* Wu, c
  *          K <= 28672). Larger sizes return BL_ERR_WORKSPACE and launch nothing.
  *   No call allocates device memory or calls an allocating library routine.
  *   The first call on each device looks up the array's device address
- *   (cudaGetSymbolAddress); make that first call before any stream capture.
- *   After a cudaDeviceReset the next call on that device looks it up again
- *   (the same rule applies to that call).
+ *   (cudaGetSymbolAddress). After a cudaDeviceReset the next call on that
+ *   device looks it up again.
  *   Every call on a device shares the one array, which keeps the last call's
  *   contents (nothing in it needs to start at zero). Calls that can overlap on
  *   the GPU (other streams, unordered host threads) race on it: order them.
