@@ -178,6 +178,62 @@ def test_host_validation_rowwise():
     assert F(P(A), P(A), 512, 256, P(A), 1, None, P(A), None, P(A), need - 1, None) == WS
 
 
+def test_host_validation_tensor_parallel():
+    """The five tensor-parallel calls reject bad dtypes, shapes, pointers,
+    alignments and workspaces on the host, and treat M = 0 as a no-op."""
+    L = bl.lib()
+    need = L.bitlinear_workspace_bytes(bl.BL_OP_PACK, 0, 8, 16)
+    asum = L.bitlinear_absmean_sum
+    assert asum(P(A), 7, 8, 16, P(A), P(A), need, None) == DTYPE
+    assert asum(P(A), bl.BL_BF16, 0, 16, P(A), P(A), need, None) == SHAPE
+    assert asum(P(A), bl.BL_BF16, 8, 18, P(A), P(A), need, None) == SHAPE
+    assert asum(P(A), bl.BL_BF16, 8, 16, None, P(A), need, None) == NULL
+    assert asum(P(A), bl.BL_BF16, 8, 16, P(A + 4), P(A), need, None) == ALIGN
+    assert asum(P(A), bl.BL_BF16, 8, 16, P(A), P(A), need - 1, None) == WS
+
+    glob = L.bitlinear_pack_weights_global
+    assert glob(P(A), 7, 8, 16, P(A), 256, P(A), P(A), None) == DTYPE
+    assert glob(P(A), bl.BL_BF16, 8, 16, P(A), 127, P(A), P(A), None) == SHAPE  # count below N * K
+    assert glob(P(A), bl.BL_BF16, 8, 16, None, 256, P(A), P(A), None) == NULL
+    assert glob(P(A), bl.BL_BF16, 8, 16, P(A + 4), 256, P(A), P(A), None) == ALIGN
+
+    up = L.bitlinear_ffn_tp_up
+    need = L.bitlinear_workspace_bytes(bl.BL_OP_FFN_TP_UP, 2, 256, 64)
+    w4 = [P(A)] * 4
+
+    def call_up(d=64, fl=256, M=2, h=A, ss=A, ws=A, wsb=need):
+        return up(*w4, d, fl, P(A), M, P(h), P(ss), P(A), P(ws), wsb, None)
+
+    assert call_up(d=66) == SHAPE
+    assert call_up(fl=2) == SHAPE
+    assert call_up(M=-1) == SHAPE
+    assert call_up(M=0) == OK
+    assert call_up(h=None) == NULL
+    assert call_up(ss=A + 4) == ALIGN
+    assert call_up(ws=A + 16) == ALIGN
+    assert call_up(wsb=need - 1) == WS
+
+    down = L.bitlinear_ffn_tp_down
+    need = L.bitlinear_workspace_bytes(bl.BL_OP_FFN_TP_DOWN, 2, 64, 256)
+
+    def call_down(d=64, fl=256, f_total=512, M=2, ss=A, acc=A, wsb=need):
+        return down(P(A), d, fl, f_total, P(A), M, P(ss), P(A), P(acc), P(A), P(A), wsb, None)
+
+    assert call_down(f_total=200) == SHAPE   # the whole width below the rank's share
+    assert call_down(fl=258) == SHAPE
+    assert call_down(d=0) == SHAPE
+    assert call_down(M=0) == OK
+    assert call_down(acc=None) == NULL
+    assert call_down(ss=A + 4) == ALIGN
+    assert call_down(wsb=need - 1) == WS
+
+    fin = L.bitlinear_ffn_tp_finish
+    assert fin(P(A), P(A), P(A), None, P(A), -1, 64, None) == SHAPE
+    assert fin(P(A), P(A), P(A), None, P(A), 0, 64, None) == OK
+    assert fin(P(A), None, P(A), None, P(A), 2, 64, None) == NULL
+    assert fin(P(A), P(A), P(A), P(A + 1), P(A), 2, 64, None) == ALIGN
+
+
 def test_host_validation_selftest():
     L = bl.lib()
     assert L.bitlinear_selftest_timeout(0, None) == SHAPE
