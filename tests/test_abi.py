@@ -234,6 +234,29 @@ def test_host_validation_tensor_parallel():
     assert fin(P(A), P(A), P(A), P(A + 1), P(A), 2, 64, None) == ALIGN
 
 
+def test_host_validation_noalloc():
+    """The allocation-free forward checks its arguments like bitlinear_forward, and
+    refuses sizes whose codes and per-token words would not fit its fixed 1 MiB
+    scratch, before touching a device."""
+    F = bl.lib().bitlinear_forward_noalloc
+
+    def call(N=512, K=256, M=1, g=A, x=A, y=A, res=None, acc=None):
+        return F(P(A), P(g), N, K, P(x), M, P(res), P(y), P(acc), None)
+
+    assert call(K=258) == SHAPE
+    assert call(M=-1) == SHAPE
+    assert call(N=-1) == SHAPE
+    assert call(M=0) == OK
+    assert call(N=0) == OK
+    assert call(x=None) == NULL
+    assert call(g=None) == NULL
+    assert call(g=A + 2) == ALIGN
+    assert call(y=A + 1) == ALIGN
+    assert call(res=A + 1) == ALIGN
+    assert call(acc=A + 2) == ALIGN
+    assert call(M=64, K=32768) == WS      # 2 MiB of codes
+
+
 def test_host_validation_selftest():
     L = bl.lib()
     assert L.bitlinear_selftest_timeout(0, None) == SHAPE
@@ -245,6 +268,8 @@ def test_valid_call_without_device_is_unsupported():
     L = bl.lib()
     need = L.bitlinear_workspace_bytes(bl.BL_OP_FORWARD, 1, 512, 256)
     st = L.bitlinear_forward(P(A), P(A), 512, 256, P(A), 1, None, P(A), None, P(A), need, None)
+    assert st == UNSUP
+    st = L.bitlinear_forward_noalloc(P(A), P(A), 512, 256, P(A), 1, None, P(A), None, None)
     assert st == UNSUP
     assert L.bitlinear_get_device_error(None) == UNSUP
 
